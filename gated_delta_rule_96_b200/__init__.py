@@ -1,0 +1,189 @@
+"""Python binding of libgdn2 (Gated DeltaNet-2 recurrence on B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels
+behind the C ABI declared in ``include/gdn2.h``.  PyTorch supplies device memory and
+streams.  There is no CPU fallback: if ``libgdn2.so`` is missing or no CUDA device
+is present the calls raise.
+
+The operation (page "NVIDIA представила Gated DeltaNet-2 ...", section
+"Техническая схема"):  S_t = (I - k_t (b_t ⊙ k_t)^T) Diag(alpha_t) S_{t-1}
++ k_t (w_t ⊙ v_t)^T,  o_t = S_t^T q_t.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GDN2Error", "load_library", "library_path", "gdn2_chunk_fwd", "gdn2_decode_step",
+    "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
+    "chunk_fwd", "decode_step", "new_workspace",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libgdn2.so"
+_lib = None
+
+GDN2_F32, GDN2_BF16 = 0, 1
+STATUS_HEADER_BYTES = 256
+
+
+class GDN2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({gdn2_status_str(status)})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load_library():
+    """Load the in-tree libgdn2.so (built by __graft_entry__.build() / build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run `python -c 'import __graft_entry__ as g; g.build()'` "
+                           "(the CUDA library is required: there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.gdn2_chunk_fwd_workspace_bytes.argtypes = [i] * 7
+    lib.gdn2_chunk_fwd_workspace_bytes.restype = sz
+    lib.gdn2_chunk_fwd_path.argtypes = [i] * 7
+    lib.gdn2_chunk_fwd_path.restype = i
+    lib.gdn2_chunk_fwd.argtypes = [vp] * 9 + [i] * 7 + [vp, sz, vp]
+    lib.gdn2_chunk_fwd.restype = i
+    lib.gdn2_decode_step.argtypes = [vp] * 8 + [i] * 5 + [vp]
+    lib.gdn2_decode_step.restype = i
+    lib.gdn2_workspace_status.argtypes = [vp, i, ctypes.POINTER(i), vp]
+    lib.gdn2_workspace_status.restype = i
+    lib.gdn2_status_str.argtypes = [i]
+    lib.gdn2_status_str.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def gdn2_status_str(status: int) -> str:
+    return load_library().gdn2_status_str(int(status)).decode()
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GDN2_BF16
+    if t.dtype == torch.float32:
+        return GDN2_F32
+    raise TypeError(f"token tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+def gdn2_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, C=64, dtype=GDN2_BF16) -> int:
+    return int(load_library().gdn2_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, C, int(dtype)))
+
+
+def gdn2_chunk_fwd_path(B, H, T, d_k, d_v, C=64, dtype=GDN2_BF16) -> int:
+    return int(load_library().gdn2_chunk_fwd_path(B, H, T, d_k, d_v, C, int(dtype)))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def new_workspace(nbytes: int, device=None):
+    """Workspace tensor with its status header zeroed."""
+    import torch
+    ws = torch.empty(max(int(nbytes), STATUS_HEADER_BYTES), dtype=torch.uint8, device=device or "cuda")
+    ws[:STATUS_HEADER_BYTES].zero_()
+    return ws
+
+
+def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, C=64, workspace=None, stream=None) -> None:
+    """Prefill through the C ABI.  Shapes: q,k,b,alpha [B,T,H,d_k]; v,w,o [B,T,H,d_v];
+    S0 (or None), S_T [B,H,d_k,d_v] fp32.  Raises GDN2Error on a nonzero status."""
+    import torch
+    _check_cuda(q, k, v, alpha, b, w, S0, o, S_T, workspace)
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    dt = _dtype_code(q)
+    if alpha.dtype != torch.float32 or S_T.dtype != torch.float32 or (S0 is not None and S0.dtype != torch.float32):
+        raise TypeError("alpha and the states must be float32")
+    for name, t in (("k", k), ("b", b), ("v", v), ("w", w), ("o", o)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must have the dtype of q ({q.dtype})")
+    for name, t, shp in (("k", k, (B, T, H, K)), ("b", b, (B, T, H, K)), ("alpha", alpha, (B, T, H, K)),
+                         ("w", w, (B, T, H, V)), ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)),
+                         ("S0", S0, (B, H, K, V))):
+        if t is not None and tuple(t.shape) != shp:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    need = gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, C, dt)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = load_library().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                       _ptr(o), _ptr(S_T), B, H, T, K, V, C, dt, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_chunk_fwd")
+
+
+def gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=None) -> None:
+    """One decode token: q,k,b,alpha [B,H,d_k]; v,w,o [B,H,d_v]; S [B,H,d_k,d_v] fp32 in place."""
+    import torch
+    _check_cuda(q, k, v, alpha, b, w, S, o)
+    B, H, K = q.shape
+    V = v.shape[-1]
+    dt = _dtype_code(q)
+    if alpha.dtype != torch.float32 or S.dtype != torch.float32:
+        raise TypeError("alpha and S must be float32")
+    if tuple(S.shape) != (B, H, K, V) or tuple(o.shape) != (B, H, V):
+        raise ValueError("S must be [B,H,d_k,d_v] and o [B,H,d_v]")
+    rc = load_library().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S),
+                                         _ptr(o), B, H, K, V, dt, _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_decode_step")
+
+
+def gdn2_workspace_status(workspace, clear=False, stream=None) -> int:
+    out = ctypes.c_int(0)
+    rc = load_library().gdn2_workspace_status(_ptr(workspace), 1 if clear else 0, ctypes.byref(out),
+                                              _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_workspace_status")
+    return out.value
+
+
+def chunk_fwd(q, k, v, alpha, b, w, S0=None, C=64, workspace=None, stream=None):
+    """Allocating convenience wrapper: returns (o, S_T)."""
+    import torch
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    o = torch.empty((B, T, H, V), dtype=q.dtype, device=q.device)
+    S_T = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device)
+    gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, C=C, workspace=workspace, stream=stream)
+    return o, S_T
+
+
+def decode_step(q, k, v, alpha, b, w, S, stream=None):
+    """Allocating convenience wrapper: updates S in place, returns o."""
+    import torch
+    B, H, K = q.shape
+    o = torch.empty((B, H, v.shape[-1]), dtype=q.dtype, device=q.device)
+    gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=stream)
+    return o

@@ -1,0 +1,121 @@
+// extern "C" boundary of libgdn2: argument checking, path selection, launches.
+// Declarations and the meaning of every argument: include/gdn2.h.
+#include <stdint.h>
+
+#include "gdn2.h"
+#include "gdn2_internal.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dim_ok(int d) { return d == 64 || d == 128; }
+
+int check_common(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                 const void *o, int B, int H, int K, int V, int dtype) {
+    if (B < 0 || H < 0 || K <= 0 || V <= 0) return GDN2_ERR_SHAPE;
+    if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (!dim_ok(K) || !dim_ok(V)) return GDN2_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !b || !w || !o) return GDN2_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(b) || !aligned16(w) ||
+        !aligned16(o))
+        return GDN2_ERR_ALIGN;
+    return GDN2_OK;
+}
+
+bool use_tc(int B, int H, int T, int K, int V, int C, int dtype) {
+    return gdn2::tc_supported(B, H, T, K, V, C, dtype == GDN2_BF16 ? 1 : 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn2_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C, int dtype) {
+    if (B < 0 || H < 0 || T < 0 || !dim_ok(d_k) || !dim_ok(d_v) || C != 64) return gdn2::kStatusBytes;
+    if (use_tc(B, H, T, d_k, d_v, C, dtype)) return gdn2::tc_workspace_bytes(B, H, T, d_k, d_v, C);
+    return gdn2::simt_workspace_bytes(B, H, T, d_k, d_v, C);
+}
+
+int gdn2_chunk_fwd_path(int B, int H, int T, int d_k, int d_v, int C, int dtype) {
+    return use_tc(B, H, T, d_k, d_v, C, dtype) ? 1 : 0;
+}
+
+int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                   const float *S0, void *o, float *S_T, int B, int H, int T, int d_k, int d_v, int C, int dtype,
+                   void *workspace, size_t workspace_bytes, void *stream) {
+    if (T < 0) return GDN2_ERR_SHAPE;
+    int rc;
+    if (T == 0) {
+        // no tokens: token and output pointers are not read (empty tensors may be NULL)
+        if (B < 0 || H < 0) return GDN2_ERR_SHAPE;
+        if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
+        if (!dim_ok(d_k) || !dim_ok(d_v)) return GDN2_ERR_UNSUPPORTED;
+    } else {
+        rc = check_common(q, k, v, alpha, b, w, o, B, H, d_k, d_v, dtype);
+        if (rc != GDN2_OK) return rc;
+    }
+    if (C != 64) return GDN2_ERR_UNSUPPORTED;
+    if (!S_T) return GDN2_ERR_NULL;
+    if (!aligned16(S_T) || (S0 && !aligned16(S0))) return GDN2_ERR_ALIGN;
+    if (!workspace) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    if (workspace_bytes < gdn2_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, C, dtype)) return GDN2_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (B == 0 || H == 0) return GDN2_OK;
+    const size_t state_bytes = sizeof(float) * (size_t)B * H * d_k * d_v;
+    if (T == 0) {
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, st))
+                           : cudaMemsetAsync(S_T, 0, state_bytes, st);
+        return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+    }
+    const int bf16 = dtype == GDN2_BF16 ? 1 : 0;
+    if (use_tc(B, H, T, d_k, d_v, C, dtype))
+        rc = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, B, H, T, d_k, d_v, C, workspace, st);
+    else
+        rc = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, B, H, T, d_k, d_v, C, bf16, workspace, st);
+    return rc;
+}
+
+int gdn2_decode_step(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                     float *S, void *o, int B, int H, int d_k, int d_v, int dtype, void *stream) {
+    int rc = check_common(q, k, v, alpha, b, w, o, B, H, d_k, d_v, dtype);
+    if (rc != GDN2_OK) return rc;
+    if (!S) return GDN2_ERR_NULL;
+    if (!aligned16(S)) return GDN2_ERR_ALIGN;
+    if (B == 0 || H == 0) return GDN2_OK;
+    return gdn2::launch_decode(q, k, v, alpha, b, w, S, o, B, H, d_k, d_v, dtype == GDN2_BF16 ? 1 : 0,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gdn2_workspace_status(void *workspace, int clear, int *out, void *stream) {
+    if (!workspace || !out) return GDN2_ERR_NULL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GDN2_ERR_CUDA;
+    *out = (int)word;
+    if (clear && word) {
+        if (cudaMemsetAsync(workspace, 0, gdn2::kStatusBytes, st) != cudaSuccess) return GDN2_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return GDN2_ERR_CUDA;
+    }
+    return GDN2_OK;
+}
+
+const char *gdn2_status_str(int status) {
+    switch (status) {
+        case GDN2_OK: return "ok";
+        case GDN2_ERR_NULL: return "a required pointer is NULL";
+        case GDN2_ERR_SHAPE: return "a size is negative or inconsistent";
+        case GDN2_ERR_DTYPE: return "unknown dtype code";
+        case GDN2_ERR_UNSUPPORTED: return "unsupported size (d_k and d_v must be 64 or 128, C must be 64)";
+        case GDN2_ERR_WORKSPACE: return "workspace missing or too small";
+        case GDN2_ERR_CUDA: return "CUDA runtime or launch error";
+        case GDN2_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case GDN2_ERR_DEVICE: return "a kernel reported an internal error";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

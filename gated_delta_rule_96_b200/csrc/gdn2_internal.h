@@ -1,0 +1,29 @@
+// Host-side launchers shared between the ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdn2 {
+
+// Status header at the start of every prefill workspace (device status words).
+constexpr size_t kStatusBytes = 256;
+
+// Decode: one token per (b, h); S updated in place.
+int launch_decode(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                  const void *w, float *S, void *o, int B, int H, int K, int V, int bf16, cudaStream_t st);
+
+// SIMT two-kernel prefill (fp32 FMA everywhere; any token dtype).
+size_t simt_workspace_bytes(int B, int H, int T, int K, int V, int C);
+int launch_chunk_simt(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                      const void *w, const float *S0, void *o, float *ST, int B, int H, int T, int K, int V,
+                      int C, int bf16, void *ws, cudaStream_t st);
+
+// Fused tcgen05 prefill (bf16 tokens, d_k = d_v = 128, C = 64).
+bool tc_supported(int B, int H, int T, int K, int V, int C, int bf16);
+size_t tc_workspace_bytes(int B, int H, int T, int K, int V, int C);
+int launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                    const void *w, const float *S0, void *o, float *ST, int B, int H, int T, int K, int V,
+                    int C, void *ws, cudaStream_t st);
+
+}  // namespace gdn2

@@ -1,0 +1,116 @@
+/*
+ * gdn2.h -- C ABI of the Gated DeltaNet-2 recurrence library (libgdn2.so), sm_100a.
+ *
+ * The operation (page "NVIDIA представила Gated DeltaNet-2 с канал-wise гейтами ...",
+ * section "Техническая схема", the state-update equation), per batch element and head:
+ *
+ *     S_t = (I - k_t (b_t ⊙ k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t ⊙ v_t)^T
+ *     o_t = S_t^T q_t
+ *
+ * S in R^{d_k x d_v} (fp32).  b_t in [0,1]^{d_k} is the erase gate on the key axis,
+ * w_t in [0,1]^{d_v} the write gate on the value axis, alpha_t in (0,1]^{d_k} the
+ * channel-wise decay.  The read-out uses the post-update state and no 1/sqrt(d_k)
+ * scale.  Collapsing b and w to one scalar per token gives KDA; collapsing alpha to a
+ * scalar as well gives Gated DeltaNet (page "NVIDIA улучшила память LLM ...", the
+ * quoted remark on special cases): pass such gates as broadcast (materialised) tensors.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers to contiguous, row-major buffers, each
+ *     16-byte aligned.  The caller owns every buffer; the library allocates nothing
+ *     and keeps no state between calls.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream).  The return value reports argument checking and launch
+ *     errors only; device-side errors are read with gdn2_workspace_status().
+ *   - Nothing throws across the ABI.  Every entry point returns a gdn2_status.
+ *   - d_k, d_v in {64, 128}.  Token dtype (q, k, v, b, w and o) is fp32 or bf16;
+ *     alpha and the states are always fp32.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN2_OK = 0,
+    GDN2_ERR_NULL = -1,         /* a required pointer is NULL                        */
+    GDN2_ERR_SHAPE = -2,        /* a size is negative or inconsistent                */
+    GDN2_ERR_DTYPE = -3,        /* unknown dtype code                                */
+    GDN2_ERR_UNSUPPORTED = -4,  /* valid but unsupported (d_k/d_v not 64/128, C!=64) */
+    GDN2_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than required           */
+    GDN2_ERR_CUDA = -6,         /* a CUDA runtime call or kernel launch failed       */
+    GDN2_ERR_ALIGN = -7,        /* a pointer is not 16-byte aligned                  */
+    GDN2_ERR_DEVICE = -8        /* a kernel reported an internal error (bounded wait
+                                   expired); read by gdn2_workspace_status           */
+} gdn2_status;
+
+typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
+
+/* Bytes of device workspace gdn2_chunk_fwd needs for these sizes (0 on bad sizes is
+ * never returned: at least the 256-byte status header is always required).
+ * Depends only on its arguments. */
+GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C, int dtype);
+
+/*
+ * Chunkwise-parallel prefill over T tokens (page "NVIDIA представила Gated DeltaNet-2 ...",
+ * the paragraph on the chunkwise WY form with chunk size C = 64).
+ *
+ *   q, k, b       [B, T, H, d_k]   token dtype
+ *   v, w          [B, T, H, d_v]   token dtype
+ *   alpha         [B, T, H, d_k]   fp32, each value in (0, 1]
+ *   S0            [B, H, d_k, d_v] fp32 initial state, or NULL for a zero state
+ *   o   (out)     [B, T, H, d_v]   token dtype
+ *   S_T (out)     [B, H, d_k, d_v] fp32 final state; may alias S0 (in-place resume)
+ *   C             chunk size; must be 64
+ *   workspace     device scratch of at least gdn2_chunk_fwd_workspace_bytes(...) bytes,
+ *                 16-byte aligned; its first 256 bytes hold the device status words
+ *                 (see gdn2_workspace_status) and must have been zeroed once by the
+ *                 caller before first use (cudaMemset), after which calls keep them.
+ *   T = 0 copies S0 (or zeros) to S_T; the token and o pointers are then not read and
+ *   may be NULL.  A last partial chunk (T % C != 0) is handled.
+ */
+GDN2_API int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                   const void *w, const float *S0, void *o, float *S_T, int B, int H, int T, int d_k,
+                   int d_v, int C, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode token per sequence, state updated in place (constant memory per token,
+ * page "NVIDIA улучшила память LLM ...", section "Контекст").
+ *
+ *   q, k, b       [B, H, d_k]      token dtype
+ *   v, w          [B, H, d_v]      token dtype
+ *   alpha         [B, H, d_k]      fp32
+ *   S   (in/out)  [B, H, d_k, d_v] fp32, read and overwritten
+ *   o   (out)     [B, H, d_v]      token dtype
+ */
+GDN2_API int gdn2_decode_step(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                     const void *w, float *S, void *o, int B, int H, int d_k, int d_v, int dtype,
+                     void *stream);
+
+/* Reads the device status word of a workspace (synchronises `stream` first).
+ * *out receives 0 when every kernel that used this workspace finished normally, or a
+ * nonzero code naming the first internal error.  With clear != 0 the word is reset.
+ * Returns GDN2_OK, or GDN2_ERR_NULL / GDN2_ERR_CUDA. */
+GDN2_API int gdn2_workspace_status(void *workspace, int clear, int *out, void *stream);
+
+/* Static description of a status code (never NULL). */
+GDN2_API const char *gdn2_status_str(int status);
+
+/* Which prefill implementation gdn2_chunk_fwd selects for these sizes:
+ * 0 = SIMT two-kernel path (fp32 FMA), 1 = fused tcgen05 tensor-core path. */
+GDN2_API int gdn2_chunk_fwd_path(int B, int H, int T, int d_k, int d_v, int C, int dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */

@@ -18,8 +18,10 @@ Recipe (one place, used everywhere):
   beta = sigmoid(N(0,1)) per (token, head) broadcast over the channels
   ("kda"); "gdn" additionally draws alpha once per (token, head);
 * S0: N(0, s0_std^2) or absent (zero state);
-* values are drawn in fp64 and rounded to the storage dtype (fp64 -> fp32
-  -> bf16, each round-to-nearest-even); the oracle is fed the rounded values.
+* values are drawn and shaped in fp64 (in synth_gen.c) and rounded to the
+  storage dtype (fp64 -> fp32 -> bf16, each round-to-nearest-even); arrays are
+  returned as float32 holding exactly the stored values, and the oracle is fed
+  those values widened to fp64.
 
 Token tensors are [B, T, H, d] (d fastest); states are [B, H, d_k, d_v].
 Decode tokens are [B, H, d]; decode step s uses streams 16*(s+1) + id.
@@ -59,6 +61,10 @@ def _load():
         lib.synth_uniform.argtypes = [u64, u64, u64, sz, dp]
         lib.synth_normal_mt.argtypes = [u64, u64, u64, sz, dp, ctypes.c_int]
         lib.synth_normal_rows.argtypes = [u64, u64, ctypes.POINTER(ctypes.c_uint64), sz, sz, dp]
+        lib.synth_rows.argtypes = [u64, u64, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                   ctypes.POINTER(ctypes.c_uint64), u64, sz, sz, ctypes.c_int, ctypes.c_int,
+                                   ctypes.POINTER(ctypes.c_float), ctypes.c_int]
+        lib.synth_rows.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -96,21 +102,32 @@ def normal_rows(seed: int, stream: int, offsets: np.ndarray, rowlen: int) -> np.
 
 # ----------------------------------------------------------------------------- shaping
 
-def softplus(x):
-    return np.logaddexp(0.0, x)
+KIND_NORMAL, KIND_L2, KIND_SIGMOID, KIND_DECAY = 0, 1, 2, 3
 
 
-def sigmoid(x):
-    return 1.0 / (1.0 + np.exp(-x))
-
-
-def l2_normalise(x):
-    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
-    return x / np.maximum(n, 1e-300)
+def rows(seed: int, stream: int, kind: int, d: int, row_index=None, nrows: int | None = None, row0: int = 0,
+         mu: float = 0.0, scale: float = 1.0, per_token: bool = False, bf16: bool = False,
+         threads: int | None = None) -> np.ndarray:
+    """Shaped rows ([nrows, d] float32); see synth_rows in synth_gen.c."""
+    lib = _load()
+    if row_index is not None:
+        idx = np.ascontiguousarray(row_index, dtype=np.uint64)
+        n = idx.size
+        iptr = idx.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64))
+    else:
+        idx, n, iptr = None, int(nrows), None
+    out = np.empty((n, d), dtype=np.float32)
+    if n:
+        nt = threads if threads is not None else min(os.cpu_count() or 1, 32)
+        rc = lib.synth_rows(seed, stream, kind, mu, scale, iptr, row0, n, d, 1 if per_token else 0,
+                            1 if bf16 else 0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), nt)
+        if rc != 0:
+            raise ValueError("synth_rows rejected its arguments")
+    return out
 
 
 def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
-    """Round fp64 values to the storage dtype; returned as fp64 (exactly representable)."""
+    """Round values to the storage dtype; returned as fp64 (exactly representable)."""
     if dtype == "f64":
         return np.asarray(x, dtype=np.float64)
     x32 = np.asarray(x, dtype=np.float32)
@@ -118,7 +135,6 @@ def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
         return x32.astype(np.float64)
     if dtype == "bf16":
         u = x32.view(np.uint32).astype(np.uint64)
-        # round-to-nearest-even on the top 16 bits (inputs here are finite)
         lsb = (u >> 16) & 1
         u = (u + 0x7FFF + lsb) & 0xFFFF0000
         return u.astype(np.uint32).view(np.float32).astype(np.float64)
@@ -142,8 +158,7 @@ class Workload:
     seed: int = 0x9D2
     steps: int = 0        # decode steps (decode workloads only)
     decode: bool = False
-    alpha_scale: float = 1.0  # multiplies softplus (stress variant uses 0.02)
-    extra: dict = field(default_factory=dict, compare=False)
+    alpha_scale: float = 1.0  # multiplies softplus (slow-decay stress variant uses 0.02)
 
 
 WORKLOADS = {
@@ -162,84 +177,76 @@ WORKLOADS = {
 }
 
 
-def _token_offsets(B, T, H, d, chains, t0, t1):
-    """Counter offsets of rows (b, t, h, :) for t in [t0, t1) of each chain (b, h)."""
-    rows = []
-    for (b, h) in chains:
-        t = np.arange(t0, t1, dtype=np.uint64)
-        rows.append(((np.uint64(b) * np.uint64(T) + t) * np.uint64(H) + np.uint64(h)) * np.uint64(d))
-    return np.concatenate(rows) if rows else np.zeros(0, dtype=np.uint64)
-
-
-def _draw_tokens(wl: Workload, name: str, d: int, chains, t0, t1, stream_base, T_full):
-    """Normals for token tensor `name` as [n_chains, t1-t0, d] (chain subset) or [B,T,H,d]."""
-    seed, st = wl.seed, stream_base + STREAM[name]
+def _row_index(wl: Workload, T_full: int, chains, t0: int, t1: int):
+    """Flat (b, t, h) row indices of the requested rows, or None for the full tensor."""
+    if chains is None and (t0, t1) == (0, T_full):
+        return None
     if chains is None:
-        x = normal(seed, st, wl.B * T_full * wl.H * d)
-        return x.reshape(wl.B, T_full, wl.H, d)
-    offs = _token_offsets(wl.B, T_full, wl.H, d, chains, t0, t1)
-    return normal_rows(seed, st, offs, d).reshape(len(chains), t1 - t0, d)
-
-
-def _draw_per_token(wl: Workload, name: str, chains, t0, t1, stream_base, T_full):
-    """One normal per (b, t, h): returned as [..., 1] to broadcast over channels."""
-    seed, st = wl.seed, stream_base + STREAM[name]
-    if chains is None:
-        x = normal(seed, st, wl.B * T_full * wl.H)
-        return x.reshape(wl.B, T_full, wl.H, 1)
-    offs = _token_offsets(wl.B, T_full, wl.H, 1, chains, t0, t1)
-    return normal_rows(seed, st, offs, 1).reshape(len(chains), t1 - t0, 1)
+        chains = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    t = np.arange(t0, t1, dtype=np.uint64)
+    parts = [(np.uint64(b) * np.uint64(T_full) + t) * np.uint64(wl.H) + np.uint64(h) for (b, h) in chains]
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.uint64)
 
 
 def make_inputs(wl: Workload, chains=None, t_range=None, step: int | None = None):
-    """Inputs of a workload, rounded to their storage dtypes, as fp64 numpy arrays.
+    """Inputs of a workload as float32 arrays holding exactly the stored values.
 
-    chains=None gives full tensors ([B,T,H,d] tokens, [B,H,K,V] state); a list of
-    (b, h) gives the same values for just those chains ([n, T, d] tokens,
-    [n, K, V] state).  For decode workloads, `step` selects the token of that
-    step (T = 1) and S0 is the state before step 0.
+    chains=None gives full tensors ([B,T,H,d] tokens); a list of (b, h) gives the
+    same values for just those chains ([n, T, d]).  For decode workloads `step`
+    selects the token of that step and tokens drop the T axis ([B,H,d] / [n,d]).
     """
     T_full = 1 if wl.decode else wl.T
     t0, t1 = (0, T_full) if t_range is None else t_range
-    stream_base = 0 if step is None else 16 * (step + 1)
-    tok = wl.dtype
+    base = 0 if step is None else 16 * (step + 1)
+    idx = _row_index(wl, T_full, chains, t0, t1)
+    nrows = wl.B * T_full * wl.H if idx is None else idx.size
+    bf = wl.dtype == "bf16"
     K, V = wl.K, wl.V
-    out = {}
-    q = _draw_tokens(wl, "q", K, chains, t0, t1, stream_base, T_full)
-    out["q"] = round_to(l2_normalise(q), tok)
-    k = _draw_tokens(wl, "k", K, chains, t0, t1, stream_base, T_full)
-    out["k"] = round_to(l2_normalise(k), tok)
-    out["v"] = round_to(_draw_tokens(wl, "v", V, chains, t0, t1, stream_base, T_full), tok)
+
+    def tok(name, kind, d, bf16=bf, mu=0.0, scale=1.0, per_token=False, stream_name=None):
+        st = base + STREAM[stream_name or name]
+        return rows(wl.seed, st, kind, d, row_index=idx, nrows=nrows, mu=mu, scale=scale,
+                    per_token=per_token, bf16=bf16)
+
+    out = {
+        "q": tok("q", KIND_L2, K),
+        "k": tok("k", KIND_L2, K),
+        "v": tok("v", KIND_NORMAL, V),
+    }
     if wl.gates == "gdn":
-        a = _draw_per_token(wl, "alpha_s", chains, t0, t1, stream_base, T_full) + wl.alpha_mu
-        a = np.broadcast_to(np.exp(-wl.alpha_scale * softplus(a)), q.shape[:-1] + (K,))
+        out["alpha"] = tok("alpha", KIND_DECAY, K, bf16=False, mu=wl.alpha_mu, scale=wl.alpha_scale,
+                           per_token=True, stream_name="alpha_s")
     else:
-        a = _draw_tokens(wl, "alpha", K, chains, t0, t1, stream_base, T_full) + wl.alpha_mu
-        a = np.exp(-wl.alpha_scale * softplus(a))
-    out["alpha"] = round_to(np.ascontiguousarray(a), "f32")
+        out["alpha"] = tok("alpha", KIND_DECAY, K, bf16=False, mu=wl.alpha_mu, scale=wl.alpha_scale)
     if wl.gates in ("kda", "gdn"):
-        beta = sigmoid(_draw_per_token(wl, "beta", chains, t0, t1, stream_base, T_full))
-        out["b"] = round_to(np.ascontiguousarray(np.broadcast_to(beta, q.shape[:-1] + (K,))), tok)
-        out["w"] = round_to(np.ascontiguousarray(np.broadcast_to(beta, q.shape[:-1] + (V,))), tok)
+        out["b"] = tok("b", KIND_SIGMOID, K, per_token=True, stream_name="beta")
+        out["w"] = tok("w", KIND_SIGMOID, V, per_token=True, stream_name="beta")
     else:
-        out["b"] = round_to(sigmoid(_draw_tokens(wl, "b", K, chains, t0, t1, stream_base, T_full)), tok)
-        out["w"] = round_to(sigmoid(_draw_tokens(wl, "w", V, chains, t0, t1, stream_base, T_full)), tok)
-    if wl.decode:
-        # decode tokens drop the T axis: [B, H, d] (or [n, d] for a chain subset)
-        for key in ("q", "k", "v", "alpha", "b", "w"):
-            out[key] = out[key][:, 0] if chains is None else out[key][:, 0]
+        out["b"] = tok("b", KIND_SIGMOID, K)
+        out["w"] = tok("w", KIND_SIGMOID, V)
+    n_ch = None if chains is None else len(chains)
+    for key, a in out.items():
+        d = a.shape[1]
+        if wl.decode:
+            out[key] = a.reshape(wl.B, wl.H, d) if n_ch is None else a.reshape(n_ch, d)
+        else:
+            out[key] = a.reshape(wl.B, t1 - t0, wl.H, d) if n_ch is None else a.reshape(n_ch, t1 - t0, d)
     return out
 
 
 def make_state(wl: Workload, chains=None):
-    """Initial state S0 ([B,H,K,V] or [n,K,V]) rounded to fp32, or None for a zero state."""
+    """Initial state S0 ([B,H,K,V] or [n,K,V]) as float32, or None for a zero state."""
     if wl.s0_std is None:
         return None
     K, V = wl.K, wl.V
-    st = STREAM["S0"]
     if chains is None:
-        x = normal(wl.seed, st, wl.B * wl.H * K * V).reshape(wl.B, wl.H, K, V)
-    else:
-        offs = np.array([((b * wl.H + h) * K * V) for (b, h) in chains], dtype=np.uint64)
-        x = normal_rows(wl.seed, st, offs, K * V).reshape(len(chains), K, V)
-    return round_to(wl.s0_std * x, "f32")
+        x = rows(wl.seed, STREAM["S0"], KIND_NORMAL, K * V, nrows=wl.B * wl.H, scale=wl.s0_std)
+        return x.reshape(wl.B, wl.H, K, V)
+    idx = np.array([b * wl.H + h for (b, h) in chains], dtype=np.uint64)
+    x = rows(wl.seed, STREAM["S0"], KIND_NORMAL, K * V, row_index=idx, scale=wl.s0_std)
+    return x.reshape(len(chains), K, V)
+
+
+def as_f64(d: dict) -> dict:
+    """fp64 copies (for the oracle) of a dict of float32 input arrays."""
+    return {k: (None if v is None else np.asarray(v, dtype=np.float64)) for k, v in d.items()}

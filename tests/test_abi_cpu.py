@@ -1,0 +1,107 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_96_b200 as g
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn2.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN2_API\s+[\w\s\*]+?\b(gdn2_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return g.load_library()
+
+
+def test_header_declares_entry_points():
+    syms = declared_symbols()
+    for name in ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_fwd_workspace_bytes", "gdn2_status_str",
+                 "gdn2_workspace_status", "gdn2_chunk_fwd_path"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in gdn2.h but not exported"
+
+
+def test_status_strings(lib):
+    for code in range(-8, 1):
+        assert g.gdn2_status_str(code)
+    assert g.gdn2_status_str(0) == "ok"
+    assert g.gdn2_status_str(12345) == "unknown status"
+
+
+def test_workspace_bytes():
+    # the status header is always required
+    assert g.gdn2_chunk_fwd_workspace_bytes(0, 0, 0, 128, 128) >= 256
+    n1 = g.gdn2_chunk_fwd_workspace_bytes(1, 1, 64, 128, 128, 64, g.GDN2_F32)
+    n2 = g.gdn2_chunk_fwd_workspace_bytes(1, 1, 128, 128, 128, 64, g.GDN2_F32)
+    n3 = g.gdn2_chunk_fwd_workspace_bytes(2, 3, 128, 128, 128, 64, g.GDN2_F32)
+    assert n2 - 256 == 2 * (n1 - 256) and n3 - 256 == 6 * (n2 - 256)
+    # a ragged tail costs a whole chunk
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 1, 65, 128, 128, 64, g.GDN2_F32) == n2
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)       # never dereferenced: every case below fails validation first
+
+
+def call_fwd(lib, B=1, H=1, T=8, K=128, V=128, C=64, dtype=1, ptr=FAKE, ST=FAKE, ws=FAKE, ws_bytes=1 << 30,
+             o=FAKE):
+    return lib.gdn2_chunk_fwd(ptr, ptr, ptr, ptr, ptr, ptr, None, o, ST, B, H, T, K, V, C, dtype, ws, ws_bytes,
+                              None)
+
+
+def test_chunk_fwd_validation(lib):
+    assert call_fwd(lib, T=-1) == -2
+    assert call_fwd(lib, B=-1) == -2
+    assert call_fwd(lib, dtype=7) == -3
+    assert call_fwd(lib, K=96) == -4
+    assert call_fwd(lib, V=32) == -4
+    assert call_fwd(lib, C=32) == -4
+    assert call_fwd(lib, ptr=None) == -1
+    assert call_fwd(lib, o=None) == -1
+    assert call_fwd(lib, ST=None) == -1
+    assert call_fwd(lib, ptr=P(0x10004)) == -7
+    assert call_fwd(lib, ws=None) == -5
+    assert call_fwd(lib, ws=P(0x10008)) == -7
+    assert call_fwd(lib, ws_bytes=16) == -5
+    # empty batch: nothing to launch
+    assert call_fwd(lib, B=0) == 0
+    assert call_fwd(lib, H=0) == 0
+
+
+def test_decode_validation(lib):
+    f = lambda **kw: lib.gdn2_decode_step(*(kw.get("ptr", FAKE),) * 6, kw.get("S", FAKE), kw.get("o", FAKE),
+                                         kw.get("B", 1), kw.get("H", 1), kw.get("K", 128), kw.get("V", 128),
+                                         kw.get("dtype", 1), None)
+    assert f(B=-1) == -2
+    assert f(dtype=2) == -3
+    assert f(K=256) == -4
+    assert f(ptr=None) == -1
+    assert f(S=None) == -1
+    assert f(S=P(0x10002)) == -7
+    assert f(B=0) == 0
+
+
+def test_workspace_status_null(lib):
+    out = ctypes.c_int(0)
+    assert lib.gdn2_workspace_status(None, 0, ctypes.byref(out), None) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((1, 4, 1, 64), dtype=torch.bfloat16)
+    a = torch.zeros((1, 4, 1, 64))
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdn2_chunk_fwd(x, x, x, a, x, x, None, x, torch.zeros(1, 1, 64, 64))

@@ -1,0 +1,156 @@
+"""GPU parity of gdn2_chunk_fwd against the fp64 oracle (same seeded inputs).
+
+Bar: max|gpu - oracle| / max|oracle| <= 1e-4 for fp32 tokens, <= 2e-2 for bf16 tokens
+with fp32 state, on o and on S_T.  Small cases compare every element; the full-size
+workloads run the whole launch and compare sampled (b, h) chains, which the oracle
+recomputes alone from the same counter-based generator.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.gpu_util import TOL, assert_close, cuda_or_skip, f64, prefill, to_device, workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(wl, S0_np=None, C=64):
+    torch, g = cuda_or_skip()
+    x = synth.make_inputs(wl)
+    xd = to_device(torch, x, wl.dtype)
+    S0 = None if S0_np is None else torch.from_numpy(S0_np).cuda()
+    o, ST = prefill(torch, g, xd, S0, C=C)
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0_np)
+    e1 = assert_close("o", f64(o), ref_o, TOL[wl.dtype])
+    e2 = assert_close("S_T", f64(ST), ref_S, TOL[wl.dtype])
+    return e1, e2
+
+
+def test_tiny_f32_workload():
+    _full_check(synth.WORKLOADS["tiny_f32"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("K,V", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_small_shapes(dtype, K, V, T):
+    wl = synth.Workload("s", 2, 3, T, K, V, dtype, 1.0 if dtype == "bf16" else 0.0, s0_std=0.05,
+                        seed=1000 + T + K + 3 * V)
+    _full_check(wl, synth.make_state(wl))
+
+
+@pytest.mark.parametrize("gates", ["kda", "gdn"])
+def test_collapsed_gates_small(gates):
+    wl = synth.Workload("c", 2, 4, 192, 128, 128, "bf16", 1.0, gates=gates, seed=77)
+    _full_check(wl)
+
+
+def test_slow_decay_small():
+    wl = synth.Workload("sd", 2, 4, 320, 128, 128, "bf16", 1.0, alpha_scale=0.02, s0_std=0.01, seed=78)
+    _full_check(wl, synth.make_state(wl))
+
+
+def test_extreme_decay_and_unit_decay():
+    """alpha spanning 1e-30 .. 1 (every factor stays finite), exact alpha = 1 rows."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("x", 1, 2, 130, 128, 128, "bf16", 1.0, seed=79, s0_std=0.05)
+    x = synth.make_inputs(wl)
+    rng = np.random.default_rng(5)
+    a = x["alpha"].copy()
+    mask = rng.random(a.shape) < 0.05
+    a[mask] = np.float32(1e-30)
+    a[:, 10:20] = 1.0
+    x["alpha"] = a
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    o, ST = prefill(torch, g, xd, torch.from_numpy(S0).cuda())
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
+    assert_close("o", f64(o), ref_o, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
+def test_T0_copies_state_and_empty_batch():
+    torch, g = cuda_or_skip()
+    B, H, K, V = 2, 3, 64, 128
+    z = lambda d: torch.zeros((B, 0, H, d), device="cuda", dtype=torch.bfloat16)
+    S0 = torch.randn(B, H, K, V, device="cuda")
+    o = torch.empty((B, 0, H, V), device="cuda", dtype=torch.bfloat16)
+    S_T = torch.full((B, H, K, V), float("nan"), device="cuda")
+    ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, 0, K, V, 64, g.GDN2_BF16))
+    alpha = torch.zeros((B, 0, H, K), device="cuda")
+    g.gdn2_chunk_fwd(z(K), z(K), z(V), alpha, z(K), z(V), S0, o, S_T, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(S_T, S0)
+    g.gdn2_chunk_fwd(z(K), z(K), z(V), alpha, z(K), z(V), None, o, S_T, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S_T).item() == 0
+
+
+def test_in_place_resume_and_split():
+    """S_T aliasing S0; two calls joined by the state equal one call."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("r", 2, 2, 200, 128, 128, "bf16", 1.0, seed=80, s0_std=0.02)
+    x = synth.make_inputs(wl)
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    o_all, S_all = prefill(torch, g, xd, torch.from_numpy(S0).cuda())
+    S = torch.from_numpy(S0).cuda()
+    cut = 96
+    part = lambda s: {k: v[:, s].contiguous() for k, v in xd.items()}
+    B, T, H, K = xd["q"].shape
+    for sl in (slice(0, cut), slice(cut, T)):
+        p = part(sl)
+        o = torch.empty((B, sl.stop - sl.start, H, 128), dtype=torch.bfloat16, device="cuda")
+        ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, sl.stop - sl.start, K, 128, 64, g.GDN2_BF16))
+        g.gdn2_chunk_fwd(p["q"], p["k"], p["v"], p["alpha"], p["b"], p["w"], S, o, S, workspace=ws)
+        torch.cuda.synchronize()
+        if sl.start == 0:
+            o1 = o
+        else:
+            o2 = o
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
+    assert_close("o split", f64(torch.cat([o1, o2], dim=1)), ref_o, TOL["bf16"])
+    assert_close("S split", f64(S), ref_S, TOL["bf16"])
+    assert_close("S one call", f64(S_all), ref_S, TOL["bf16"])
+
+
+def _sampled_check(name, chains, threads=None):
+    torch, g = cuda_or_skip()
+    wl = synth.WORKLOADS[name]
+    x = synth.make_inputs(wl)
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    del x
+    S0d = None if S0 is None else torch.from_numpy(S0).cuda()
+    o, ST = prefill(torch, g, xd, S0d, poison=True)
+    del xd
+    xs = synth.make_inputs(wl, chains=chains)
+    S0s = synth.make_state(wl, chains=chains)
+    ref_o, ref_S = oracle.chain_recurrence(*(xs[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0s,
+                                           threads=threads)
+    for n, (b, h) in enumerate(chains):
+        assert_close(f"o chain {b},{h}", f64(o[b, :, h]), ref_o[n], TOL[wl.dtype])
+        assert_close(f"S_T chain {b},{h}", f64(ST[b, h]), ref_S[n], TOL[wl.dtype])
+    assert torch.isfinite(o.float()).all().item()
+    assert torch.isfinite(ST).all().item()
+
+
+def test_prefill_1p3b_full_size_sampled():
+    _sampled_check("prefill_1p3b", [(0, 0), (3, 7), (7, 15), (5, 2)])
+
+
+def test_prefill_kda_full_size_sampled():
+    _sampled_check("prefill_kda", [(0, 1), (6, 9)])
+
+
+def test_prefill_gdn_full_size_sampled():
+    _sampled_check("prefill_gdn", [(1, 0), (7, 14)])
+
+
+def test_prefill_long_full_size_sampled():
+    _sampled_check("prefill_long", [(0, 0), (0, 11)])
+
+
+def test_prefill_slow_decay_full_size_sampled():
+    _sampled_check("prefill_slow_decay", [(2, 3)])

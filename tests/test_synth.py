@@ -38,7 +38,8 @@ def test_small_workload_shapes_and_ranges():
     wl = synth.WORKLOADS["tiny_f32"]
     x = synth.make_inputs(wl)
     assert x["q"].shape == (1, 256, 2, 64) and x["v"].shape == (1, 256, 2, 64)
-    np.testing.assert_allclose(np.linalg.norm(x["k"], axis=-1), 1.0, rtol=1e-6)
+    assert x["q"].dtype == np.float32
+    np.testing.assert_allclose(np.linalg.norm(x["k"].astype(np.float64), axis=-1), 1.0, rtol=1e-6)
     assert np.all(x["alpha"] > 0) and np.all(x["alpha"] <= 1)
     assert np.all(x["b"] > 0) and np.all(x["b"] < 1)
     assert synth.make_state(wl) is None
@@ -76,3 +77,19 @@ def test_time_window_matches_full():
     full = synth.make_inputs(wl)
     part = synth.make_inputs(wl, chains=[(0, 1)], t_range=(10, 30))
     np.testing.assert_array_equal(part["q"][0], full["q"][0, 10:30, 1])
+
+
+def test_bf16_workload_values_are_bf16_representable():
+    wl = synth.Workload("r", 2, 3, 10, 16, 8, "bf16", 1.0, seed=11)
+    x = synth.make_inputs(wl)
+    for key in ("q", "k", "v", "b", "w"):
+        assert np.all((x[key].view(np.uint32) & 0xFFFF) == 0), key
+    assert np.any((x["alpha"].view(np.uint32) & 0xFFFF) != 0)   # alpha stays fp32
+
+
+def test_decay_distribution_matches_recipe():
+    wl = synth.Workload("a", 4, 4, 512, 64, 8, "bf16", 1.0, seed=12)
+    a = synth.make_inputs(wl)["alpha"].astype(np.float64)
+    # alpha = exp(-softplus(x)), x ~ N(1, 1): the median is exp(-softplus(1)) ~ 0.2725
+    assert abs(np.median(a) - np.exp(-np.logaddexp(0, 1.0))) < 0.01
+    assert a.min() > 0 and a.max() <= 1
