@@ -1,0 +1,482 @@
+"""Benchmark of the GDN-2 recurrence hot path on B200: one step = one chunkwise prefill
+over the 1.3B-scale layer workload (B=8, H=16, T=4096, d_k=d_v=128, bf16 tokens, fp32
+alpha and state, C=64) plus one batched decode step (B=256, H=16, d=128, 256 MiB fp32
+state updated in place).  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU; every rank runs the same per-GPU workload
+on its own seeded shard (independent chains, no data-path collective: weak scaling).
+The only collectives are the barrier and the max-over-ranks of the device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s GDN-2 chunk fwd (B8 H16 T4k d128) + decode; % tensor/HBM roofline"
+PREFILL = "prefill_1p3b"
+DECODE = "decode_b256"
+
+
+# ----------------------------------------------------------------------------- work accounting
+
+def prefill_bytes(B, T, H, K, V, tok_bytes=2, s0=False):
+    """Algorithmic HBM bytes of one prefill call: every input read once, every output
+    written once (q, k, b: d_k; v, w: d_v in the token dtype; alpha fp32; o; S_T; S0)."""
+    per_token_head = (3 * K + 2 * V) * tok_bytes + 4 * K + V * tok_bytes
+    state = 4 * B * H * K * V
+    return B * T * H * per_token_head + state * (2 if s0 else 1)
+
+
+def prefill_flops(B, T, H, K, V, C=64):
+    """Chunked-algorithm flops: intra-chunk Gram matrices and WY factors (2*C*(2K) + 2*C*(K+V)
+    per token-head... counted as the tensor-core products), inter-chunk products and the
+    C x C triangular inverse."""
+    per_chunk = (2 * C * C * K * 2          # A and P
+                 + 2 * C * C * (K + V)      # W = T E+, U~ = T U
+                 + 2 * C * K * V * 3        # W S, Q+ S, K^T Delta
+                 + 2 * C * C * V            # P Delta
+                 + C ** 3 // 3)             # (I + A)^-1
+    n_chunks = B * H * ((T + C - 1) // C)
+    return n_chunks * per_chunk
+
+
+def decode_bytes(B, H, K, V, tok_bytes=2):
+    state = 4 * B * H * K * V
+    return 2 * state + B * H * ((3 * K + 2 * V) * tok_bytes + 4 * K + V * tok_bytes)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]), "src": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+        if kernel_source_sha(rec["sources"]) != rec["sources_sha"]:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(x, pg, device):
+    """Max of a float over ranks (the only reduction: timing)."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, pg, device):
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_workload(name, rank):
+    """Per-rank shard: same shapes, its own seed (independent chains)."""
+    import synth
+    wl = synth.WORKLOADS[name]
+    if rank == 0:
+        return wl
+    fields = {f: getattr(wl, f) for f in wl.__dataclass_fields__}
+    fields["seed"] = wl.seed + 0x10000 * rank
+    return synth.Workload(**fields)
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample_time(prefill_wl, decode_wl, budget_s=12.0, max_chains=None):
+    """Time the fp64 oracle as it stands on a bounded sample of the step's work.
+
+    Prefill: whole (b, h) chains of the prefill workload (full T), as many as fit the
+    budget (at least 2*cores, capped by the workload); decode: one decode step of a
+    slice of the heads.  Returns (seconds for a FULL step extrapolated by work share,
+    description, threads used)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    cores = os.cpu_count() or 1
+    B, H, T = prefill_wl.B, prefill_wl.H, prefill_wl.T
+    all_chains = [(b, h) for b in range(B) for h in range(H)]
+    n = min(len(all_chains), max(2 * cores, 4)) if max_chains is None else min(max_chains, len(all_chains))
+    chains = all_chains[:n]
+    x = synth.as_f64(synth.make_inputs(prefill_wl, chains=chains))
+    S0 = synth.make_state(prefill_wl, chains=chains)
+    t0 = time.perf_counter()
+    oracle.chain_recurrence(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], S0, threads=cores)
+    t_pre = time.perf_counter() - t0
+    # grow the sample while well under budget (more chains give a steadier rate)
+    if max_chains is None and t_pre < budget_s / 4 and n < len(all_chains):
+        n2 = min(len(all_chains), int(n * max(2.0, (budget_s / 2) / max(t_pre, 1e-3))))
+        chains = all_chains[:n2]
+        x = synth.as_f64(synth.make_inputs(prefill_wl, chains=chains))
+        S0 = synth.make_state(prefill_wl, chains=chains)
+        t0 = time.perf_counter()
+        oracle.chain_recurrence(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], S0, threads=cores)
+        t_pre = time.perf_counter() - t0
+        n = n2
+    full_pre = t_pre * len(all_chains) / n
+    # decode: one step over a slice of the heads
+    heads = [(b, h) for b in range(min(decode_wl.B, 64)) for h in range(decode_wl.H)]
+    xd = synth.as_f64(synth.make_inputs(decode_wl, chains=heads, step=0))
+    S = synth.make_state(decode_wl, chains=heads).astype(np.float64).reshape(len(heads), 1, decode_wl.K,
+                                                                              decode_wl.V)
+    t0 = time.perf_counter()
+    oracle.decode_step(*(xd[k][:, None] for k in ("q", "k", "v", "alpha", "b", "w")), S, threads=cores)
+    t_dec = time.perf_counter() - t0
+    full_dec = t_dec * (decode_wl.B * decode_wl.H) / len(heads)
+    desc = (f"fp64 oracle on {n} of {len(all_chains)} prefill chains (full T={T}) and one decode step of "
+            f"{len(heads)} of {decode_wl.B * decode_wl.H} heads, scaled to one full step by work share")
+    return full_pre + full_dec, desc, cores
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    pw, dw = synth.WORKLOADS[PREFILL], synth.WORKLOADS[DECODE]
+    tokens_step = pw.B * pw.T + dw.B
+    cores = os.cpu_count() or 1
+    times, desc = [], ""
+    for i in range(args.warmup + args.steps):
+        t_full, desc, cores = oracle_sample_time(pw, dw, budget_s=4.0, max_chains=max(2, cores))
+        if i >= args.warmup:
+            times.append(t_full)
+    sec = statistics.mean(times)
+    value = tokens_step / sec
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{PREFILL} (B8 H16 T4096 d128) + {DECODE} (B256 H16 d128)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc + " (each step)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+
+    import gated_delta_rule_96_b200 as g
+    import synth
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    g.load_library()
+    pw, dw = rank_workload(PREFILL, rank), rank_workload(DECODE, rank)
+
+    def dev_tokens(x, dtype):
+        out = {}
+        for k, a in x.items():
+            t = torch.from_numpy(a).to(dev)
+            out[k] = t if k == "alpha" else t.to(dtype)
+        return out
+
+    # ---- inputs resident in HBM
+    xp = synth.make_inputs(pw)
+    P = dev_tokens(xp, torch.bfloat16)
+    B, T, H, K = P["q"].shape
+    V = P["v"].shape[-1]
+    o_p = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((B, H, K, V), dtype=torch.float32, device=dev)
+    ws_bytes = g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_BF16)
+    ws = g.new_workspace(ws_bytes, dev)
+    path = g.gdn2_chunk_fwd_path(B, H, T, K, V, 64, g.GDN2_BF16)
+    xd = synth.make_inputs(dw, step=0)
+    D = dev_tokens(xd, torch.bfloat16)
+    S_dec = torch.from_numpy(synth.make_state(dw)).to(dev)
+    o_d = torch.empty((dw.B, dw.H, dw.V), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    parts = set(args.parts.split(","))
+
+    def prefill():
+        if "prefill" not in parts:
+            return
+        g.gdn2_chunk_fwd(P["q"], P["k"], P["v"], P["alpha"], P["b"], P["w"], None, o_p, S_T, workspace=ws,
+                         stream=stream)
+
+    def decode():
+        if "decode" not in parts:
+            return
+        g.gdn2_decode_step(D["q"], D["k"], D["v"], D["alpha"], D["b"], D["w"], S_dec, o_d, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    torch.cuda.synchronize(dev)
+    if g.gdn2_workspace_status(ws) != 0:
+        raise SystemExit("prefill kernel reported an internal error during warm-up")
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    marks = [(ev(), ev(), ev()) for _ in range(args.steps)]
+    start, stop = ev(), ev()
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for (a, b_, c) in marks:
+            a.record(stream)
+            prefill()
+            b_.record(stream)
+            decode()
+            c.record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(pg)
+    clocks = clk.summary()
+    if g.gdn2_workspace_status(ws) != 0:
+        raise SystemExit("prefill kernel reported an internal error in the timed region")
+    total_ms = start.elapsed_time(stop)
+    pre_ms = statistics.mean(a.elapsed_time(b_) for a, b_, _ in marks)
+    dec_ms = statistics.mean(b_.elapsed_time(c) for _, b_, c in marks)
+    total_ms = max_over_ranks(total_ms, pg, dev)
+    pre_ms_max = max_over_ranks(pre_ms, pg, dev)
+    dec_ms_max = max_over_ranks(dec_ms, pg, dev)
+
+    tokens_rank = B * T + dw.B
+    tokens_all = sum_over_ranks(tokens_rank, pg, dev)
+    ms_per_step = total_ms / args.steps
+    value = tokens_all / (ms_per_step * 1e-3)
+
+    peaks = load_peaks()
+    pb = prefill_bytes(B, T, H, K, V)
+    db = decode_bytes(dw.B, dw.H, dw.K, dw.V)
+    pre_gbs = pb / (pre_ms * 1e-3) / 1e9
+    dec_gbs = db / (dec_ms * 1e-3) / 1e9
+    pflops = prefill_flops(B, T, H, K, V)
+    pre_kernel_key = "prefill_tc" if path == 1 else "prefill_simt"
+    pre_src = (["gated_delta_rule_96_b200/csrc/gdn2_chunk_tc.cu"] if path == 1
+               else ["gated_delta_rule_96_b200/csrc/gdn2_chunk_simt.cu"])
+    tr_pre = recorded_traffic(pre_kernel_key)
+    tr_dec = recorded_traffic("decode")
+    roof_pre = {"bound": "hbm", "achieved": pre_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": pre_gbs / peaks["hbm_gbs"], "traffic": tr_pre, "peak_src": peaks["src"],
+                "kernel": pre_kernel_key, "algorithmic_bytes_per_launch": pb,
+                "tensor_tflops": pflops / (pre_ms * 1e-3) / 1e12}
+    roof_dec = {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": dec_gbs / peaks["hbm_gbs"], "traffic": tr_dec, "peak_src": peaks["src"],
+                "kernel": "decode", "algorithmic_bytes_per_launch": db}
+
+    # ---- end to end through the public API: pinned host inputs -> device -> results -> host
+    host = {k: v.to("cpu").pin_memory() for k, v in P.items()}
+    host_d = {k: v.to("cpu").pin_memory() for k, v in D.items()}
+    o_h = torch.empty(o_p.shape, dtype=o_p.dtype).pin_memory()
+    S_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    od_h = torch.empty(o_d.shape, dtype=o_d.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + \
+        sum(t.numel() * t.element_size() for t in host_d.values())
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size() + od_h.numel() * od_h.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for k2 in P:
+            P[k2].copy_(host[k2], non_blocking=True)
+        prefill()
+        o_h.copy_(o_p, non_blocking=True)
+        S_h.copy_(S_T, non_blocking=True)
+        for k2 in D:
+            D[k2].copy_(host_d[k2], non_blocking=True)
+        decode()
+        od_h.copy_(o_d, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(pg)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
+    e2e_value = tokens_all / (e2e_ms * 1e-3)
+
+    launches_per_step = (1 if path == 1 else 2) + 1
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{PREFILL} (B8 H16 T4096 d_k=d_v=128, C=64, bf16 tokens, fp32 alpha/state) + "
+                               f"{DECODE} (B256 H16 d128 decode step, 256 MiB fp32 state in place)",
+                   "per_gpu": {"prefill": [B, T, H, K, V], "decode": [dw.B, dw.H, dw.K, dw.V]},
+                   "global_batch": {"prefill": B * world, "decode": dw.B * world},
+                   "l2": "inputs larger than L2 (1.09 GB prefill inputs, 256 MiB decode state); no flush",
+                   "prefill_path": "tcgen05" if path == 1 else "simt",
+                   "parallelism": f"replicas x{world} (independent chains, no collective)"},
+        "roofline": roof_pre,
+        "parts": {"prefill": {"ms": pre_ms_max, "tokens_per_s": B * T * world / (pre_ms_max * 1e-3),
+                              "roofline": roof_pre},
+                  "decode": {"ms": dec_ms_max, "tokens_per_s": dw.B * world / (dec_ms_max * 1e-3),
+                             "roofline": roof_dec}},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if parts != {"prefill", "decode"}:
+        out["config"]["parts_only"] = sorted(parts)   # profiling run: not a bench line
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, desc, cores = oracle_sample_time(pw, dw)
+        out["cpu_baseline"] = {"value": tokens_rank / sec, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": desc}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--parts", default="prefill,decode",
+                    help="profiling aid: run only some parts of the step (the default runs the whole step)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,96 @@
+"""Host-side logic of bench.py: work accounting, the reference (oracle) arm's JSON line,
+and the multi-rank plumbing (world size 2 over gloo on the CPU)."""
+import json
+import os
+import socket
+
+import pytest
+
+import bench
+
+
+def test_prefill_bytes_per_token_head():
+    # q, k, b (3*128) and v, w (2*128) in bf16, alpha fp32, o bf16: 2,048 B per token-head
+    B, T, H, K, V = 8, 4096, 16, 128, 128
+    assert bench.prefill_bytes(B, T, H, K, V) == B * T * H * 2048 + 4 * B * H * K * V
+    assert bench.prefill_bytes(1, 1, 1, K, V, s0=True) - bench.prefill_bytes(1, 1, 1, K, V) == 4 * K * V
+
+
+def test_decode_bytes():
+    # state read + write dominates: 2 x 256 MiB
+    b = bench.decode_bytes(256, 16, 128, 128)
+    assert b == 2 * 4 * 256 * 16 * 128 * 128 + 256 * 16 * (5 * 128 * 2 + 4 * 128 + 128 * 2)
+
+
+def test_prefill_flops_positive_and_scaling():
+    f1 = bench.prefill_flops(1, 64, 1, 128, 128)
+    assert bench.prefill_flops(2, 128, 3, 128, 128) == 12 * f1
+
+
+def test_peaks_loaded():
+    p = bench.load_peaks()
+    assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
+
+
+def test_reference_arm_json(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setattr(bench, "oracle_sample_time", lambda pw, dw, budget_s, max_chains: (2.0, "stub", 3))
+    assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "1"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["metric"] == bench.METRIC
+    assert line["value"] == pytest.approx((8 * 4096 + 256) / 2.0)
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_nonzero_rank_is_silent(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_oracle_sample_time_small():
+    import synth
+    pw = synth.Workload("p", 1, 2, 128, 16, 16, "bf16", 1.0, seed=3)
+    dw = synth.Workload("d", 4, 2, 1, 16, 16, "bf16", 1.0, s0_std=0.01, seed=4, decode=True)
+    sec, desc, cores = bench.oracle_sample_time(pw, dw, budget_s=0.5, max_chains=2)
+    assert sec > 0 and cores >= 1 and "oracle" in desc
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import torch
+    torch.cuda.is_available = lambda: False   # force the gloo branch on any box
+    r, w, local, pg = bench.dist_setup(world)
+    bench.barrier(pg)
+    mx = bench.max_over_ranks(float(rank + 1) * 10.0, pg, "cpu")
+    sm = bench.sum_over_ranks(float(rank + 1), pg, "cpu")
+    seed = bench.rank_workload(bench.PREFILL, rank).seed
+    pg.destroy_process_group()
+    q.put((r, w, mx, sm, seed))
+
+
+def test_two_rank_plumbing_gloo():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[0] for r in res] == [0, 1]
+    assert all(r[2] == 20.0 and r[3] == 3.0 for r in res)     # max and sum over ranks
+    assert res[0][4] != res[1][4]                              # distinct shards
