@@ -17,6 +17,7 @@ import os
 __all__ = [
     "GDN2Error", "load_library", "library_path", "gdn2_chunk_fwd", "gdn2_decode_step",
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
+    "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace",
 ]
 
@@ -26,6 +27,7 @@ _lib = None
 
 GDN2_F32, GDN2_BF16 = 0, 1
 STATUS_HEADER_BYTES = 256
+NOALLOC_SCRATCH_BYTES = 32 << 20   # GDN2_NOALLOC_SCRATCH_BYTES in include/gdn2.h
 
 
 class GDN2Error(RuntimeError):
@@ -59,6 +61,8 @@ def load_library():
     lib.gdn2_decode_step.restype = i
     lib.gdn2_workspace_status.argtypes = [vp, i, ctypes.POINTER(i), vp]
     lib.gdn2_workspace_status.restype = i
+    lib.gdn2_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i] * 7 + [vp]
+    lib.gdn2_chunk_fwd_noalloc.restype = i
     lib.gdn2_status_str.argtypes = [i]
     lib.gdn2_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -141,6 +145,20 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, C=64, workspace=None, strea
                                        workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_fwd")
+
+
+def gdn2_chunk_fwd_noalloc(q, k, v, alpha, b, w, S0, o, S_T, C=64, stream=None) -> None:
+    """Prefill for callers that cannot allocate device memory: no workspace argument; the
+    library's fixed scratch array is used instead (see include/gdn2.h for the size limit
+    and for the rule that overlapping calls race on the shared array)."""
+    _check_cuda(q, k, v, alpha, b, w, S0, o, S_T)
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    rc = load_library().gdn2_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                                               _ptr(S0), _ptr(o), _ptr(S_T), B, H, T, K, V, C, _dtype_code(q),
+                                               _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_chunk_fwd_noalloc")
 
 
 def gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=None) -> None:

@@ -114,6 +114,8 @@ const char *gdn2_status_str(int status) {
         case GDN2_ERR_CUDA: return "CUDA runtime or launch error";
         case GDN2_ERR_ALIGN: return "a pointer is not 16-byte aligned";
         case GDN2_ERR_DEVICE: return "a kernel reported an internal error";
+        case GDN2_ERR_NOALLOC_LIMIT:
+            return "problem needs more scratch than the no-allocation entry point's fixed array";
         default: return "unknown status";
     }
 }

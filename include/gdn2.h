@@ -49,8 +49,10 @@ typedef enum {
     GDN2_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than required           */
     GDN2_ERR_CUDA = -6,         /* a CUDA runtime call or kernel launch failed       */
     GDN2_ERR_ALIGN = -7,        /* a pointer is not 16-byte aligned                  */
-    GDN2_ERR_DEVICE = -8        /* a kernel reported an internal error (bounded wait
+    GDN2_ERR_DEVICE = -8,       /* a kernel reported an internal error (bounded wait
                                    expired); read by gdn2_workspace_status           */
+    GDN2_ERR_NOALLOC_LIMIT = -9 /* gdn2_chunk_fwd_noalloc: the problem needs more
+                                   scratch than GDN2_NOALLOC_SCRATCH_BYTES           */
 } gdn2_status;
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
@@ -104,6 +106,34 @@ GDN2_API int gdn2_workspace_status(void *workspace, int clear, int *out, void *s
 
 /* Static description of a status code (never NULL). */
 GDN2_API const char *gdn2_status_str(int status);
+
+/*
+ * Prefill for callers that cannot allocate device memory.  (The pages have no
+ * counterpart: this is a deployment convenience of this library.)
+ *
+ * Who needs it: hosts that own all device memory (a framework's pool allocator or a
+ * fixed per-process budget) and do not let a plugin call cudaMalloc, and callers that
+ * forbid allocation on a latency-critical path because cudaMalloc can synchronise the
+ * device.  They cannot hand gdn2_chunk_fwd a workspace.
+ *
+ * Same arguments and results as gdn2_chunk_fwd without the workspace; it always runs
+ * the CUDA-core (SIMT) chunkwise path.  Its scratch is one fixed array of
+ * GDN2_NOALLOC_SCRATCH_BYTES (32 MiB) in the library's device memory, reserved on every
+ * GPU that loads the library until the process exits.  The call allocates nothing.
+ *   - Limit: 256 + 4 * B * H * ceil(T/64) * (3*64*d_k + 64*d_v + 64*64 + d_k) bytes must
+ *     not exceed GDN2_NOALLOC_SCRATCH_BYTES (e.g. B*H*ceil(T/64) <= 226 chunk-heads at
+ *     d_k = d_v = 128); larger problems return GDN2_ERR_NOALLOC_LIMIT and launch nothing.
+ *   - The first call on a device looks up the array's device address on that device
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (nothing in it
+ *     needs to start at zero).  Calls that overlap on the GPU -- on different streams or
+ *     from different host threads -- race on it: serialise them.
+ */
+#define GDN2_NOALLOC_SCRATCH_BYTES (32u << 20)
+GDN2_API int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *alpha,
+                                    const void *b, const void *w, const float *S0, void *o, float *S_T, int B,
+                                    int H, int T, int d_k, int d_v, int C, int dtype, void *stream);
 
 /* Which prefill implementation gdn2_chunk_fwd selects for these sizes:
  * 0 = SIMT two-kernel path (fp32 FMA), 1 = fused tcgen05 tensor-core path. */
