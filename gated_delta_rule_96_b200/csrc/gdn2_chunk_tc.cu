@@ -70,9 +70,10 @@ constexpr uint32_t SM_U = 81920;                  // U [i x v] 64 x 128
 constexpr uint32_t SM_DL = 98304;                 // Delta [i x v] 64 x 128
 constexpr uint32_t SM_T = 114688;                 // T [r x i] 64 x 64, followed by
 constexpr uint32_t SM_P = 122880;                 // P [r x i]: [T; P] is one K-major 128-row operand
-constexpr uint32_t SM_AS = 131072;                // A fp32 [64][65]
-constexpr uint32_t SM_TF = SM_AS + 64 * 65 * 4;   // T fp32 [64][65]
-constexpr uint32_t SM_VEC = SM_TF + 64 * 65 * 4;  // [2 chunks][sS, sZ, sPost] + g_0 (7 x 128 fp32)
+constexpr int LDA = 68;                           // fp32 row stride: conflict-free mma fragment loads
+constexpr uint32_t SM_AS = 131072;                // A fp32 [64][LDA]
+constexpr uint32_t SM_TF = SM_AS + 64 * LDA * 4;  // T fp32 [64][LDA]
+constexpr uint32_t SM_VEC = SM_TF + 64 * LDA * 4;  // [2 chunks][sS, sZ, sPost] + g_0 (7 x 128 fp32)
 constexpr uint32_t SM_WT = SM_VEC + 3584;         // fp32 [8][128] warp totals / solve scratch
 constexpr uint32_t SM_ALPHA = SM_WT + 4096;       // alpha of the next chunk, fp32 [64][128]
 constexpr uint32_t SM_MISC = SM_ALPHA + 32768;    // mbarriers, TMEM slot, flags
@@ -372,9 +373,14 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
             if (quarter < 2) {   // rows 0..63: A, strictly lower
                 const int r = crow;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 32; i += 4) {
                     const int col = 32 * chalf + i;
-                    AS[r * 65 + col] = col < r ? __uint_as_float(r32[i]) : 0.f;
+                    float4 x;
+                    x.x = col < r ? __uint_as_float(r32[i]) : 0.f;
+                    x.y = col + 1 < r ? __uint_as_float(r32[i + 1]) : 0.f;
+                    x.z = col + 2 < r ? __uint_as_float(r32[i + 2]) : 0.f;
+                    x.w = col + 3 < r ? __uint_as_float(r32[i + 3]) : 0.f;
+                    *reinterpret_cast<float4 *>(AS + r * LDA + col) = x;
                 }
             } else {             // rows 64..127: P, lower with diagonal -> bf16 tile
                 const int r = crow - 64;
@@ -424,8 +430,8 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
                         }
                     }
                     if (lane == 0) {
-                        AS[r * 65 + i] = i < r ? a : 0.f;
-                        TF[r * 65 + i] = i <= r ? pp : 0.f;
+                        AS[r * LDA + i] = i < r ? a : 0.f;
+                        TF[r * LDA + i] = i <= r ? pp : 0.f;
                     }
                 }
             }
@@ -434,7 +440,7 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
                 const int r = tid1 >> 2, i0 = 16 * (tid1 & 3);
                 uint32_t pk[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(TF[r * 65 + i0 + 2 * i], TF[r * 65 + i0 + 2 * i + 1]);
+                for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(TF[r * LDA + i0 + 2 * i], TF[r * LDA + i0 + 2 * i + 1]);
                 *reinterpret_cast<uint4 *>(sm + SM_P + sw_off(r, i0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 *reinterpret_cast<uint4 *>(sm + SM_P + sw_off(r, i0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
@@ -458,10 +464,10 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
                     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
                     for (int i = 0; i < r; i += 4) {
-                        s0 += AS[(o16 + r) * 65 + o16 + i] * col[i];
-                        if (i + 1 < r) s1 += AS[(o16 + r) * 65 + o16 + i + 1] * col[i + 1];
-                        if (i + 2 < r) s2 += AS[(o16 + r) * 65 + o16 + i + 2] * col[i + 2];
-                        if (i + 3 < r) s3 += AS[(o16 + r) * 65 + o16 + i + 3] * col[i + 3];
+                        s0 += AS[(o16 + r) * LDA + o16 + i] * col[i];
+                        if (i + 1 < r) s1 += AS[(o16 + r) * LDA + o16 + i + 1] * col[i + 1];
+                        if (i + 2 < r) s2 += AS[(o16 + r) * LDA + o16 + i + 2] * col[i + 2];
+                        if (i + 3 < r) s3 += AS[(o16 + r) * LDA + o16 + i + 3] * col[i + 3];
                     }
                     acc = -((s0 + s1) + (s2 + s3));
                 }
@@ -469,26 +475,26 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                TF[(o16 + r) * 65 + o16 + j] = col[r];
+                TF[(o16 + r) * LDA + o16 + j] = col[r];
                 *reinterpret_cast<__nv_bfloat16 *>(sm + SM_T + sw_off(o16 + r, o16 + j, 64)) = __float2bfloat16_rn(col[r]);
             }
         }
         group_sync(BAR_CHUNK, CHUNK_THREADS);
         if (sw < 2) {   // blocks (1,0) and (3,2): T_RI = -T_RR (A_RI T_II), within one warp
             const int R = 16 * (2 * sw + 1), I = 16 * (2 * sw);
-            float *X = WT + sw * 256;   // 16 x 16, private to this warp
+            float *X = WT + sw * 384;   // 16 x 16 (row stride 24), private to this warp
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, AS, 65, R, I, TF, 65, I, I + 8 * nt, 0, 2, lane);
-                tile_store(X, 16, 0, 8 * nt, d, 1.f, lane);
+                tile_mm(d, AS, LDA, R, I, TF, LDA, I, I + 8 * nt, 0, 2, lane);
+                tile_store(X, 24, 0, 8 * nt, d, 1.f, lane);
             }
             __syncwarp();
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, TF, 65, R, R, X, 16, 0, 8 * nt, 0, 2, lane);
-                tile_store(TF, 65, R, I + 8 * nt, d, -1.f, lane);
+                tile_mm(d, TF, LDA, R, R, X, 24, 0, 8 * nt, 0, 2, lane);
+                tile_store(TF, LDA, R, I + 8 * nt, d, -1.f, lane);
                 tile_store_bf16(sm + SM_T, R, I + 8 * nt, d, -1.f, lane);
             }
         }
@@ -499,14 +505,14 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {   // block (0,1) of T is zero: skipped for columns >= 16
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, AS, 65, 32 + 16 * mt, 0, TF, 65, 0, 8 * nt, nt >= 2 ? 2 : 0, 4, lane);
+                tile_mm(d, AS, LDA, 32 + 16 * mt, 0, TF, LDA, 0, 8 * nt, nt >= 2 ? 2 : 0, 4, lane);
                 tile_store(X, 8, 16 * mt, 0, d, 1.f, lane);
             }
             __syncwarp();
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {   // block (2,3) of T is zero: skipped for rows < 48
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, TF, 65, 32 + 16 * mt, 32, X, 8, 0, 0, 0, mt == 0 ? 2 : 4, lane);
+                tile_mm(d, TF, LDA, 32 + 16 * mt, 32, X, 8, 0, 0, 0, mt == 0 ? 2 : 4, lane);
                 tile_store_bf16(sm + SM_T, 32 + 16 * mt, 8 * nt, d, -1.f, lane);
             }
         }
