@@ -24,19 +24,25 @@
 // factor exp(±(g - m)) lies in [e^-60, e^60] while the chunk's log-decay span
 // g_0 - g_63 stays <= 120 in every channel, and each product exp(g_r - g_i) that A and P
 // need is formed by the tensor core from two representable factors.  A chunk with a
-// wider span computes A and P on CUDA cores from exp(g_r - g_i) <= 1 per element and
-// uses unscaled factors elsewhere (m = 0), so any alpha in (0, 1] is handled.
+// wider span forms A and P on CUDA cores from exp(g_r - g_i) <= 1 per element (written
+// straight into the TMEM accumulator G1 would have produced) and uses unscaled factors
+// elsewhere (m = 0), so any alpha in (0, 1] is handled.
 //
-// Warp roles (16 warps, registers rebalanced per warpgroup with setmaxnreg):
-//   warps 0-3   state group (56 regs): rescales Z, writes its bf16 copy, Delta and o
-//               epilogues
-//   warps 4-11  chunk group (200 regs): loads, build, A/P readout, triangular solve, -W'
-//               epilogue for chunk n+1 while the state group finishes chunk n
-//   warp 12     MMA issuer (56 regs): one thread issues every tcgen05.mma as its inputs
-//               become ready (mbarrier signals), in any order the dependencies allow
-//   warp 13     producer (56 regs): stages alpha of the next chunk into shared memory with
-//               bulk asynchronous copies
-//   warps 14-15 value group (56 regs): U = w ⊙ v of the next chunk
+// Only the state update (G3 -> Delta -> G4/G5 -> rescale) is serial from chunk to chunk;
+// everything before it depends on the tokens alone.  The block therefore runs three
+// CUDA-core stages as a pipeline over chunks, each in its own warpgroup:
+//   warps 0-3   state group: rescales Z and writes its bf16 copy, Delta epilogue of chunk n
+//   warps 4-7   build group: loads, log-decay prefix and the bf16 operands of chunk n+1
+//               (double-buffered [Ê; Q̂] and K̃)
+//   warps 8-11  solve group: A/P readout, triangular solve, [T; P] tile and the -W'
+//               epilogue of chunk n
+//   warps 12-13 u group: U = w ⊙ v of the next chunk
+//   warps 14-15 o group: o epilogue of chunk n
+// Each GEMM is issued by thread 0 of the group that wrote its last operand (G1 build, G2
+// solve, G3 and G4/G5 state), so no thread polls for work.
+// Registers are rebalanced per warpgroup with setmaxnreg (the build group holds a whole
+// chunk's loads in flight).
+// Every event that a waiter may see two chunks late has one mbarrier per buffer slot.
 // Every wait is bounded; on expiry the block sets the workspace status word and exits.
 #include "gdn2_common.cuh"
 #include "gdn2_internal.h"
@@ -49,44 +55,43 @@ using namespace gdn2::tc;
 
 constexpr int C = 64, KD = 128, VD = 128;
 constexpr int NT = 512;                       // 16 warps
-constexpr int STATE_THREADS = 128, CHUNK_THREADS = 256;
-constexpr uint32_t BAR_STATE = 1, BAR_CHUNK = 2;   // named barrier ids
+constexpr int GROUP = 128;                    // threads of the state, build and solve groups
+constexpr uint32_t BAR_STATE = 1, BAR_BUILD = 2, BAR_SOLVE = 3;   // named barrier ids
 constexpr float SPAN_MAX_LOG2 = 173.123f;     // 120 nats in log2 units
 constexpr uint32_t WAIT_LIMIT = 1u << 22;
-constexpr uint32_t POLL_LIMIT = 1u << 26;
 
 // TMEM columns (512 allocated)
-constexpr uint32_t TM_D2 = 0;                 // [W'; *] (128); [A; P] (64) in its first columns
-constexpr uint32_t TM_D1 = 0;
-constexpr uint32_t TM_D3 = 128;               // [U~ -> Delta; O], two buffers of 128
-constexpr uint32_t TM_Z = 384;                // Z fp32 (128)
+constexpr uint32_t TM_D1 = 0;                 // [A; P] fp32 (64)
+constexpr uint32_t TM_D2 = 64;                // [W'; *] (128)
+constexpr uint32_t TM_D3 = 192;               // [U~ -> Delta; O] (128)
+constexpr uint32_t TM_Z = 320;                // Z fp32 (128)
 constexpr uint32_t TM_COLS = 512;
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t SM_S = 0;                      // Z in bf16 [c x v], B of G3 (MN-major)
-constexpr uint32_t SM_EQ = 32768;                 // [Ê -> -W'; Q̂] 128 x 128 (K-major A of G1 / G3)
-constexpr uint32_t SM_KT = 65536;                 // K̃ [i x c] 64 x 128
-constexpr uint32_t SM_U = 81920;                  // U [i x v] 64 x 128
-constexpr uint32_t SM_DL = 98304;                 // Delta [i x v] 64 x 128
-constexpr uint32_t SM_T = 114688;                 // T [r x i] 64 x 64, followed by
-constexpr uint32_t SM_P = 122880;                 // P [r x i]: [T; P] is one K-major 128-row operand
+constexpr uint32_t SM_EQ = 32768;                 // 2 slots of [Ê -> -W'; Q̂] 128 x 128 (K-major A of G1 / G3)
+constexpr uint32_t EQ_BYTES = 32768;
+constexpr uint32_t SM_KT = 98304;                 // 2 slots of K̃ [i x c] 64 x 128
+constexpr uint32_t KT_BYTES = 16384;
+constexpr uint32_t SM_U = 131072;                 // 2 slots of U [i x v] 64 x 128
+constexpr uint32_t U_BYTES = 16384;
+constexpr uint32_t SM_DL = 163840;                // Delta [i x v] 64 x 128
+constexpr uint32_t SM_T = 180224;                 // T [r x i] 64 x 64, followed by
+constexpr uint32_t SM_P = 188416;                 // P [r x i]: [T; P] is one K-major 128-row operand
 constexpr int LDA = 68;                           // fp32 row stride: conflict-free mma fragment loads
-constexpr uint32_t SM_AS = 131072;                // A fp32 [64][LDA]
-constexpr uint32_t SM_TF = SM_AS + 64 * LDA * 4;  // T fp32 [64][LDA]
-constexpr uint32_t SM_VEC = SM_TF + 64 * LDA * 4;  // [2 chunks][sS, sZ, sPost] + g_0 (7 x 128 fp32)
-constexpr uint32_t SM_WT = SM_VEC + 3584;         // fp32 [8][128] warp totals / solve scratch
-constexpr uint32_t SM_ALPHA = SM_WT + 4096;       // alpha of the next chunk, fp32 [64][128]
-constexpr uint32_t SM_MISC = SM_ALPHA + 32768;    // mbarriers, TMEM slot, flags
+constexpr uint32_t SM_AS = 196608;                // fp32 [64][LDA]: A below the diagonal, T^T on and above it
+constexpr uint32_t SM_VEC = SM_AS + 64 * LDA * 4; // [2 slots][sS, sZ, sPost] (6 x 128 fp32)
+constexpr uint32_t SM_WT = SM_VEC + 3072;         // build group: [4][128] warp totals + g_0 [128]
+constexpr uint32_t SM_X = SM_WT + 2560;           // solve group: per-warp mma scratch (4 KB)
+constexpr uint32_t SM_MISC = SM_X + 4096;         // mbarriers, TMEM slot, flags
 constexpr uint32_t SM_BYTES = SM_MISC + 256 + 1024;
-constexpr uint32_t SM_G32 = SM_DL;                // wide-span chunks: g fp32 [64][128] over Delta, T, P
 
-// mbarriers (byte offsets inside SM_MISC)
+// mbarriers (byte offsets inside SM_MISC); the first five are pairs indexed by chunk & 1
 enum : uint32_t {
-    MB_BUILD = 0, MB_G1 = 8, MB_SOLVE = 16, MB_G2 = 24, MB_S1DONE = 32, MB_VEC = 40, MB_STILDE = 48,
-    MB_G3 = 56, MB_DELTA = 64, MB_G45 = 72, MB_D3FREE0 = 80, MB_D3FREE1 = 88, MB_AFULL = 96, MB_AEMPTY = 104,
-    MB_U = 112, MB_COUNT = 15
+    MB_VEC = 0, MB_G3 = 16, MB_G45 = 32, MB_U = 48, MB_G2 = 64,
+    MB_G1 = 80, MB_READOUT = 88, MB_S1DONE = 96, MB_D3FREE = 104, MB_END = 112
 };
-constexpr uint32_t MISC_TSLOT = 128, MISC_ABORT = 132;
+constexpr uint32_t MISC_TSLOT = 160, MISC_ABORT = 164;
 
 constexpr uint32_t ID_G1 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t ID_G2 = idesc_bf16(128, 128, 0, 1);
@@ -109,6 +114,12 @@ __device__ __forceinline__ float fast_log2(float x) {
 __device__ __forceinline__ float2 unpack2(uint32_t u) {
     __nv_bfloat162 p = *reinterpret_cast<__nv_bfloat162 *>(&u);
     return make_float2(__low2float(p), __high2float(p));
+}
+// product of two packed bf16 pairs, rounded to bf16 (the exact product of two bf16 values is
+// representable in fp32, so this is one rounding of the exact product)
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
 }
 __device__ __forceinline__ uint32_t tf32(float x) {
     uint32_t r;
@@ -155,6 +166,48 @@ __device__ __forceinline__ void tile_store_bf16(unsigned char *tile, int r0, int
     *reinterpret_cast<uint32_t *>(tile + sw_off(r0 + gq + 8, c0 + 2 * tq, 64)) = pack_bf16(sc * d[2], sc * d[3]);
 }
 
+// T is kept transposed on and above the diagonal of the A scratch (A is strictly lower):
+// T[x][y] (x >= y) lives at AS[y * LDA + x]; entries with x < y are zero and read as zero.
+__device__ __forceinline__ float t_at(const float *AS, int x, int y) { return x >= y ? AS[y * LDA + x] : 0.f; }
+// 16x8 tile of L(16 x 8k) * T(8k x 8), T rows rr0.., columns rc0.. (B operand from T^T)
+__device__ __forceinline__ void tile_mm_tb(float (&d)[4], const float *Lm, int ldl, int l0, int lc0, const float *AS,
+                                           int rr0, int rc0, int ks, int ke, int lane) {
+    const int gq = lane >> 2, tq = lane & 3;
+    for (int s = ks; s < ke; ++s) {
+        const int kc = 8 * s;
+        const uint32_t a0 = tf32(Lm[(l0 + gq) * ldl + lc0 + kc + tq]);
+        const uint32_t a1 = tf32(Lm[(l0 + gq + 8) * ldl + lc0 + kc + tq]);
+        const uint32_t a2 = tf32(Lm[(l0 + gq) * ldl + lc0 + kc + tq + 4]);
+        const uint32_t a3 = tf32(Lm[(l0 + gq + 8) * ldl + lc0 + kc + tq + 4]);
+        const uint32_t b0 = tf32(t_at(AS, rr0 + kc + tq, rc0 + gq));
+        const uint32_t b1 = tf32(t_at(AS, rr0 + kc + tq + 4, rc0 + gq));
+        mma_tf32(d, a0, a1, a2, a3, b0, b1);
+    }
+}
+// 16x8 tile of T(16 x 8k) * R(8k x 8), T rows l0.., columns lc0.. (A operand from T^T)
+__device__ __forceinline__ void tile_mm_ta(float (&d)[4], const float *AS, int l0, int lc0, const float *Rm, int ldr,
+                                           int rr0, int rc0, int ks, int ke, int lane) {
+    const int gq = lane >> 2, tq = lane & 3;
+    for (int s = ks; s < ke; ++s) {
+        const int kc = 8 * s;
+        const uint32_t a0 = tf32(t_at(AS, l0 + gq, lc0 + kc + tq));
+        const uint32_t a1 = tf32(t_at(AS, l0 + gq + 8, lc0 + kc + tq));
+        const uint32_t a2 = tf32(t_at(AS, l0 + gq, lc0 + kc + tq + 4));
+        const uint32_t a3 = tf32(t_at(AS, l0 + gq + 8, lc0 + kc + tq + 4));
+        const uint32_t b0 = tf32(Rm[(rr0 + kc + tq) * ldr + rc0 + gq]);
+        const uint32_t b1 = tf32(Rm[(rr0 + kc + tq + 4) * ldr + rc0 + gq]);
+        mma_tf32(d, a0, a1, a2, a3, b0, b1);
+    }
+}
+// the 16x8 fragment (scaled) as a block of T at rows r0.., columns c0.. (r0 > c0 + 7)
+__device__ __forceinline__ void tile_store_t(float *AS, int r0, int c0, const float (&d)[4], float sc, int lane) {
+    const int gq = lane >> 2, tq = lane & 3;
+    AS[(c0 + 2 * tq) * LDA + r0 + gq] = sc * d[0];
+    AS[(c0 + 2 * tq + 1) * LDA + r0 + gq] = sc * d[1];
+    AS[(c0 + 2 * tq) * LDA + r0 + gq + 8] = sc * d[2];
+    AS[(c0 + 2 * tq + 1) * LDA + r0 + gq + 8] = sc * d[3];
+}
+
 struct Ctx {
     unsigned char *sm;
     uint32_t tmem, misc;
@@ -165,6 +218,9 @@ struct Ctx {
 };
 
 __device__ __forceinline__ uint32_t mbar(const Ctx &c, uint32_t off) { return c.misc + off; }
+// slot barrier of chunk n and the parity of chunk n's phase on it
+__device__ __forceinline__ uint32_t mbar_slot(const Ctx &c, uint32_t off, int n) { return c.misc + off + 8u * (n & 1); }
+__device__ __forceinline__ uint32_t slot_par(int n) { return (uint32_t)((n >> 1) & 1); }
 __device__ __forceinline__ volatile uint32_t *abort_flag(const Ctx &c) {
     return reinterpret_cast<volatile uint32_t *>(c.sm + SM_MISC + MISC_ABORT);
 }
@@ -180,82 +236,191 @@ __device__ __forceinline__ bool group_wait(const Ctx &c, uint32_t mb, uint32_t p
     return !fail;
 }
 
-// ============================================================================ chunk group
-__device__ void chunk_group(const Ctx &c, int tid1) {
+// ============================================================================ MMA issue
+// Every GEMM is issued by thread 0 of the group that produced its last operand, right after
+// the group's barrier (the operand writes are fenced to the async proxy before it); the
+// thread first waits, bounded, for the other inputs and for its accumulator to be free.
+// A failed wait sets the abort flag and skips the GEMM; the waiting consumers then give up.
+__device__ __forceinline__ bool issue_wait(const Ctx &c, uint32_t mb, uint32_t parity) {
+    if (!mbar_wait(mb, parity, WAIT_LIMIT) || *abort_flag(c)) {
+        *abort_flag(c) = 1u;
+        return false;
+    }
+    fence_after();
+    return true;
+}
+// G1(n) = [Ê; Q̂] K̃^T -> D1, once chunk n-1's A and P were read out of D1
+__device__ __forceinline__ void issue_g1(const Ctx &c, int n, bool slow) {
+    fence_after();
+    if (n > 0 && !issue_wait(c, mbar(c, MB_READOUT), (uint32_t)((n - 1) & 1))) return;
+    if (slow) {   // A and P were written into D1 directly
+        mbar_arrive(mbar(c, MB_G1));
+        return;
+    }
+    const uint32_t aEQ = smem_u32(c.sm + SM_EQ) + (n & 1) * EQ_BYTES, aKT = smem_u32(c.sm + SM_KT) + (n & 1) * KT_BYTES;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        mma_ss(c.tmem + TM_D1, desc_kmajor(aEQ, 128, j), desc_kmajor(aKT, 64, j), ID_G1, j > 0);
+    mma_commit(mbar(c, MB_G1));
+}
+// G2(n): [W'; *] = [T; P] Ê -> D2 and [U~; *] = [T; P] U -> D3, once U (slot n & 1) is written
+// and the o rows of chunk n-1 have left D3
+__device__ __forceinline__ void issue_g2(const Ctx &c, int n) {
+    fence_after();
+    if (!issue_wait(c, mbar_slot(c, MB_U, n), slot_par(n))) return;
+    if (n > 0 && !issue_wait(c, mbar(c, MB_D3FREE), (uint32_t)((n - 1) & 1))) return;
+    const uint32_t aEQ = smem_u32(c.sm + SM_EQ) + (n & 1) * EQ_BYTES, aU = smem_u32(c.sm + SM_U) + (n & 1) * U_BYTES,
+                   aTP = smem_u32(c.sm + SM_T);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        mma_ss(c.tmem + TM_D2, desc_kmajor(aTP, 128, j), desc_mnmajor(aEQ, 128, j), ID_G2, j > 0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        mma_ss(c.tmem + TM_D3, desc_kmajor(aTP, 128, j), desc_mnmajor(aU, 64, j), ID_G2, j > 0);
+    mma_commit(mbar_slot(c, MB_G2, n));
+}
+// G3(n): [Delta; O] += [-W'; Q̂] S~, once -W' is written
+__device__ __forceinline__ void issue_g3(const Ctx &c, int n) {
+    fence_after();
+    if (!issue_wait(c, mbar(c, MB_S1DONE), (uint32_t)(n & 1))) return;
+    const uint32_t aEQ = smem_u32(c.sm + SM_EQ) + (n & 1) * EQ_BYTES, aS = smem_u32(c.sm + SM_S);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        mma_ss(c.tmem + TM_D3, desc_kmajor(aEQ, 128, j), desc_mnmajor(aS, 128, j), ID_G3, 1);
+    mma_commit(mbar_slot(c, MB_G3, n));
+}
+// G4/G5(n): O += P Delta, Z += K̃^T Delta
+__device__ __forceinline__ void issue_g45(const Ctx &c, int n) {
+    fence_after();
+    const uint32_t aKT = smem_u32(c.sm + SM_KT) + (n & 1) * KT_BYTES, aDL = smem_u32(c.sm + SM_DL),
+                   aTP = smem_u32(c.sm + SM_T);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        mma_ss(c.tmem + TM_D3, desc_kmajor(aTP, 128, j), desc_mnmajor(aDL, 64, j), ID_G4, 1);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        mma_ss(c.tmem + TM_Z, desc_mnmajor(aKT, 64, j), desc_mnmajor(aDL, 64, j), ID_G5, 1);
+    mma_commit(mbar_slot(c, MB_G45, n));
+}
+
+// ============================================================================ build group
+// Wide-span chunk: A_ri = sum_c e_rc k_ic exp2(g_rc - g_ic) for i < r and P_ri likewise with
+// q for i <= r, one row per thread (rows of A on threads 0-63, of P on 64-127: the TMEM lane
+// of D1 that G1 would have written).  For each channel the exponent g_rc - g_ic is summed from
+// log2 alpha while i walks down from r, so it never leaves [-inf, 0]; tokens are re-read from
+// global memory (resident in L2).
+__device__ __forceinline__ void wide_span_ap(const Ctx &c, int tid1, int t0, int L) {
+    const int r = tid1 & 63;
+    const bool isP = tid1 >= 64;
+    const int T = c.T, H = c.H, bb = c.bb, h = c.h;
+    const uint32_t lane_base = c.tmem + ((uint32_t)((tid1 >> 5) * 32) << 16) + TM_D1;
+    const size_t rowr = ((size_t)bb * T + t0 + min(r, L - 1)) * H + h;
+#pragma unroll 1
+    for (int i0 = 0; i0 < 64; i0 += 16) {
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+        if (r < L && i0 <= r) {
+#pragma unroll 1
+            for (int cc = 0; cc < KD; ++cc) {
+                const float x = isP ? __bfloat162float(c.q[rowr * KD + cc])
+                                    : __bfloat162float(c.b[rowr * KD + cc]) * __bfloat162float(c.k[rowr * KD + cc]);
+                // exponent at i = i0 + 15 (or r): log2 of alpha over positions i+1 .. r
+                const int itop = min(i0 + 15, r);
+                float d = 0.f;
+#pragma unroll 1
+                for (int j = r; j > itop; --j)
+                    d += fast_log2(fmaxf(c.alpha[(((size_t)bb * T + t0 + j) * H + h) * KD + cc], 1.17549435e-38f));
+#pragma unroll
+                for (int i = 15; i >= 0; --i) {
+                    if (i0 + i <= itop) {
+                        const size_t rowi = ((size_t)bb * T + t0 + i0 + i) * H + h;
+                        acc[i] += x * __bfloat162float(c.k[rowi * KD + cc]) * exp2f(d);
+                        d += fast_log2(fmaxf(c.alpha[rowi * KD + cc], 1.17549435e-38f));
+                    }
+                }
+            }
+        }
+        uint32_t r16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int col = i0 + i;
+            const bool keep = r < L && (isP ? col <= r : col < r);
+            r16[i] = __float_as_uint(keep ? acc[i] : 0.f);
+        }
+        tmem_st16(lane_base + i0, r16);
+    }
+    wait_st();
+}
+
+// Builds the bf16 operands of every chunk into slot n & 1 as soon as the slot is free
+// (G3 and G4/G5 of chunk n-2 complete).  Warp w1 owns positions 16 w1 .. 16 w1 + 15, lane l
+// the channels 4l .. 4l+3; the positions are processed as two halves of 8.
+__device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
     unsigned char *sm = c.sm;
-    float *AS = reinterpret_cast<float *>(sm + SM_AS);
-    float *TF = reinterpret_cast<float *>(sm + SM_TF);
     float *vec = reinterpret_cast<float *>(sm + SM_VEC);
-    float *v_g0 = vec + 768;
     float *WT = reinterpret_cast<float *>(sm + SM_WT);
-    float *G32 = reinterpret_cast<float *>(sm + SM_G32);
-    const int sw = tid1 >> 5, lane = tid1 & 31;       // chunk-group warp 0..7
-    const int quarter = sw & 3, chalf = sw >> 2;      // TMEM lane quarter, column half
-    const uint32_t lrow = (uint32_t)(quarter * 32) << 16;
-    const int crow = quarter * 32 + lane;
-    const int c4 = lane * 4, p0 = sw * 8;
+    float *v_g0 = WT + 512;
+    const int w1 = tid1 >> 5, lane = tid1 & 31;
+    const int c4 = lane * 4, p0 = w1 * 16;
     const int T = c.T, H = c.H, bb = c.bb, h = c.h;
 
-    for (int i = tid1; i < 512; i += CHUNK_THREADS)   // T tile: blocks above the diagonal stay zero
-        reinterpret_cast<uint4 *>(sm + SM_T)[i] = make_uint4(0u, 0u, 0u, 0u);
     for (int n = 0; n < c.NC; ++n) {
         const int t0 = n * C, L = min(C, T - t0);
-        const uint32_t par = (uint32_t)(n & 1);
+        unsigned char *EQ = sm + SM_EQ + (n & 1) * EQ_BYTES;
+        unsigned char *KT = sm + SM_KT + (n & 1) * KT_BYTES;
         // ---------------------------------------------------------------- loads and log-decay prefix
-        float al[8][4];   // alpha (1 past the end of the sequence)
-        uint2 rq[8], rk[8], rb[8];
+        float al[16][4];   // alpha (1 past the end of the sequence)
+        uint2 rq[16], rk[16], rb[16];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
+        for (int p = 0; p < 16; ++p) {
             const int t = min(p0 + p, L - 1);
             const size_t row = ((size_t)bb * T + t0 + t) * H + h;
+            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(c.alpha + row * KD + c4));
+            al[p][0] = a4.x; al[p][1] = a4.y; al[p][2] = a4.z; al[p][3] = a4.w;
             rq[p] = __ldg(reinterpret_cast<const uint2 *>(c.q + row * KD + c4));
             rk[p] = __ldg(reinterpret_cast<const uint2 *>(c.k + row * KD + c4));
             rb[p] = __ldg(reinterpret_cast<const uint2 *>(c.b + row * KD + c4));
         }
-        // alpha of this chunk, staged in shared memory by the producer warp
-        if (!group_wait(c, mbar(c, MB_AFULL), par, BAR_CHUNK, CHUNK_THREADS)) return;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(sm + SM_ALPHA + (p0 + p) * 512 + c4 * 4);
-            al[p][0] = a4.x; al[p][1] = a4.y; al[p][2] = a4.z; al[p][3] = a4.w;
-        }
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
+        for (int p = 0; p < 16; ++p) {
+            if (p0 + p >= L) rq[p] = rk[p] = rb[p] = make_uint2(0u, 0u);
 #pragma unroll
             for (int j = 0; j < 4; ++j)   // past the end: alpha = 1; subnormal alpha: smallest normal
                 al[p][j] = p0 + p >= L ? 1.f : fmaxf(al[p][j], 1.17549435e-38f);
-            if (p0 + p >= L) rq[p] = rk[p] = rb[p] = make_uint2(0u, 0u);
         }
-        // log2 of the product of this thread's 8 alphas per channel: sum of the exponent fields plus
+        // log2 of the product of each half's 8 alphas per channel: sum of the exponent fields plus
         // log2 of the product of the mantissas (in [1, 256): cannot under- or overflow)
-        float lw[4];
+        float lw[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int ex = 0;
-            float mp = 1.f;
+        for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const uint32_t u = __float_as_uint(al[p][j]);
-                ex += (int)(u >> 23) - 127;
-                mp *= __uint_as_float((u & 0x7FFFFFu) | 0x3F800000u);
+            for (int j = 0; j < 4; ++j) {
+                int ex = 0;
+                float mp = 1.f;
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const uint32_t u = __float_as_uint(al[8 * hf + p][j]);
+                    ex += (int)(u >> 23) - 127;
+                    mp *= __uint_as_float((u & 0x7FFFFFu) | 0x3F800000u);
+                }
+                lw[hf][j] = (float)ex + fast_log2(mp);
             }
-            lw[j] = (float)ex + fast_log2(mp);
-        }
-        *reinterpret_cast<float4 *>(WT + sw * 128 + c4) = make_float4(lw[0], lw[1], lw[2], lw[3]);
-        if (sw == 0)
+        *reinterpret_cast<float4 *>(WT + w1 * 128 + c4) =
+            make_float4(lw[0][0] + lw[1][0], lw[0][1] + lw[1][1], lw[0][2] + lw[1][2], lw[0][3] + lw[1][3]);
+        if (w1 == 0)
             *reinterpret_cast<float4 *>(v_g0 + c4) = make_float4(fast_log2(al[0][0]), fast_log2(al[0][1]),
                                                                  fast_log2(al[0][2]), fast_log2(al[0][3]));
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
-        if (tid1 == 0) mbar_arrive(mbar(c, MB_AEMPTY));   // the alpha buffer may be refilled
+        group_sync(BAR_BUILD, GROUP);
         float pre[4] = {0.f, 0.f, 0.f, 0.f}, gC[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int w2 = 0; w2 < 8; ++w2) {
+        for (int w2 = 0; w2 < 4; ++w2) {
             const float4 t4 = *reinterpret_cast<const float4 *>(WT + w2 * 128 + c4);
             const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 gC[j] += tv[j];
-                if (w2 < sw) pre[j] += tv[j];
+                if (w2 < w1) pre[j] += tv[j];
             }
         }
         const float4 g04 = *reinterpret_cast<const float4 *>(v_g0 + c4);
@@ -263,19 +428,18 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
         int wide = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) wide |= (g0[j] - gC[j] > SPAN_MAX_LOG2);
-        const bool slow = group_or(BAR_CHUNK, CHUNK_THREADS, wide != 0);   // WT and v_g0 reads done
+        const bool slow = group_or(BAR_BUILD, GROUP, wide != 0);   // WT and v_g0 reads done
         float m2[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) m2[j] = slow ? 0.f : 0.5f * (g0[j] + gC[j]);
 
-        // ---------------------------------------------------------------- wait for the state group
-        // EQ, K̃, [T; P], Delta and the vector slot of chunk n-2 are free once G3 and G4/G5 of
-        // chunk n-1 have completed.
-        if (n > 0) {
-            if (!group_wait(c, mbar(c, MB_G3), par ^ 1u, BAR_CHUNK, CHUNK_THREADS)) return;
-            if (!group_wait(c, mbar(c, MB_G45), par ^ 1u, BAR_CHUNK, CHUNK_THREADS)) return;
+        // ---------------------------------------------------------------- wait for the slot
+        // [Ê; Q̂], K̃ and the vector slot of chunk n-2 are free once its G3 and G4/G5 completed.
+        if (n >= 2) {
+            if (!group_wait(c, mbar_slot(c, MB_G3, n), slot_par(n - 2), BAR_BUILD, GROUP)) return;
+            if (!group_wait(c, mbar_slot(c, MB_G45, n), slot_par(n - 2), BAR_BUILD, GROUP)) return;
         }
-        if (sw == 0) {   // per-channel factors of this chunk for the state group
+        if (w1 == 0) {   // per-channel factors of this chunk for the state group
             // sS: scale of the bf16 state operand of G3 (exp(m)); sZ: scale of the TMEM state that
             // G5 accumulates into; sPost: factor that turns the accumulated Z into the next state.
             // Tensor-core chunk: sS = sZ = exp(m), sPost = exp(g_C - m) (G5 uses K̃).
@@ -291,171 +455,136 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
             *reinterpret_cast<float4 *>(vs + c4) = make_float4(sS[0], sS[1], sS[2], sS[3]);
             *reinterpret_cast<float4 *>(vs + 128 + c4) = make_float4(sZ[0], sZ[1], sZ[2], sZ[3]);
             *reinterpret_cast<float4 *>(vs + 256 + c4) = make_float4(sP[0], sP[1], sP[2], sP[3]);
-            mbar_arrive(mbar(c, MB_VEC));   // 32 arrivals
+            mbar_arrive(mbar_slot(c, MB_VEC, n));   // 32 arrivals
         }
         // ---------------------------------------------------------------- build
         if (!slow) {
-            // exp(g - m) and exp(m - g) at the 8 positions from one exponential at each end of the
-            // thread's span and running products of alpha: exp(g_p - m) = exp(g_(p-1) - m) alpha_p
-            float f1[4], f2[4];
+            // exp(g - m) at each position from one exponential before the thread's first position
+            // and running products of alpha; exp(m - g) backwards from one exponential at the last
+            // position of each half
+            float f1[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                f1[j] = fast_exp2(pre[j] - m2[j]);             // before the first position
-                f2[j] = fast_exp2(m2[j] - (pre[j] + lw[j]));   // at the last position
-            }
+            for (int j = 0; j < 4; ++j) f1[j] = fast_exp2(pre[j] - m2[j]);
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int r = p0 + p;
-                const float2 q01 = unpack2(rq[p].x), q23 = unpack2(rq[p].y);
-                const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
-                const float2 b01 = unpack2(rb[p].x), b23 = unpack2(rb[p].y);
-                const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
-                const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
-                float E[4], Qh[4];
+            for (int hf = 0; hf < 2; ++hf) {
+                // packed bf16 arithmetic: each factor is rounded to bf16 once, each product once
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    f1[j] *= al[p][j];
-                    E[j] = bv[j] * kk[j] * f1[j];
-                    Qh[j] = qq[j] * f1[j];
+                for (int p = 0; p < 8; ++p) {
+                    const int r = p0 + 8 * hf + p, pp = 8 * hf + p;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) f1[j] *= al[pp][j];
+                    const uint32_t F01 = pack_bf16(f1[0], f1[1]), F23 = pack_bf16(f1[2], f1[3]);
+                    *reinterpret_cast<uint2 *>(EQ + sw_off(r, c4, 128)) =
+                        make_uint2(bmul2(bmul2(rb[pp].x, rk[pp].x), F01), bmul2(bmul2(rb[pp].y, rk[pp].y), F23));
+                    *reinterpret_cast<uint2 *>(EQ + sw_off(64 + r, c4, 128)) =
+                        make_uint2(bmul2(rq[pp].x, F01), bmul2(rq[pp].y, F23));
                 }
-                *reinterpret_cast<uint2 *>(sm + SM_EQ + sw_off(r, c4, 128)) =
-                    make_uint2(pack_bf16(E[0], E[1]), pack_bf16(E[2], E[3]));
-                *reinterpret_cast<uint2 *>(sm + SM_EQ + sw_off(64 + r, c4, 128)) =
-                    make_uint2(pack_bf16(Qh[0], Qh[1]), pack_bf16(Qh[2], Qh[3]));
-            }
+                float f2[4];
 #pragma unroll
-            for (int p = 7; p >= 0; --p) {
-                const int r = p0 + p;
-                const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
-                *reinterpret_cast<uint2 *>(sm + SM_KT + sw_off(r, c4, 64)) =
-                    make_uint2(pack_bf16(k01.x * f2[0], k01.y * f2[1]), pack_bf16(k23.x * f2[2], k23.y * f2[3]));
+                for (int j = 0; j < 4; ++j)
+                    f2[j] = fast_exp2(m2[j] - (pre[j] + lw[0][j] + (hf ? lw[1][j] : 0.f)));
 #pragma unroll
-                for (int j = 0; j < 4; ++j) f2[j] *= al[p][j];
+                for (int p = 7; p >= 0; --p) {
+                    const int r = p0 + 8 * hf + p, pp = 8 * hf + p;
+                    *reinterpret_cast<uint2 *>(KT + sw_off(r, c4, 64)) =
+                        make_uint2(bmul2(rk[pp].x, pack_bf16(f2[0], f2[1])), bmul2(rk[pp].y, pack_bf16(f2[2], f2[3])));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) f2[j] *= al[pp][j];
+                }
             }
         } else {
+            // D1 is free once chunk n-1's A and P were read out of it
+            if (n > 0 && !group_wait(c, mbar(c, MB_READOUT), (uint32_t)((n - 1) & 1), BAR_BUILD, GROUP)) return;
             float run[4] = {pre[0], pre[1], pre[2], pre[3]};
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int r = p0 + p;
-                const float2 q01 = unpack2(rq[p].x), q23 = unpack2(rq[p].y);
-                const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
-                const float2 b01 = unpack2(rb[p].x), b23 = unpack2(rb[p].y);
-                const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
-                const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
-                float E[4], Qh[4], Kt[4];
+            for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    run[j] += fast_log2(al[p][j]);
-                    const float gam = exp2f(run[j]);
-                    E[j] = bv[j] * kk[j] * gam;
-                    Qh[j] = qq[j] * gam;
-                    Kt[j] = kk[j] * exp2f(gC[j] - run[j]);
+                for (int p = 0; p < 8; ++p) {
+                    const int r = p0 + 8 * hf + p;
+                    const float2 q01 = unpack2(rq[8 * hf + p].x), q23 = unpack2(rq[8 * hf + p].y);
+                    const float2 k01 = unpack2(rk[8 * hf + p].x), k23 = unpack2(rk[8 * hf + p].y);
+                    const float2 b01 = unpack2(rb[8 * hf + p].x), b23 = unpack2(rb[8 * hf + p].y);
+                    const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
+                    const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
+                    float E[4], Qh[4], Kt[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        run[j] += fast_log2(al[8 * hf + p][j]);
+                        const float gam = exp2f(run[j]);
+                        E[j] = bv[j] * kk[j] * gam;
+                        Qh[j] = qq[j] * gam;
+                        Kt[j] = kk[j] * exp2f(gC[j] - run[j]);
+                    }
+                    *reinterpret_cast<uint2 *>(EQ + sw_off(r, c4, 128)) =
+                        make_uint2(pack_bf16(E[0], E[1]), pack_bf16(E[2], E[3]));
+                    *reinterpret_cast<uint2 *>(EQ + sw_off(64 + r, c4, 128)) =
+                        make_uint2(pack_bf16(Qh[0], Qh[1]), pack_bf16(Qh[2], Qh[3]));
+                    *reinterpret_cast<uint2 *>(KT + sw_off(r, c4, 64)) =
+                        make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
                 }
-                *reinterpret_cast<uint2 *>(sm + SM_EQ + sw_off(r, c4, 128)) =
-                    make_uint2(pack_bf16(E[0], E[1]), pack_bf16(E[2], E[3]));
-                *reinterpret_cast<uint2 *>(sm + SM_EQ + sw_off(64 + r, c4, 128)) =
-                    make_uint2(pack_bf16(Qh[0], Qh[1]), pack_bf16(Qh[2], Qh[3]));
-                *reinterpret_cast<uint2 *>(sm + SM_KT + sw_off(r, c4, 64)) =
-                    make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
-                *reinterpret_cast<float4 *>(G32 + r * 128 + c4) = make_float4(run[0], run[1], run[2], run[3]);
             }
+            wide_span_ap(c, tid1, t0, L);
         }
         fence_async_smem();
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
+        fence_before();
+        group_sync(BAR_BUILD, GROUP);
+        if (tid1 == 0) issue_g1(c, n, slow);
+    }
+}
 
-        // ---------------------------------------------------------------- A (fp32 smem) and P (bf16 tile)
-        if (tid1 == 0) mbar_arrive(mbar(c, MB_BUILD));   // on a wide-span chunk G1 runs but is not read
-        if (!group_wait(c, mbar(c, MB_G1), par, BAR_CHUNK, CHUNK_THREADS)) return;
-        if (!slow) {
-            uint32_t r32[32];
-            tmem_ld32(c.tmem + lrow + TM_D1 + 32 * chalf, r32);
-            wait_ld();
-            if (quarter < 2) {   // rows 0..63: A, strictly lower
-                const int r = crow;
+// ============================================================================ solve group
+// Per chunk: A and P out of TMEM, T = (I + A)^-1, the [T; P] operand tile, then -W' over
+// Ê once G2 has run.  Warp pw of the group reads TMEM lanes 32 pw .. 32 pw + 31 (rows of
+// A for pw < 2, of P for pw >= 2).
+__device__ __forceinline__ void solve_group(const Ctx &c, int tid2) {
+    unsigned char *sm = c.sm;
+    float *AS = reinterpret_cast<float *>(sm + SM_AS);
+    float *XS = reinterpret_cast<float *>(sm + SM_X);
+    const int pw = tid2 >> 5, lane = tid2 & 31;
+    const uint32_t lrow = (uint32_t)(pw * 32) << 16;
+
+    for (int i = tid2; i < 512; i += GROUP)   // T tile: blocks above the diagonal stay zero
+        reinterpret_cast<uint4 *>(sm + SM_T)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int n = 0; n < c.NC; ++n) {
+        unsigned char *EQ = sm + SM_EQ + (n & 1) * EQ_BYTES;
+        // ---------------------------------------------------------------- A (fp32 smem) and P (registers)
+        if (!group_wait(c, mbar(c, MB_G1), (uint32_t)(n & 1), BAR_SOLVE, GROUP)) return;
+        uint32_t ra[32], rb[32];
+        tmem_ld32(c.tmem + lrow + TM_D1, ra);
+        tmem_ld32(c.tmem + lrow + TM_D1 + 32, rb);
+        wait_ld();
+        fence_before();
+        group_sync(BAR_SOLVE, GROUP);
+        if (tid2 == 0) mbar_arrive(mbar(c, MB_READOUT));   // D1 may be overwritten
+        uint32_t pk[32];
+        if (pw < 2) {   // rows 0..63: A, strictly lower
+            const int r = pw * 32 + lane;
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const int col = 32 * chalf + i;
-                    float4 x;
-                    x.x = col < r ? __uint_as_float(r32[i]) : 0.f;
-                    x.y = col + 1 < r ? __uint_as_float(r32[i + 1]) : 0.f;
-                    x.z = col + 2 < r ? __uint_as_float(r32[i + 2]) : 0.f;
-                    x.w = col + 3 < r ? __uint_as_float(r32[i + 3]) : 0.f;
-                    *reinterpret_cast<float4 *>(AS + r * LDA + col) = x;
-                }
-            } else {             // rows 64..127: P, lower with diagonal -> bf16 tile
-                const int r = crow - 64;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int c0 = 32 * chalf + 8 * u + 2 * i;
-                        const float x0 = c0 <= r ? __uint_as_float(r32[8 * u + 2 * i]) : 0.f;
-                        const float x1 = c0 + 1 <= r ? __uint_as_float(r32[8 * u + 2 * i + 1]) : 0.f;
-                        pk[i] = pack_bf16(x0, x1);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + SM_P + sw_off(r, 32 * chalf + 8 * u, 64)) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
+            for (int i = 0; i < 64; i += 4) {
+                const uint32_t *src = i < 32 ? ra + i : rb + (i - 32);
+                float4 x;
+                x.x = i < r ? __uint_as_float(src[0]) : 0.f;
+                x.y = i + 1 < r ? __uint_as_float(src[1]) : 0.f;
+                x.z = i + 2 < r ? __uint_as_float(src[2]) : 0.f;
+                x.w = i + 3 < r ? __uint_as_float(src[3]) : 0.f;
+                *reinterpret_cast<float4 *>(AS + r * LDA + i) = x;
             }
-        } else {
-            // wide-span chunk: A_ri = sum_c e_rc k_ic 2^(g_rc - g_ic) (i < r), P (i <= r) on CUDA cores;
-            // raw tokens are re-read from global memory (resident in L2), P goes through TF first.
-            for (int r = sw; r < 64; r += 8) {
-                const bool rv_ok = r < L;
-                float er[4], qr[4], gr[4];
-                const size_t rowr = ((size_t)bb * T + t0 + r) * H + h;
+        } else {        // rows 64..127: P, lower with the diagonal, kept packed until its tile is free
+            const int r = (pw - 2) * 32 + lane;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int cc = lane + 32 * u;
-                    er[u] = rv_ok ? __bfloat162float(c.b[rowr * KD + cc]) * __bfloat162float(c.k[rowr * KD + cc]) : 0.f;
-                    qr[u] = rv_ok ? __bfloat162float(c.q[rowr * KD + cc]) : 0.f;
-                    gr[u] = G32[r * 128 + cc];
-                }
-                for (int i = 0; i < 64; ++i) {
-                    float a = 0.f, pp = 0.f;
-                    if (i <= r && i < L) {
-                        const size_t rowi = ((size_t)bb * T + t0 + i) * H + h;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int cc = lane + 32 * u;
-                            const float kd = __bfloat162float(c.k[rowi * KD + cc]) * exp2f(gr[u] - G32[i * 128 + cc]);
-                            a += er[u] * kd;
-                            pp += qr[u] * kd;
-                        }
-#pragma unroll
-                        for (int msk = 16; msk > 0; msk >>= 1) {
-                            a += __shfl_xor_sync(0xffffffffu, a, msk);
-                            pp += __shfl_xor_sync(0xffffffffu, pp, msk);
-                        }
-                    }
-                    if (lane == 0) {
-                        AS[r * LDA + i] = i < r ? a : 0.f;
-                        TF[r * LDA + i] = i <= r ? pp : 0.f;
-                    }
-                }
-            }
-            group_sync(BAR_CHUNK, CHUNK_THREADS);
-            {
-                const int r = tid1 >> 2, i0 = 16 * (tid1 & 3);
-                uint32_t pk[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(TF[r * LDA + i0 + 2 * i], TF[r * LDA + i0 + 2 * i + 1]);
-                *reinterpret_cast<uint4 *>(sm + SM_P + sw_off(r, i0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4 *>(sm + SM_P + sw_off(r, i0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            for (int i = 0; i < 32; ++i) {
+                const int c0 = 2 * i;
+                const uint32_t *src = c0 < 32 ? ra + c0 : rb + (c0 - 32);
+                pk[i] = pack_bf16(c0 <= r ? __uint_as_float(src[0]) : 0.f, c0 + 1 <= r ? __uint_as_float(src[1]) : 0.f);
             }
         }
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
+        group_sync(BAR_SOLVE, GROUP);
 
         // ---------------------------------------------------------------- T = (I + A)^-1
-        // The bf16 tile is written block by block as T is formed; its blocks above the diagonal
-        // stay zero (set once, and again after a wide-span chunk reused the space).
-        if (slow) {
-            for (int i = tid1; i < 512; i += CHUNK_THREADS)
-                reinterpret_cast<uint4 *>(sm + SM_T)[i] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (tid1 < 64) {   // diagonal 16x16 blocks, one column per thread
-            const int J = tid1 >> 4, j = tid1 & 15, o16 = 16 * J;
+        // The bf16 T tile is written block by block as T is formed (G2 of the previous chunk,
+        // its reader, has completed); its blocks above the diagonal stay zero.
+        if (tid2 < 64) {   // diagonal 16x16 blocks, one column per thread
+            const int J = tid2 >> 4, j = tid2 & 15, o16 = 16 * J;
             float col[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
@@ -475,102 +604,107 @@ __device__ void chunk_group(const Ctx &c, int tid1) {
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                TF[(o16 + r) * LDA + o16 + j] = col[r];
+                if (r >= j) AS[(o16 + j) * LDA + o16 + r] = col[r];   // T^T, on and above the diagonal
                 *reinterpret_cast<__nv_bfloat16 *>(sm + SM_T + sw_off(o16 + r, o16 + j, 64)) = __float2bfloat16_rn(col[r]);
             }
         }
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
-        if (sw < 2) {   // blocks (1,0) and (3,2): T_RI = -T_RR (A_RI T_II), within one warp
-            const int R = 16 * (2 * sw + 1), I = 16 * (2 * sw);
-            float *X = WT + sw * 384;   // 16 x 16 (row stride 24), private to this warp
+        group_sync(BAR_SOLVE, GROUP);
+        if (pw < 2) {   // blocks (1,0) and (3,2): T_RI = -T_RR (A_RI T_II), within one warp
+            const int R = 16 * (2 * pw + 1), I = 16 * (2 * pw);
+            float *X = XS + pw * 384;   // 16 x 16 (row stride 24), private to this warp
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, AS, LDA, R, I, TF, LDA, I, I + 8 * nt, 0, 2, lane);
+                tile_mm_tb(d, AS, LDA, R, I, AS, I, I + 8 * nt, 0, 2, lane);
                 tile_store(X, 24, 0, 8 * nt, d, 1.f, lane);
             }
             __syncwarp();
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, TF, LDA, R, R, X, 24, 0, 8 * nt, 0, 2, lane);
-                tile_store(TF, LDA, R, I + 8 * nt, d, -1.f, lane);
+                tile_mm_ta(d, AS, R, R, X, 24, 0, 8 * nt, 0, 2, lane);
+                tile_store_t(AS, R, I + 8 * nt, d, -1.f, lane);
                 tile_store_bf16(sm + SM_T, R, I + 8 * nt, d, -1.f, lane);
             }
         }
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
-        if (sw < 4) {   // rows 32..63 x cols 8sw..8sw+7: T = -T_hi (A_hi,lo T_lo), within one warp
-            const int nt = sw;
-            float *X = WT + sw * 256;   // 32 x 8, private to this warp
+        group_sync(BAR_SOLVE, GROUP);
+        {   // rows 32..63 x cols 8pw..8pw+7: T = -T_hi (A_hi,lo T_lo), within one warp
+            const int nt = pw;
+            float *X = XS + pw * 256;   // 32 x 8, private to this warp
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {   // block (0,1) of T is zero: skipped for columns >= 16
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, AS, LDA, 32 + 16 * mt, 0, TF, LDA, 0, 8 * nt, nt >= 2 ? 2 : 0, 4, lane);
+                tile_mm_tb(d, AS, LDA, 32 + 16 * mt, 0, AS, 0, 8 * nt, nt >= 2 ? 2 : 0, 4, lane);
                 tile_store(X, 8, 16 * mt, 0, d, 1.f, lane);
             }
             __syncwarp();
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {   // block (2,3) of T is zero: skipped for rows < 48
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mm(d, TF, LDA, 32 + 16 * mt, 32, X, 8, 0, 0, 0, mt == 0 ? 2 : 4, lane);
+                tile_mm_ta(d, AS, 32 + 16 * mt, 32, X, 8, 0, 0, 0, mt == 0 ? 2 : 4, lane);
                 tile_store_bf16(sm + SM_T, 32 + 16 * mt, 8 * nt, d, -1.f, lane);
             }
         }
+        // ---------------------------------------------------------------- P tile (after G4 of chunk n-1)
+        if (n > 0 && !group_wait(c, mbar_slot(c, MB_G45, n - 1), slot_par(n - 1), BAR_SOLVE, GROUP)) return;
+        if (pw >= 2) {
+            const int r = (pw - 2) * 32 + lane;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4 *>(sm + SM_P + sw_off(r, 8 * u, 64)) =
+                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
         fence_async_smem();
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
-        if (tid1 == 0) mbar_arrive(mbar(c, MB_SOLVE));
+        group_sync(BAR_SOLVE, GROUP);
+        if (tid2 == 0) issue_g2(c, n);
 
         // ---------------------------------------------------------------- -W' over Ê; zero the O rows of D3
-        if (!group_wait(c, mbar(c, MB_G2), par, BAR_CHUNK, CHUNK_THREADS)) return;
-        if (quarter < 2) {
-            const int r = crow;
+        if (!group_wait(c, mbar_slot(c, MB_G2, n), slot_par(n), BAR_SOLVE, GROUP)) return;
+        if (pw < 2) {
+            const int r = pw * 32 + lane;
 #pragma unroll
-            for (int u2 = 0; u2 < 2; ++u2) {
+            for (int u2 = 0; u2 < 4; ++u2) {
                 uint32_t r32[32];
-                tmem_ld32(c.tmem + lrow + TM_D2 + 64 * chalf + 32 * u2, r32);
+                tmem_ld32(c.tmem + lrow + TM_D2 + 32 * u2, r32);
                 wait_ld();
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int cc = 64 * chalf + 32 * u2 + 8 * u;
-                    uint32_t pk[4];
+                    const int cc = 32 * u2 + 8 * u;
+                    uint32_t q4[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        pk[i] = pack_bf16(-__uint_as_float(r32[8 * u + 2 * i]), -__uint_as_float(r32[8 * u + 2 * i + 1]));
-                    *reinterpret_cast<uint4 *>(sm + SM_EQ + sw_off(r, cc, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        q4[i] = pack_bf16(-__uint_as_float(r32[8 * u + 2 * i]), -__uint_as_float(r32[8 * u + 2 * i + 1]));
+                    *reinterpret_cast<uint4 *>(EQ + sw_off(r, cc, 128)) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
                 }
             }
         } else {
             uint32_t z[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) z[i] = 0u;
-            const uint32_t d3 = TM_D3 + 128 * (n & 1);
-            tmem_st32(c.tmem + lrow + d3 + 64 * chalf, z);
-            tmem_st32(c.tmem + lrow + d3 + 64 * chalf + 32, z);
+#pragma unroll
+            for (int u2 = 0; u2 < 4; ++u2) tmem_st32(c.tmem + lrow + TM_D3 + 32 * u2, z);
             wait_st();
         }
         fence_async_smem();
         fence_before();
-        group_sync(BAR_CHUNK, CHUNK_THREADS);
-        if (tid1 == 0) mbar_arrive(mbar(c, MB_S1DONE));
+        group_sync(BAR_SOLVE, GROUP);
+        if (tid2 == 0) mbar_arrive(mbar(c, MB_S1DONE));
     }
 }
 
 // ============================================================================ state group
-__device__ void state_group(const Ctx &c, int tid, float *ST, size_t chain) {
+__device__ __forceinline__ void state_group(const Ctx &c, int tid, float *ST, size_t chain) {
     unsigned char *sm = c.sm;
     const float *vec = reinterpret_cast<const float *>(sm + SM_VEC);
     const int warp = tid >> 5;
     const uint32_t lrow = (uint32_t)(warp * 32) << 16;
     const int crow = tid;   // TMEM lane = row c of Z (and row r of D3)
-    const int T = c.T, H = c.H;
     float egm_prev = 1.f;
 
     for (int n = 0; n < c.NC; ++n) {
-        const uint32_t par = (uint32_t)(n & 1);
-        const int t0 = n * C, L = min(C, T - t0);
         // ---------------------------------------------------------------- S_n = sPost_n-1 Z; Z <- sZ_n S_n; bf16(sS_n S_n)
-        if (!group_wait(c, mbar(c, MB_VEC), par, BAR_STATE, STATE_THREADS)) return;
-        if (n > 0 && !group_wait(c, mbar(c, MB_G45), par ^ 1u, BAR_STATE, STATE_THREADS)) return;
+        if (!group_wait(c, mbar_slot(c, MB_VEC, n), slot_par(n), BAR_STATE, GROUP)) return;
+        if (n > 0 && !group_wait(c, mbar_slot(c, MB_G45, n - 1), slot_par(n - 1), BAR_STATE, GROUP)) return;
         const float *vs = vec + (n & 1) * 384;
         const float ssc = vs[crow] * egm_prev;         // scale of the bf16 operand
         const float zsc = vs[128 + crow] * egm_prev;   // scale of the TMEM state
@@ -598,17 +732,16 @@ __device__ void state_group(const Ctx &c, int tid, float *ST, size_t chain) {
         wait_st();
         fence_async_smem();
         fence_before();
-        group_sync(BAR_STATE, STATE_THREADS);
-        if (tid == 0) mbar_arrive(mbar(c, MB_STILDE));
+        group_sync(BAR_STATE, GROUP);
+        if (tid == 0) issue_g3(c, n);
 
         // ---------------------------------------------------------------- Delta rows -> bf16 tile
-        if (!group_wait(c, mbar(c, MB_G3), par, BAR_STATE, STATE_THREADS)) return;
-        const uint32_t d3 = TM_D3 + 128 * (n & 1);
+        if (!group_wait(c, mbar_slot(c, MB_G3, n), slot_par(n), BAR_STATE, GROUP)) return;
         if (warp < 2) {
 #pragma unroll
             for (int u2 = 0; u2 < 4; ++u2) {
                 uint32_t r32[32];
-                tmem_ld32(c.tmem + lrow + d3 + 32 * u2, r32);
+                tmem_ld32(c.tmem + lrow + TM_D3 + 32 * u2, r32);
                 wait_ld();
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -624,36 +757,11 @@ __device__ void state_group(const Ctx &c, int tid, float *ST, size_t chain) {
         }
         fence_async_smem();
         fence_before();
-        group_sync(BAR_STATE, STATE_THREADS);
-        if (tid == 0) mbar_arrive(mbar(c, MB_DELTA));
-
-        // ---------------------------------------------------------------- o rows (16-byte stores)
-        if (!group_wait(c, mbar(c, MB_G45), par, BAR_STATE, STATE_THREADS)) return;
-        if (warp >= 2) {
-            const int r = crow - 64;
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-                uint32_t r32[32];
-                tmem_ld32(c.tmem + lrow + d3 + 32 * u2, r32);
-                wait_ld();
-                if (r < L) {
-                    __nv_bfloat16 *dst = c.o + (((size_t)c.bb * T + t0 + r) * H + c.h) * VD + 32 * u2;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        uint4 pk;
-                        pk.x = pack_bf16(__uint_as_float(r32[8 * u]), __uint_as_float(r32[8 * u + 1]));
-                        pk.y = pack_bf16(__uint_as_float(r32[8 * u + 2]), __uint_as_float(r32[8 * u + 3]));
-                        pk.z = pack_bf16(__uint_as_float(r32[8 * u + 4]), __uint_as_float(r32[8 * u + 5]));
-                        pk.w = pack_bf16(__uint_as_float(r32[8 * u + 6]), __uint_as_float(r32[8 * u + 7]));
-                        *reinterpret_cast<uint4 *>(dst + 8 * u) = pk;
-                    }
-                }
-            }
-        }
-        fence_before();
-        group_sync(BAR_STATE, STATE_THREADS);
-        if (tid == 0) mbar_arrive(mbar(c, (n & 1) ? MB_D3FREE1 : MB_D3FREE0));
+        group_sync(BAR_STATE, GROUP);
+        if (tid == 0) issue_g45(c, n);
     }
+    // the last chunk's G4/G5 must be complete before Z is read
+    if (!group_wait(c, mbar_slot(c, MB_G45, c.NC - 1), slot_par(c.NC - 1), BAR_STATE, GROUP)) return;
     // S_T = Diag(sPost) Z of the last chunk
     float *dst = ST + (chain * KD + crow) * VD;
 #pragma unroll
@@ -669,48 +777,29 @@ __device__ void state_group(const Ctx &c, int tid, float *ST, size_t chain) {
     }
 }
 
-// ============================================================================ producer
-// Stages alpha of chunk n into shared memory (bulk copies completing on MB_AFULL) once the
-// chunk group has consumed chunk n-1's.
-__device__ void producer(const Ctx &c, int lane) {
-    const uint32_t dst = smem_u32(c.sm + SM_ALPHA);
-    const int T = c.T, H = c.H, bb = c.bb, h = c.h;
-    for (int n = 0; n < c.NC; ++n) {
-        const int t0 = n * C, L = min(C, T - t0);
-        if (n > 0) {
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(mbar(c, MB_AEMPTY), (uint32_t)((n - 1) & 1), WAIT_LIMIT) && !*abort_flag(c);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) {
-                if (lane == 0) *abort_flag(c) = 1u;
-                return;
-            }
-        }
-        if (lane == 0) mbar_arrive_expect_tx(mbar(c, MB_AFULL), (uint32_t)L * 512u);
-        __syncwarp();
-        for (int r = lane; r < L; r += 32)   // one 512-byte row per copy, spread over the warp
-            bulk_g2s(dst + (uint32_t)r * 512u, c.alpha + (((size_t)bb * T + t0 + r) * H + h) * KD, 512u,
-                     mbar(c, MB_AFULL));
+// ============================================================================ value and o groups
+// u group (warps 12-13): U = w ⊙ v of chunk n into slot n & 1, written once G2 of chunk n-2
+// (the slot's last reader) has completed; signals MB_U of the slot (64 arrivals).  Lane l
+// holds channels 4l..4l+3, the warp picks 32 positions; rows past the end are zero.
+// o group (warps 14-15, TMEM lanes 64-127 = the O rows of D3): the o rows of chunk n once
+// its G4 has completed; signals MB_D3FREE (64 arrivals).
+__device__ __forceinline__ bool warp_wait(const Ctx &c, uint32_t mb, uint32_t parity) {
+    const bool ok = mbar_wait(mb, parity, WAIT_LIMIT) && !*abort_flag(c);
+    if (!__all_sync(0xffffffffu, ok)) {
+        *abort_flag(c) = 1u;
+        return false;
     }
+    fence_after();
+    return true;
 }
 
-// ============================================================================ value group
-// U = w ⊙ v of chunk n, written once G2 of chunk n-1 (its last reader) has completed;
-// signals MB_U (64 arrivals).  Warps 14-15: lane l holds channels 4l..4l+3, warp half
-// picks positions; rows past the end of the sequence are zero.
-__device__ void value_group(const Ctx &c, int tid2) {
+__device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
     const int vw = tid2 >> 5, lane = tid2 & 31, c4 = lane * 4;
     const int T = c.T, H = c.H, bb = c.bb, h = c.h;
     for (int n = 0; n < c.NC; ++n) {
         const int t0 = n * C, L = min(C, T - t0);
-        if (n > 0) {
-            bool ok = mbar_wait(mbar(c, MB_G2), (uint32_t)((n - 1) & 1), WAIT_LIMIT) && !*abort_flag(c);
-            if (!__all_sync(0xffffffffu, ok)) {
-                *abort_flag(c) = 1u;
-                return;
-            }
-            fence_after();
-        }
+        unsigned char *U = c.sm + SM_U + (n & 1) * U_BYTES;
+        if (n >= 2 && !warp_wait(c, mbar_slot(c, MB_G2, n), slot_par(n - 2))) return;
 #pragma unroll 1
         for (int p0 = 32 * vw; p0 < 32 * vw + 32; p0 += 8) {
             uint2 rv[8], rw[8];
@@ -722,86 +811,45 @@ __device__ void value_group(const Ctx &c, int tid2) {
                 rw[p] = __ldg(reinterpret_cast<const uint2 *>(c.w + row * VD + c4));
             }
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const float2 v01 = unpack2(rv[p].x), v23 = unpack2(rv[p].y);
-                const float2 w01 = unpack2(rw[p].x), w23 = unpack2(rw[p].y);
-                const bool ok = p0 + p < L;
-                *reinterpret_cast<uint2 *>(c.sm + SM_U + sw_off(p0 + p, c4, 64)) =
-                    ok ? make_uint2(pack_bf16(w01.x * v01.x, w01.y * v01.y), pack_bf16(w23.x * v23.x, w23.y * v23.y))
-                       : make_uint2(0u, 0u);
-            }
+            for (int p = 0; p < 8; ++p)
+                *reinterpret_cast<uint2 *>(U + sw_off(p0 + p, c4, 64)) =
+                    p0 + p < L ? make_uint2(bmul2(rw[p].x, rv[p].x), bmul2(rw[p].y, rv[p].y)) : make_uint2(0u, 0u);
         }
         fence_async_smem();
-        mbar_arrive(mbar(c, MB_U));
+        mbar_arrive(mbar_slot(c, MB_U, n));
     }
 }
 
-// ============================================================================ MMA issuer
-__device__ void mma_issuer(const Ctx &c) {
-    const uint32_t aS = smem_u32(c.sm + SM_S), aEQ = smem_u32(c.sm + SM_EQ), aKT = smem_u32(c.sm + SM_KT),
-                   aU = smem_u32(c.sm + SM_U), aDL = smem_u32(c.sm + SM_DL), aTP = smem_u32(c.sm + SM_T);
-    const uint32_t tm = c.tmem;
-    int i1 = 0, i2 = 0, i3 = 0, i45 = 0;
-    uint32_t idle = 0;
-    while (i45 < c.NC) {
-        bool did = false;
-        if (i1 < c.NC && mbar_test(mbar(c, MB_BUILD), (uint32_t)(i1 & 1))) {
-            fence_after();
+__device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
+    const int r = tid2;   // row of O = TMEM lane 64 + r
+    const uint32_t lrow = (uint32_t)(64 + (tid2 >> 5) * 32) << 16;
+    for (int n = 0; n < c.NC; ++n) {
+        const int t0 = n * C, L = min(C, c.T - t0);
+        if (!warp_wait(c, mbar_slot(c, MB_G45, n), slot_par(n))) return;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                mma_ss(tm + TM_D1, desc_kmajor(aEQ, 128, j), desc_kmajor(aKT, 64, j), ID_G1, j > 0);
-            mma_commit(mbar(c, MB_G1));
-            ++i1;
-            did = true;
+        for (int u2 = 0; u2 < 4; ++u2) {
+            uint32_t r32[32];
+            tmem_ld32(c.tmem + lrow + TM_D3 + 32 * u2, r32);
+            wait_ld();
+            if (r < L) {
+                __nv_bfloat16 *dst = c.o + (((size_t)c.bb * c.T + t0 + r) * c.H + c.h) * VD + 32 * u2;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 pk;
+                    pk.x = pack_bf16(__uint_as_float(r32[8 * u]), __uint_as_float(r32[8 * u + 1]));
+                    pk.y = pack_bf16(__uint_as_float(r32[8 * u + 2]), __uint_as_float(r32[8 * u + 3]));
+                    pk.z = pack_bf16(__uint_as_float(r32[8 * u + 4]), __uint_as_float(r32[8 * u + 5]));
+                    pk.w = pack_bf16(__uint_as_float(r32[8 * u + 6]), __uint_as_float(r32[8 * u + 7]));
+                    *reinterpret_cast<uint4 *>(dst + 8 * u) = pk;
+                }
+            }
         }
-        if (i2 < i1 && mbar_test(mbar(c, MB_SOLVE), (uint32_t)(i2 & 1)) && mbar_test(mbar(c, MB_U), (uint32_t)(i2 & 1)) &&
-            (i2 < 2 || mbar_test(mbar(c, (i2 & 1) ? MB_D3FREE1 : MB_D3FREE0), (uint32_t)(((i2 - 2) >> 1) & 1)))) {
-            fence_after();
-            const uint32_t d3 = TM_D3 + 128 * (i2 & 1);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_ss(tm + TM_D2, desc_kmajor(aTP, 128, j), desc_mnmajor(aEQ, 128, j), ID_G2, j > 0);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_ss(tm + d3, desc_kmajor(aTP, 128, j), desc_mnmajor(aU, 64, j), ID_G2, j > 0);
-            mma_commit(mbar(c, MB_G2));
-            ++i2;
-            did = true;
-        }
-        if (i3 < i2 && mbar_test(mbar(c, MB_S1DONE), (uint32_t)(i3 & 1)) &&
-            mbar_test(mbar(c, MB_STILDE), (uint32_t)(i3 & 1))) {
-            fence_after();
-            const uint32_t d3 = TM_D3 + 128 * (i3 & 1);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                mma_ss(tm + d3, desc_kmajor(aEQ, 128, j), desc_mnmajor(aS, 128, j), ID_G3, 1);
-            mma_commit(mbar(c, MB_G3));
-            ++i3;
-            did = true;
-        }
-        if (i45 < i3 && mbar_test(mbar(c, MB_DELTA), (uint32_t)(i45 & 1))) {
-            fence_after();
-            const uint32_t d3 = TM_D3 + 128 * (i45 & 1);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_ss(tm + d3, desc_kmajor(aTP, 128, j), desc_mnmajor(aDL, 64, j), ID_G4, 1);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_ss(tm + TM_Z, desc_mnmajor(aKT, 64, j), desc_mnmajor(aDL, 64, j), ID_G5, 1);
-            mma_commit(mbar(c, MB_G45));
-            ++i45;
-            did = true;
-        }
-        if (did) {
-            idle = 0;
-        } else if (++idle > POLL_LIMIT || *abort_flag(c)) {
-            *abort_flag(c) = 1u;
-            return;
-        }
+        fence_before();
+        mbar_arrive(mbar(c, MB_D3FREE));
     }
 }
 
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ alpha,
                     const __nv_bfloat16 *__restrict__ b, const __nv_bfloat16 *__restrict__ w,
@@ -819,8 +867,9 @@ __global__ void __launch_bounds__(NT)
 
     if (warp == 12) tmem_alloc(c.misc + MISC_TSLOT, TM_COLS);
     if (tid == 0) {
-        for (uint32_t i = 0; i < MB_COUNT; ++i)
-            mbar_init(c.misc + 8 * i, i * 8 == MB_VEC ? 32u : i * 8 == MB_U ? 64u : 1u);
+        for (uint32_t off = 0; off < MB_END; off += 8)
+            mbar_init(c.misc + off, (off == MB_VEC || off == MB_VEC + 8) ? 32u
+                                     : (off == MB_U || off == MB_U + 8 || off == MB_D3FREE) ? 64u : 1u);
         *reinterpret_cast<volatile uint32_t *>(sm + SM_MISC + MISC_ABORT) = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -830,7 +879,7 @@ __global__ void __launch_bounds__(NT)
     c.tmem = *reinterpret_cast<volatile uint32_t *>(sm + SM_MISC + MISC_TSLOT);
 
     if (warp < 4) {   // Z <- S0 (the first rescale multiplies by exp(m) of chunk 0)
-        regs_dec<56>();
+        regs_dec<104>();
         const int crow = tid;
         const uint32_t lrow = (uint32_t)(warp * 32) << 16;
         const float *src = S0 ? S0 + ((size_t)chain * KD + crow) * VD : nullptr;
@@ -847,17 +896,25 @@ __global__ void __launch_bounds__(NT)
         }
         wait_st();
         fence_before();
-        group_sync(BAR_STATE, STATE_THREADS);
+        group_sync(BAR_STATE, GROUP);
         fence_after();
         state_group(c, tid, ST, (size_t)chain);
+        regs_inc<128>();   // every warpgroup leaves its role with the launch budget
+    } else if (warp < 8) {
+        regs_inc<208>();
+        build_group(c, tid - 128);
+        regs_dec<128>();
     } else if (warp < 12) {
-        regs_inc<200>();
-        chunk_group(c, tid - 128);
+        regs_inc<128>();
+        solve_group(c, tid - 256);
+        regs_dec<128>();
     } else {
-        regs_dec<56>();
-        if (warp == 12 && (tid & 31) == 0) mma_issuer(c);
-        if (warp == 13) producer(c, tid & 31);
-        if (warp >= 14) value_group(c, tid - 448);
+        regs_dec<72>();
+        if (warp < 14)
+            u_group(c, tid - 384);
+        else
+            o_group(c, tid - 448);
+        regs_inc<128>();
     }
 
     fence_before();
