@@ -584,23 +584,19 @@ __device__ __forceinline__ void solve_group(const Ctx &c, int tid2) {
         // The bf16 T tile is written block by block as T is formed (G2 of the previous chunk,
         // its reader, has completed); its blocks above the diagonal stay zero.
         if (tid2 < 64) {   // diagonal 16x16 blocks, one column per thread
+            // column-oriented substitution: as soon as T[i][j] is known its contribution is
+            // subtracted from every later row, so the dependent chain is one FMA per row
             const int J = tid2 >> 4, j = tid2 & 15, o16 = 16 * J;
-            float col[16];
+            const float *Ab = AS + o16 * LDA + o16;
+            float nacc[16], col[16];   // nacc[r] = -sum_{i<r} A[r][i] T[i][j]
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == j) ? 1.f : 0.f;
-                if (r > j) {
-                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            for (int r = 0; r < 16; ++r) nacc[r] = 0.f;
 #pragma unroll
-                    for (int i = 0; i < r; i += 4) {
-                        s0 += AS[(o16 + r) * LDA + o16 + i] * col[i];
-                        if (i + 1 < r) s1 += AS[(o16 + r) * LDA + o16 + i + 1] * col[i + 1];
-                        if (i + 2 < r) s2 += AS[(o16 + r) * LDA + o16 + i + 2] * col[i + 2];
-                        if (i + 3 < r) s3 += AS[(o16 + r) * LDA + o16 + i + 3] * col[i + 3];
-                    }
-                    acc = -((s0 + s1) + (s2 + s3));
-                }
-                col[r] = acc;
+            for (int i = 0; i < 16; ++i) {
+                const float t = i == j ? 1.f : (i < j ? 0.f : nacc[i]);
+                col[i] = t;
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) nacc[r] = fmaf(-Ab[r * LDA + i], t, nacc[r]);
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
@@ -663,17 +659,19 @@ __device__ __forceinline__ void solve_group(const Ctx &c, int tid2) {
         if (pw < 2) {
             const int r = pw * 32 + lane;
 #pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-                uint32_t r32[32];
-                tmem_ld32(c.tmem + lrow + TM_D2 + 32 * u2, r32);
+            for (int u2 = 0; u2 < 4; u2 += 2) {
+                uint32_t r32[2][32];
+                tmem_ld32(c.tmem + lrow + TM_D2 + 32 * u2, r32[0]);
+                tmem_ld32(c.tmem + lrow + TM_D2 + 32 * u2 + 32, r32[1]);
                 wait_ld();
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 8; ++u) {
                     const int cc = 32 * u2 + 8 * u;
+                    const uint32_t *x = r32[u >> 2] + 8 * (u & 3);
                     uint32_t q4[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        q4[i] = pack_bf16(-__uint_as_float(r32[8 * u + 2 * i]), -__uint_as_float(r32[8 * u + 2 * i + 1]));
+                        q4[i] = pack_bf16(-__uint_as_float(x[2 * i]), -__uint_as_float(x[2 * i + 1]));
                     *reinterpret_cast<uint4 *>(EQ + sw_off(r, cc, 128)) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
                 }
             }
