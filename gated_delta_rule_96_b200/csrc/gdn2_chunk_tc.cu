@@ -84,7 +84,8 @@ constexpr uint32_t SM_VEC = SM_AS + 64 * LDA * 4; // [2 slots][sS, sZ, sPost] (6
 constexpr uint32_t SM_WT = SM_VEC + 3072;         // build group: [4][128] warp totals + g_0 [128]
 constexpr uint32_t SM_X = SM_WT + 2560;           // solve group: per-warp mma scratch (4 KB)
 constexpr uint32_t SM_MISC = SM_X + 4096;         // mbarriers, TMEM slot, flags
-constexpr uint32_t SM_BYTES = SM_MISC + 256 + 1024;
+constexpr uint32_t SM_OST = SM_MISC + 256;         // o group: 2 warps x 32 rows x 80 B staging
+constexpr uint32_t SM_BYTES = SM_OST + 5120 + 1024;
 
 // mbarriers (byte offsets inside SM_MISC); the first five are pairs indexed by chunk & 1
 enum : uint32_t {
@@ -121,11 +122,9 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
     return *reinterpret_cast<uint32_t *>(&r);
 }
-__device__ __forceinline__ uint32_t tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+// tf32 operand of mma.sync: the fp32 bit pattern (the tensor core reads the top 19 bits, i.e.
+// truncates the mantissa to 10 bits; T ends up in bf16, far coarser)
+__device__ __forceinline__ uint32_t tf32(float x) { return __float_as_uint(x); }
 // D(16x8) += A(16x8) B(8x8), tf32 inputs, fp32 accumulate (warp-level)
 __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -381,6 +380,16 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
             rq[p] = __ldg(reinterpret_cast<const uint2 *>(c.q + row * KD + c4));
             rk[p] = __ldg(reinterpret_cast<const uint2 *>(c.k + row * KD + c4));
             rb[p] = __ldg(reinterpret_cast<const uint2 *>(c.b + row * KD + c4));
+        }
+        if (n + 1 < c.NC) {   // next chunk's rows of q, k, b, alpha into L2 (one 128-B line per request)
+            const int r = tid1 & 63, half = tid1 >> 6;
+            const int t = min(r, T - t0 - C - 1);
+            const size_t row = ((size_t)bb * T + t0 + C + t) * H + h;
+            const char *base[3] = {(const char *)(c.q + row * KD), (const char *)(c.k + row * KD), (const char *)(c.b + row * KD)};
+#pragma unroll
+            for (int i = 0; i < 3; ++i) prefetch_l2(base[i] + 128 * half);
+            prefetch_l2((const char *)(c.alpha + row * KD) + 256 * half);
+            prefetch_l2((const char *)(c.alpha + row * KD) + 256 * half + 128);
         }
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
@@ -780,7 +789,8 @@ __device__ __forceinline__ void state_group(const Ctx &c, int tid, float *ST, si
 // (the slot's last reader) has completed; signals MB_U of the slot (64 arrivals).  Lane l
 // holds channels 4l..4l+3, the warp picks 32 positions; rows past the end are zero.
 // o group (warps 14-15, TMEM lanes 64-127 = the O rows of D3): the o rows of chunk n once
-// its G4 has completed; signals MB_D3FREE (64 arrivals).
+// its G4 has completed, transposed through shared memory so that each store instruction
+// writes 8 rows x 64 B; signals MB_D3FREE (64 arrivals).
 __device__ __forceinline__ bool warp_wait(const Ctx &c, uint32_t mb, uint32_t parity) {
     const bool ok = mbar_wait(mb, parity, WAIT_LIMIT) && !*abort_flag(c);
     if (!__all_sync(0xffffffffu, ok)) {
@@ -797,6 +807,15 @@ __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
     for (int n = 0; n < c.NC; ++n) {
         const int t0 = n * C, L = min(C, T - t0);
         unsigned char *U = c.sm + SM_U + (n & 1) * U_BYTES;
+        if (n + 1 < c.NC) {   // next chunk's rows of v and w into L2
+            const int t = min(tid2, T - t0 - C - 1);
+            const size_t row = ((size_t)bb * T + t0 + C + t) * H + h;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                prefetch_l2((const char *)(c.v + row * VD) + 128 * i);
+                prefetch_l2((const char *)(c.w + row * VD) + 128 * i);
+            }
+        }
         if (n >= 2 && !warp_wait(c, mbar_slot(c, MB_G2, n), slot_par(n - 2))) return;
 #pragma unroll 1
         for (int p0 = 32 * vw; p0 < 32 * vw + 32; p0 += 8) {
@@ -819,8 +838,9 @@ __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
 }
 
 __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
-    const int r = tid2;   // row of O = TMEM lane 64 + r
-    const uint32_t lrow = (uint32_t)(64 + (tid2 >> 5) * 32) << 16;
+    const int ow = tid2 >> 5, lane = tid2 & 31;   // this thread's row of O: TMEM lane 64 + tid2
+    const uint32_t lrow = (uint32_t)(64 + ow * 32) << 16;
+    unsigned char *stg = c.sm + SM_OST + ow * 2560;   // 32 rows x 80 B (64 B of data + 16 B pad)
     for (int n = 0; n < c.NC; ++n) {
         const int t0 = n * C, L = min(C, c.T - t0);
         if (!warp_wait(c, mbar_slot(c, MB_G45, n), slot_par(n))) return;
@@ -829,18 +849,24 @@ __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
             uint32_t r32[32];
             tmem_ld32(c.tmem + lrow + TM_D3 + 32 * u2, r32);
             wait_ld();
-            if (r < L) {
-                __nv_bfloat16 *dst = c.o + (((size_t)c.bb * c.T + t0 + r) * c.H + c.h) * VD + 32 * u2;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    uint4 pk;
-                    pk.x = pack_bf16(__uint_as_float(r32[8 * u]), __uint_as_float(r32[8 * u + 1]));
-                    pk.y = pack_bf16(__uint_as_float(r32[8 * u + 2]), __uint_as_float(r32[8 * u + 3]));
-                    pk.z = pack_bf16(__uint_as_float(r32[8 * u + 4]), __uint_as_float(r32[8 * u + 5]));
-                    pk.w = pack_bf16(__uint_as_float(r32[8 * u + 6]), __uint_as_float(r32[8 * u + 7]));
-                    *reinterpret_cast<uint4 *>(dst + 8 * u) = pk;
-                }
+            for (int u = 0; u < 4; ++u) {
+                uint4 pk;
+                pk.x = pack_bf16(__uint_as_float(r32[8 * u]), __uint_as_float(r32[8 * u + 1]));
+                pk.y = pack_bf16(__uint_as_float(r32[8 * u + 2]), __uint_as_float(r32[8 * u + 3]));
+                pk.z = pack_bf16(__uint_as_float(r32[8 * u + 4]), __uint_as_float(r32[8 * u + 5]));
+                pk.w = pack_bf16(__uint_as_float(r32[8 * u + 6]), __uint_as_float(r32[8 * u + 7]));
+                *reinterpret_cast<uint4 *>(stg + lane * 80 + 16 * u) = pk;
             }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {   // 8 rows x 64 B per store instruction
+                const int rr = 8 * i + (lane >> 2), pc = lane & 3, orow = ow * 32 + rr;
+                const uint4 val = *reinterpret_cast<const uint4 *>(stg + rr * 80 + 16 * pc);
+                if (orow < L)
+                    *reinterpret_cast<uint4 *>(c.o + (((size_t)c.bb * c.T + t0 + orow) * c.H + c.h) * VD + 32 * u2 + 8 * pc) = val;
+            }
+            __syncwarp();
         }
         fence_before();
         mbar_arrive(mbar(c, MB_D3FREE));
