@@ -457,9 +457,9 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
             float sS[4], sZ[4], sP[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                sS[j] = slow ? 1.f : exp2f(m2[j]);
-                sZ[j] = slow ? exp2f(gC[j]) : sS[j];
-                sP[j] = slow ? 1.f : exp2f(gC[j] - m2[j]);
+                sS[j] = slow ? 1.f : fast_exp2(m2[j]);
+                sZ[j] = slow ? fast_exp2(gC[j]) : sS[j];
+                sP[j] = slow ? 1.f : fast_exp2(gC[j] - m2[j]);
             }
             *reinterpret_cast<float4 *>(vs + c4) = make_float4(sS[0], sS[1], sS[2], sS[3]);
             *reinterpret_cast<float4 *>(vs + 128 + c4) = make_float4(sZ[0], sZ[1], sZ[2], sZ[3]);
