@@ -255,6 +255,18 @@ def oracle_sample_time(prefill_wl, decode_wl, budget_s=12.0, max_chains=None):
     return full_pre + full_dec, desc, cores
 
 
+def bench_config(world):
+    """The workload description both arms print (per GPU sizes are fixed: weak scaling)."""
+    import synth
+    pw, dw = synth.WORKLOADS[PREFILL], synth.WORKLOADS[DECODE]
+    return {"workload": f"{PREFILL} (B8 H16 T4096 d_k=d_v=128, C=64, bf16 tokens, fp32 alpha/state) + "
+                        f"{DECODE} (B256 H16 d128 decode step, 256 MiB fp32 state in place)",
+            "per_gpu": {"prefill": [pw.B, pw.T, pw.H, pw.K, pw.V], "decode": [dw.B, dw.H, dw.K, dw.V]},
+            "global_batch": {"prefill": pw.B * world, "decode": dw.B * world},
+            "l2": "inputs larger than L2 (1.09 GB prefill inputs, 256 MiB decode state); no flush",
+            "parallelism": f"replicas x{world} (independent chains, no collective)"}
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -276,7 +288,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{PREFILL} (B8 H16 T4096 d128) + {DECODE} (B256 H16 d128)"},
+        "config": bench_config(args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": desc + " (each step)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -431,16 +443,10 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{PREFILL} (B8 H16 T4096 d_k=d_v=128, C=64, bf16 tokens, fp32 alpha/state) + "
-                               f"{DECODE} (B256 H16 d128 decode step, 256 MiB fp32 state in place)",
-                   "per_gpu": {"prefill": [B, T, H, K, V], "decode": [dw.B, dw.H, dw.K, dw.V]},
-                   "global_batch": {"prefill": B * world, "decode": dw.B * world},
-                   "l2": "inputs larger than L2 (1.09 GB prefill inputs, 256 MiB decode state); no flush",
-                   "prefill_path": "tcgen05" if path == 1 else "simt",
-                   "parallelism": f"replicas x{world} (independent chains, no collective)"},
+        "config": bench_config(world),
         "roofline": roof_pre,
         "parts": {"prefill": {"ms": pre_ms_max, "tokens_per_s": B * T * world / (pre_ms_max * 1e-3),
-                              "roofline": roof_pre},
+                              "path": "tcgen05" if path == 1 else "simt", "roofline": roof_pre},
                   "decode": {"ms": dec_ms_max, "tokens_per_s": dw.B * world / (dec_ms_max * 1e-3),
                              "roofline": roof_dec}},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
