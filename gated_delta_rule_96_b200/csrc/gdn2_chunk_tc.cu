@@ -713,14 +713,21 @@ __device__ __forceinline__ void state_group(const Ctx &c, int tid, float *ST, si
         if (!group_wait(c, mbar_slot(c, MB_VEC, n), slot_par(n), BAR_STATE, GROUP)) return;
         if (n > 0 && !group_wait(c, mbar_slot(c, MB_G45, n - 1), slot_par(n - 1), BAR_STATE, GROUP)) return;
         const float *vs = vec + (n & 1) * 384;
-        const float ssc = vs[crow] * egm_prev;         // scale of the bf16 operand
-        const float zsc = vs[128 + crow] * egm_prev;   // scale of the TMEM state
+        // The factors are applied one after the other: first sPost of chunk n-1, which turns Z into the
+        // true state S_n, then this chunk's sS / sZ.  Their product alone can lie far below fp32's
+        // range (both are about 2^(-span/2) for a chunk of log-decay span 'span') even though every
+        // scaled value is representable.
+        const float post = egm_prev;             // sPost of chunk n-1
+        const float ssc = vs[crow];              // scale of the bf16 operand
+        const float zsc = vs[128 + crow];        // scale of the TMEM state
         egm_prev = vs[256 + crow];
 #pragma unroll
         for (int u2 = 0; u2 < 4; ++u2) {
             uint32_t r32[32];
             tmem_ld32(c.tmem + lrow + TM_Z + 32 * u2, r32);
             wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(post * __uint_as_float(r32[i]));   // S_n
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int vv = 32 * u2 + 8 * u;

@@ -137,7 +137,8 @@ def _sampled_check(name, chains, threads=None):
 
 
 def test_prefill_1p3b_full_size_sampled():
-    _sampled_check("prefill_1p3b", [(0, 0), (3, 7), (7, 15), (5, 2)])
+    # two heads of every batch element: 16 of the 128 chains
+    _sampled_check("prefill_1p3b", [(b, h) for b in range(8) for h in ((5 * b) % 16, (5 * b + 9) % 16)])
 
 
 def test_prefill_kda_full_size_sampled():
@@ -148,8 +149,9 @@ def test_prefill_gdn_full_size_sampled():
     _sampled_check("prefill_gdn", [(1, 0), (7, 14)])
 
 
-def test_prefill_long_full_size_sampled():
-    _sampled_check("prefill_long", [(0, 0), (0, 11)])
+def test_prefill_long_all_chains():
+    # every head: 1,024 chunks each, typical per-chunk log-decay spans of 100-170 (log2)
+    _sampled_check("prefill_long", [(0, h) for h in range(16)])
 
 
 def test_prefill_slow_decay_full_size_sampled():
