@@ -70,6 +70,28 @@ def test_extreme_decay_and_unit_decay():
     assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
 
 
+@pytest.mark.parametrize("span", [120.0, 165.0, 172.0, 176.0])
+def test_chunk_spans_near_the_tensor_core_limit(span):
+    """Every chunk decays by about `span` (log2) in half of the key channels, so the kernel's
+    decay factors around the chunk midpoint reach 2^(span/2) and the frame factors of two
+    consecutive chunks multiply to about 2^-span (below fp32's range for span > 149); 176 lies
+    past the tensor-core limit (173) and takes the wide-span path.  The other channels decay
+    slowly, so the carried state stays visible in o."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("x", 1, 2, 320, 128, 128, "bf16", 1.0, seed=81, s0_std=0.05)
+    x = synth.make_inputs(wl)
+    a = x["alpha"].copy()
+    a[..., ::2] = np.float32(2.0 ** (-span / 64.0))    # per-token decay of the fast channels
+    a[..., 1::2] = np.maximum(a[..., 1::2], np.float32(0.9))
+    x["alpha"] = a
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    o, ST = prefill(torch, g, xd, torch.from_numpy(S0).cuda())
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
+    assert_close("o", f64(o), ref_o, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
 def test_T0_copies_state_and_empty_batch():
     torch, g = cuda_or_skip()
     B, H, K, V = 2, 3, 64, 128
