@@ -164,11 +164,11 @@ def test_prefill_1p3b_full_size_sampled():
 
 
 def test_prefill_kda_full_size_sampled():
-    _sampled_check("prefill_kda", [(0, 1), (6, 9)])
+    _sampled_check("prefill_kda", [(0, 1), (2, 14), (5, 6), (7, 9)])
 
 
 def test_prefill_gdn_full_size_sampled():
-    _sampled_check("prefill_gdn", [(1, 0), (7, 14)])
+    _sampled_check("prefill_gdn", [(1, 0), (3, 11), (4, 5), (7, 14)])
 
 
 def test_prefill_long_all_chains():
@@ -177,4 +177,4 @@ def test_prefill_long_all_chains():
 
 
 def test_prefill_slow_decay_full_size_sampled():
-    _sampled_check("prefill_slow_decay", [(2, 3)])
+    _sampled_check("prefill_slow_decay", [(0, 12), (2, 3), (6, 8)])
