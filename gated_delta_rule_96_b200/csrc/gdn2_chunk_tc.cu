@@ -44,6 +44,8 @@
 // chunk's loads in flight).
 // Every event that a waiter may see two chunks late has one mbarrier per buffer slot.
 // Every wait is bounded; on expiry the block sets the workspace status word and exits.
+#include <algorithm>
+
 #include "gdn2_common.cuh"
 #include "gdn2_internal.h"
 #include "tc_ptx.cuh"
@@ -93,6 +95,15 @@ enum : uint32_t {
     MB_G1 = 80, MB_READOUT = 88, MB_S1DONE = 96, MB_D3FREE = 104, MB_END = 112
 };
 constexpr uint32_t MISC_TSLOT = 160, MISC_ABORT = 164;
+
+// Launch flags of the segmented (parallel-in-time) prefill.  A block owns segment
+// blockIdx.x % nseg of chain blockIdx.x / nseg; S0 and S_T are indexed by block.
+enum : uint32_t {
+    SEG_ZERO_WRITES = 1,   // U = 0: the run propagates the state only (the homogeneous part)
+    SEG_SKIP_O = 2,        // o is not stored
+    SEG_IDENTITY_S0 = 4,   // the segment starts from S = I (d_k = d_v)
+    SEG_ST_LAST = 8,       // only the chain's last segment stores S_T, at S_T[chain]
+};
 
 constexpr uint32_t ID_G1 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t ID_G2 = idesc_bf16(128, 128, 0, 1);
@@ -214,6 +225,8 @@ struct Ctx {
     const float *alpha;
     __nv_bfloat16 *o;
     int T, H, bb, h, NC;
+    int tb, te;        // token range of this block's segment: [tb, te)
+    uint32_t flags;    // SEG_* below
 };
 
 __device__ __forceinline__ uint32_t mbar(const Ctx &c, uint32_t off) { return c.misc + off; }
@@ -365,7 +378,7 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
     const int T = c.T, H = c.H, bb = c.bb, h = c.h;
 
     for (int n = 0; n < c.NC; ++n) {
-        const int t0 = n * C, L = min(C, T - t0);
+        const int t0 = c.tb + n * C, L = min(C, c.te - t0);
         unsigned char *EQ = sm + SM_EQ + (n & 1) * EQ_BYTES;
         unsigned char *KT = sm + SM_KT + (n & 1) * KT_BYTES;
         // ---------------------------------------------------------------- loads and log-decay prefix
@@ -383,7 +396,7 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
         }
         if (n + 1 < c.NC) {   // next chunk's rows of q, k, b, alpha into L2 (one 128-B line per request)
             const int r = tid1 & 63, half = tid1 >> 6;
-            const int t = min(r, T - t0 - C - 1);
+            const int t = min(r, c.te - t0 - C - 1);
             const size_t row = ((size_t)bb * T + t0 + C + t) * H + h;
             const char *base[3] = {(const char *)(c.q + row * KD), (const char *)(c.k + row * KD), (const char *)(c.b + row * KD)};
 #pragma unroll
@@ -700,7 +713,7 @@ __device__ __forceinline__ void solve_group(const Ctx &c, int tid2) {
 }
 
 // ============================================================================ state group
-__device__ __forceinline__ void state_group(const Ctx &c, int tid, float *ST, size_t chain) {
+__device__ __forceinline__ void state_group(const Ctx &c, int tid, float *ST) {
     unsigned char *sm = c.sm;
     const float *vec = reinterpret_cast<const float *>(sm + SM_VEC);
     const int warp = tid >> 5;
@@ -777,7 +790,8 @@ __device__ __forceinline__ void state_group(const Ctx &c, int tid, float *ST, si
     // the last chunk's G4/G5 must be complete before Z is read
     if (!group_wait(c, mbar_slot(c, MB_G45, c.NC - 1), slot_par(c.NC - 1), BAR_STATE, GROUP)) return;
     // S_T = Diag(sPost) Z of the last chunk
-    float *dst = ST + (chain * KD + crow) * VD;
+    if (!ST) return;
+    float *dst = ST + crow * VD;
 #pragma unroll
     for (int u2 = 0; u2 < 4; ++u2) {
         uint32_t r32[32];
@@ -812,10 +826,10 @@ __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
     const int vw = tid2 >> 5, lane = tid2 & 31, c4 = lane * 4;
     const int T = c.T, H = c.H, bb = c.bb, h = c.h;
     for (int n = 0; n < c.NC; ++n) {
-        const int t0 = n * C, L = min(C, T - t0);
+        const int t0 = c.tb + n * C, L = min(C, c.te - t0);
         unsigned char *U = c.sm + SM_U + (n & 1) * U_BYTES;
         if (n + 1 < c.NC) {   // next chunk's rows of v and w into L2
-            const int t = min(tid2, T - t0 - C - 1);
+            const int t = min(tid2, c.te - t0 - C - 1);
             const size_t row = ((size_t)bb * T + t0 + C + t) * H + h;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
@@ -827,9 +841,10 @@ __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
 #pragma unroll 1
         for (int p0 = 32 * vw; p0 < 32 * vw + 32; p0 += 8) {
             uint2 rv[8], rw[8];
+            const int Lw = (c.flags & SEG_ZERO_WRITES) ? 0 : L;   // no writes: U = 0
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const int t = min(p0 + p, L - 1);
+                const int t = min(p0 + p, max(Lw, 1) - 1);
                 const size_t row = ((size_t)bb * T + t0 + t) * H + h;
                 rv[p] = __ldg(reinterpret_cast<const uint2 *>(c.v + row * VD + c4));
                 rw[p] = __ldg(reinterpret_cast<const uint2 *>(c.w + row * VD + c4));
@@ -837,7 +852,7 @@ __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
 #pragma unroll
             for (int p = 0; p < 8; ++p)
                 *reinterpret_cast<uint2 *>(U + sw_off(p0 + p, c4, 64)) =
-                    p0 + p < L ? make_uint2(bmul2(rw[p].x, rv[p].x), bmul2(rw[p].y, rv[p].y)) : make_uint2(0u, 0u);
+                    p0 + p < Lw ? make_uint2(bmul2(rw[p].x, rv[p].x), bmul2(rw[p].y, rv[p].y)) : make_uint2(0u, 0u);
         }
         fence_async_smem();
         mbar_arrive(mbar_slot(c, MB_U, n));
@@ -848,8 +863,9 @@ __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
     const int ow = tid2 >> 5, lane = tid2 & 31;   // this thread's row of O: TMEM lane 64 + tid2
     const uint32_t lrow = (uint32_t)(64 + ow * 32) << 16;
     unsigned char *stg = c.sm + SM_OST + ow * 2560;   // 32 rows x 80 B (64 B of data + 16 B pad)
+    const bool store = !(c.flags & SEG_SKIP_O);
     for (int n = 0; n < c.NC; ++n) {
-        const int t0 = n * C, L = min(C, c.T - t0);
+        const int t0 = c.tb + n * C, L = store ? min(C, c.te - t0) : 0;
         if (!warp_wait(c, mbar_slot(c, MB_G45, n), slot_par(n))) return;
 #pragma unroll
         for (int u2 = 0; u2 < 4; ++u2) {
@@ -885,16 +901,20 @@ __global__ void __launch_bounds__(NT, 1)
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ alpha,
                     const __nv_bfloat16 *__restrict__ b, const __nv_bfloat16 *__restrict__ w,
                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST, int H,
-                    int T, unsigned int *__restrict__ status) {
+                    int T, int seg_len, int nseg, uint32_t flags, unsigned int *__restrict__ status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int chain = blockIdx.x;
+    const int chain = blockIdx.x / nseg, seg = blockIdx.x % nseg;
     Ctx c;
     c.sm = sm;
     c.misc = smem_u32(sm + SM_MISC);
     c.q = q; c.k = k; c.v = v; c.b = b; c.w = w; c.alpha = alpha; c.o = o;
-    c.T = T; c.H = H; c.bb = chain / H; c.h = chain % H; c.NC = (T + C - 1) / C;
+    c.T = T; c.H = H; c.bb = chain / H; c.h = chain % H;
+    c.tb = seg * seg_len; c.te = min(T, c.tb + seg_len); c.NC = (c.te - c.tb + C - 1) / C;
+    c.flags = flags;
+    float *st_dst = (flags & SEG_ST_LAST) ? (seg == nseg - 1 ? ST + (size_t)chain * KD * VD : nullptr)
+                                          : ST + (size_t)blockIdx.x * KD * VD;
 
     if (warp == 12) tmem_alloc(c.misc + MISC_TSLOT, TM_COLS);
     if (tid == 0) {
@@ -913,7 +933,8 @@ __global__ void __launch_bounds__(NT, 1)
         regs_dec<104>();
         const int crow = tid;
         const uint32_t lrow = (uint32_t)(warp * 32) << 16;
-        const float *src = S0 ? S0 + ((size_t)chain * KD + crow) * VD : nullptr;
+        const float *src = S0 ? S0 + ((size_t)blockIdx.x * KD + crow) * VD : nullptr;
+        const bool ident = (flags & SEG_IDENTITY_S0) != 0;
 #pragma unroll
         for (int u2 = 0; u2 < 4; ++u2) {
             uint32_t r32[32];
@@ -923,13 +944,16 @@ __global__ void __launch_bounds__(NT, 1)
                 r32[i] = __float_as_uint(x.x); r32[i + 1] = __float_as_uint(x.y);
                 r32[i + 2] = __float_as_uint(x.z); r32[i + 3] = __float_as_uint(x.w);
             }
+            if (ident)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(32 * u2 + i == crow ? 1.f : 0.f);
             tmem_st32(c.tmem + lrow + TM_Z + 32 * u2, r32);
         }
         wait_st();
         fence_before();
         group_sync(BAR_STATE, GROUP);
         fence_after();
-        state_group(c, tid, ST, (size_t)chain);
+        state_group(c, tid, st_dst);
         regs_inc<128>();   // every warpgroup leaves its role with the launch budget
     } else if (warp < 8) {
         regs_inc<208>();
@@ -955,6 +979,43 @@ __global__ void __launch_bounds__(NT, 1)
     if (warp == 12) tmem_dealloc(c.tmem, TM_COLS);
 }
 
+
+// ============================================================================ segment scan
+// S_g = M_(g-1) S_(g-1) + N_(g-1) along the segments of each chain (g = 1 .. nseg-1), S_0 = S0.
+// One block per (chain, 16-column slice of S); fp32.
+__global__ void __launch_bounds__(256) segment_scan_kernel(const float *__restrict__ M, const float *__restrict__ N,
+                                                           const float *__restrict__ S0, float *__restrict__ Sg,
+                                                           int nseg) {
+    __shared__ float sprev[KD][16];
+    const int chain = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
+    const size_t KV = (size_t)KD * VD;
+    const int col = tid & 15, r0 = tid >> 4;   // rows r0, r0 + 16, ..., r0 + 112
+    for (int r = r0; r < KD; r += 16) {
+        const float v = S0 ? S0[chain * KV + (size_t)r * VD + c0 + col] : 0.f;
+        sprev[r][col] = v;
+        Sg[((size_t)chain * nseg) * KV + (size_t)r * VD + c0 + col] = v;
+    }
+    __syncthreads();
+    for (int g = 1; g < nseg; ++g) {
+        const float *Mg = M + ((size_t)chain * nseg + g - 1) * KV, *Ng = N + ((size_t)chain * nseg + g - 1) * KV;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = Ng[(size_t)(r0 + 16 * i) * VD + c0 + col];
+        for (int kk = 0; kk < KD; ++kk) {
+            const float sv = sprev[kk][col];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(Mg[(size_t)(r0 + 16 * i) * VD + kk], sv, acc[i]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            sprev[r0 + 16 * i][col] = acc[i];
+            Sg[((size_t)chain * nseg + g) * KV + (size_t)(r0 + 16 * i) * VD + c0 + col] = acc[i];
+        }
+        __syncthreads();
+    }
+}
+
 }  // namespace tcfwd
 
 bool tc_supported(int B, int H, int T, int K, int V, int C, int bf16) {
@@ -962,7 +1023,32 @@ bool tc_supported(int B, int H, int T, int K, int V, int C, int bf16) {
     return bf16 && K == 128 && V == 128 && C == 64;
 }
 
-size_t tc_workspace_bytes(int, int, int, int, int, int) { return kStatusBytes; }
+namespace {
+
+// Parallel-in-time plan for few, long chains: the sequence of each chain is cut into nseg
+// segments of whole chunks so that about 128 blocks run at once.  Every segment's state map
+// S_out = M S_in + N is found in parallel (N from S_in = 0, M from S_in = I with the writes
+// switched off), the maps are composed along the chain, and the segments run again from their
+// true start states.  Three passes over 1/nseg of the sequence instead of one over all of it.
+struct SegPlan {
+    int nseg, seg_len;
+};
+SegPlan seg_plan(int B, int H, int T) {
+    const int chains = B * H, NC = (T + tcfwd::C - 1) / tcfwd::C;
+    int nseg = 1;
+    if (chains > 0 && chains <= 64 && NC >= 32) nseg = std::min(128 / chains, NC / 8);
+    if (nseg < 2) return {1, NC * tcfwd::C};
+    const int per = (NC + nseg - 1) / nseg;   // chunks per segment
+    return {(NC + per - 1) / per, per * tcfwd::C};
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(int B, int H, int T, int, int, int) {
+    const SegPlan sp = seg_plan(B, H, T);
+    if (sp.nseg == 1) return kStatusBytes;
+    return kStatusBytes + 3 * sizeof(float) * (size_t)B * H * sp.nseg * tcfwd::KD * tcfwd::VD;
+}
 
 int launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
                     const float *S0, void *o, float *ST, int B, int H, int T, int K, int V, int C, void *ws,
@@ -972,10 +1058,24 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
     if (cudaFuncSetAttribute(tcfwd::chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return -6;
-    tcfwd::chunk_tc_kernel<<<B * H, tcfwd::NT, smem, st>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, alpha,
-        (const __nv_bfloat16 *)b, (const __nv_bfloat16 *)w, S0, (__nv_bfloat16 *)o, ST, H, T,
-        reinterpret_cast<unsigned int *>(ws));
+    auto run = [&](int nseg, int seg_len, uint32_t flags, const float *s0, float *st_out) {
+        tcfwd::chunk_tc_kernel<<<B * H * nseg, tcfwd::NT, smem, st>>>(
+            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, alpha,
+            (const __nv_bfloat16 *)b, (const __nv_bfloat16 *)w, s0, (__nv_bfloat16 *)o, st_out, H, T, seg_len, nseg,
+            flags, reinterpret_cast<unsigned int *>(ws));
+    };
+    const SegPlan sp = seg_plan(B, H, T);
+    if (sp.nseg == 1) {
+        run(1, sp.seg_len, 0u, S0, ST);
+        return launch_status();
+    }
+    const size_t KV = (size_t)tcfwd::KD * tcfwd::VD, per_pass = (size_t)B * H * sp.nseg * KV;
+    float *Nm = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + kStatusBytes);
+    float *Mm = Nm + per_pass, *Sg = Mm + per_pass;
+    run(sp.nseg, sp.seg_len, tcfwd::SEG_SKIP_O, nullptr, Nm);
+    run(sp.nseg, sp.seg_len, tcfwd::SEG_SKIP_O | tcfwd::SEG_ZERO_WRITES | tcfwd::SEG_IDENTITY_S0, nullptr, Mm);
+    tcfwd::segment_scan_kernel<<<dim3(B * H, tcfwd::VD / 16), 256, 0, st>>>(Mm, Nm, S0, Sg, sp.nseg);
+    run(sp.nseg, sp.seg_len, tcfwd::SEG_ST_LAST, Sg, ST);
     return launch_status();
 }
 

@@ -52,6 +52,19 @@ def test_workspace_bytes():
     assert g.gdn2_chunk_fwd_workspace_bytes(1, 1, 65, 128, 128, 64, g.GDN2_F32) == n2
 
 
+def test_workspace_bytes_tensor_core_path():
+    # many chains: the fused kernel needs only the status header
+    assert g.gdn2_chunk_fwd_workspace_bytes(8, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 256
+    # few long chains run in parallel over segments: three fp32 states per (chain, segment)
+    state = 4 * 128 * 128
+    # B1 H16 T65536: 1,024 chunks, 8 segments of 128 chunks
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 16, 65536, 128, 128, 64, g.GDN2_BF16) == 256 + 3 * 16 * 8 * state
+    # B1 H2, 41 chunks: at most 64 segments by chains, at least 8 chunks each -> 5 segments of 9 chunks
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 2, 64 * 40 + 37, 128, 128, 64, g.GDN2_BF16) == 256 + 3 * 2 * 5 * state
+    # short sequences are not split
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 2, 64 * 31, 128, 128, 64, g.GDN2_BF16) == 256
+
+
 P = ctypes.c_void_p
 FAKE = P(0x10000)       # never dereferenced: every case below fails validation first
 

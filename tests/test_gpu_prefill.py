@@ -92,6 +92,23 @@ def test_chunk_spans_near_the_tensor_core_limit(span):
     assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
 
 
+@pytest.mark.parametrize("alpha_scale", [1.0, 0.02])
+def test_segmented_prefill_few_long_chains(alpha_scale):
+    """Few chains and a long, ragged sequence (B1 H2, 41 chunks): the prefill runs in parallel
+    over five segments of each chain (state maps of every segment, composed along the chain,
+    then a rerun from the true start states); with alpha near 1 the carried state dominates."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("seg", 1, 2, 64 * 40 + 37, 128, 128, "bf16", 1.0, seed=83, s0_std=0.05,
+                        alpha_scale=alpha_scale)
+    x = synth.make_inputs(wl)
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    o, ST = prefill(torch, g, xd, torch.from_numpy(S0).cuda())
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
+    assert_close("o", f64(o), ref_o, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
 def test_T0_copies_state_and_empty_batch():
     torch, g = cuda_or_skip()
     B, H, K, V = 2, 3, 64, 128
