@@ -15,7 +15,7 @@ import ctypes
 import os
 
 __all__ = [
-    "GDN2Error", "load_library", "library_path", "gdn2_chunk_fwd", "gdn2_decode_step",
+    "GDN2Error", "load_library", "library_path", "gdn2_chunk_fwd", "gdn2_chunk_fwd_edges", "gdn2_decode_step",
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace",
@@ -63,6 +63,8 @@ def load_library():
     lib.gdn2_workspace_status.restype = i
     lib.gdn2_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i] * 7 + [vp]
     lib.gdn2_chunk_fwd_noalloc.restype = i
+    lib.gdn2_chunk_fwd_edges.argtypes = [vp] * 10 + [i] * 7 + [vp, sz, vp]
+    lib.gdn2_chunk_fwd_edges.restype = i
     lib.gdn2_status_str.argtypes = [i]
     lib.gdn2_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -145,6 +147,36 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, C=64, workspace=None, strea
                                        workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_fwd")
+
+
+def gdn2_chunk_fwd_edges(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o_weight, o, S_T, C=64, workspace=None,
+                         stream=None) -> None:
+    """Prefill with the layer edges fused (include/gdn2.h, gdn2_chunk_fwd_edges): q, k L2-normalised,
+    b = sigmoid(b_logit), w = sigmoid(w_logit), alpha = exp(-softplus(a_logit)), optional RMSNorm of o
+    with weight o_weight [d_v] (None: no norm).  bf16 tokens, d_k = d_v = 128."""
+    import torch
+    _check_cuda(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o_weight, o, S_T, workspace)
+    B, T, H, K = q_raw.shape
+    V = v.shape[-1]
+    dt = _dtype_code(q_raw)
+    for name, t in (("a_logit", a_logit), ("S_T", S_T), ("S0", S0), ("o_weight", o_weight)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    for name, t, shp in (("k_raw", k_raw, (B, T, H, K)), ("b_logit", b_logit, (B, T, H, K)),
+                         ("a_logit", a_logit, (B, T, H, K)), ("w_logit", w_logit, (B, T, H, V)),
+                         ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)), ("S0", S0, (B, H, K, V)),
+                         ("o_weight", o_weight, (V,))):
+        if t is not None and tuple(t.shape) != shp:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    need = gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, C, dt)
+    if workspace is None:
+        workspace = new_workspace(need, q_raw.device)
+    rc = load_library().gdn2_chunk_fwd_edges(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_logit), _ptr(b_logit),
+                                             _ptr(w_logit), _ptr(S0), _ptr(o_weight), _ptr(o), _ptr(S_T), B, H, T,
+                                             K, V, C, dt, _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_chunk_fwd_edges")
 
 
 def gdn2_chunk_fwd_noalloc(q, k, v, alpha, b, w, S0, o, S_T, C=64, stream=None) -> None:

@@ -77,6 +77,26 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alp
     return rc;
 }
 
+int gdn2_chunk_fwd_edges(const void *q_raw, const void *k_raw, const void *v, const float *a_logit,
+                         const void *b_logit, const void *w_logit, const float *S0, const float *o_weight, void *o,
+                         float *S_T, int B, int H, int T, int d_k, int d_v, int C, int dtype, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    if (T < 0) return GDN2_ERR_SHAPE;
+    if (T == 0) return gdn2_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, B, H,
+                                      0, d_k, d_v, C, dtype, workspace, workspace_bytes, stream);
+    int rc = check_common(q_raw, k_raw, v, a_logit, b_logit, w_logit, o, B, H, d_k, d_v, dtype);
+    if (rc != GDN2_OK) return rc;
+    if (C != 64 || !use_tc(B, H, T, d_k, d_v, C, dtype)) return GDN2_ERR_UNSUPPORTED;
+    if (!S_T) return GDN2_ERR_NULL;
+    if (!aligned16(S_T) || (S0 && !aligned16(S0)) || (o_weight && !aligned16(o_weight))) return GDN2_ERR_ALIGN;
+    if (!workspace) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    if (workspace_bytes < gdn2_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, C, dtype)) return GDN2_ERR_WORKSPACE;
+    if (B == 0 || H == 0) return GDN2_OK;
+    return gdn2::launch_chunk_tc(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o, S_T, B, H, T, d_k, d_v, C,
+                                 workspace, reinterpret_cast<cudaStream_t>(stream), 1, o_weight);
+}
+
 int gdn2_decode_step(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
                      float *S, void *o, int B, int H, int d_k, int d_v, int dtype, void *stream) {
     int rc = check_common(q, k, v, alpha, b, w, o, B, H, d_k, d_v, dtype);

@@ -135,6 +135,27 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
 }
 // tf32 operand of mma.sync: the fp32 bit pattern (the tensor core reads the top 19 bits, i.e.
 // truncates the mantissa to 10 bits; T ends up in bf16, far coarser)
+// Layer edges fused into the prefill (the layer around the recurrence: q and k L2-normalised per
+// token and head, b and w sigmoid gates, the decay from a logit, the output through RMSNorm).
+constexpr float EDGE_NORM_EPS = 1e-6f;   // q / max(|q|, eps), likewise k
+constexpr float EDGE_RMS_EPS = 1e-6f;    // o / sqrt(mean(o^2) + eps) * weight
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// alpha = exp(-softplus(a)) = 1 / (1 + e^a) (0 past fp32's range: the caller floors it)
+__device__ __forceinline__ float alpha_of_logit(float a) { return __fdividef(1.f, 1.f + __expf(a)); }
+// log2 of alpha = exp(-softplus(a)), floored at log2 of the smallest normal float
+__device__ __forceinline__ float log2_alpha_of_logit(float a) {
+    const float sp = a > 15.f ? a : __logf(1.f + __expf(a));
+    return fmaxf(-sp * 1.4426950408889634f, -126.f);
+}
+// two bf16 values scaled by s, rounded to bf16
+__device__ __forceinline__ uint32_t bscale2(uint32_t a, float s) {
+    const float2 f = unpack2(a);
+    return pack_bf16(f.x * s, f.y * s);
+}
+__device__ __forceinline__ uint32_t bsigmoid2(uint32_t a) {
+    const float2 f = unpack2(a);
+    return pack_bf16(sigmoid_f(f.x), sigmoid_f(f.y));
+}
 __device__ __forceinline__ uint32_t tf32(float x) { return __float_as_uint(x); }
 // D(16x8) += A(16x8) B(8x8), tf32 inputs, fp32 accumulate (warp-level)
 __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -226,6 +247,7 @@ struct Ctx {
     __nv_bfloat16 *o;
     int T, H, bb, h, NC;
     int tb, te;        // token range of this block's segment: [tb, te)
+    const float *onorm;   // RMSNorm weight of o (layer-edge variant; null: none)
     uint32_t flags;    // SEG_* below
 };
 
@@ -321,34 +343,50 @@ __device__ __forceinline__ void issue_g45(const Ctx &c, int n) {
 // of D1 that G1 would have written).  For each channel the exponent g_rc - g_ic is summed from
 // log2 alpha while i walks down from r, so it never leaves [-inf, 0]; tokens are re-read from
 // global memory (resident in L2).
+template <bool EDGES>
 __device__ __forceinline__ void wide_span_ap(const Ctx &c, int tid1, int t0, int L) {
     const int r = tid1 & 63;
     const bool isP = tid1 >= 64;
     const int T = c.T, H = c.H, bb = c.bb, h = c.h;
     const uint32_t lane_base = c.tmem + ((uint32_t)((tid1 >> 5) * 32) << 16) + TM_D1;
     const size_t rowr = ((size_t)bb * T + t0 + min(r, L - 1)) * H + h;
+    auto rownorm = [&](const __nv_bfloat16 *x, size_t row) {   // 1 / max(|x_row|, eps)
+        float ss = 0.f;
+        for (int cc = 0; cc < KD; ++cc) {
+            const float v = __bfloat162float(x[row * KD + cc]);
+            ss += v * v;
+        }
+        return 1.f / fmaxf(sqrtf(ss), EDGE_NORM_EPS);
+    };
+    auto log2a = [&](size_t row, int cc) {
+        const float a = c.alpha[row * KD + cc];
+        return EDGES ? log2_alpha_of_logit(a) : fast_log2(fmaxf(a, 1.17549435e-38f));
+    };
+    const float sr = EDGES ? (isP ? rownorm(c.q, rowr) : rownorm(c.k, rowr)) : 1.f;
 #pragma unroll 1
     for (int i0 = 0; i0 < 64; i0 += 16) {
-        float acc[16];
+        float acc[16], sk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 16; ++i) {
+            acc[i] = 0.f;
+            sk[i] = EDGES ? rownorm(c.k, ((size_t)bb * T + t0 + min(i0 + i, L - 1)) * H + h) : 1.f;
+        }
         if (r < L && i0 <= r) {
 #pragma unroll 1
             for (int cc = 0; cc < KD; ++cc) {
-                const float x = isP ? __bfloat162float(c.q[rowr * KD + cc])
-                                    : __bfloat162float(c.b[rowr * KD + cc]) * __bfloat162float(c.k[rowr * KD + cc]);
+                const float bg = EDGES ? sigmoid_f(__bfloat162float(c.b[rowr * KD + cc])) : __bfloat162float(c.b[rowr * KD + cc]);
+                const float x = sr * (isP ? __bfloat162float(c.q[rowr * KD + cc]) : bg * __bfloat162float(c.k[rowr * KD + cc]));
                 // exponent at i = i0 + 15 (or r): log2 of alpha over positions i+1 .. r
                 const int itop = min(i0 + 15, r);
                 float d = 0.f;
 #pragma unroll 1
-                for (int j = r; j > itop; --j)
-                    d += fast_log2(fmaxf(c.alpha[(((size_t)bb * T + t0 + j) * H + h) * KD + cc], 1.17549435e-38f));
+                for (int j = r; j > itop; --j) d += log2a(((size_t)bb * T + t0 + j) * H + h, cc);
 #pragma unroll
                 for (int i = 15; i >= 0; --i) {
                     if (i0 + i <= itop) {
                         const size_t rowi = ((size_t)bb * T + t0 + i0 + i) * H + h;
-                        acc[i] += x * __bfloat162float(c.k[rowi * KD + cc]) * exp2f(d);
-                        d += fast_log2(fmaxf(c.alpha[rowi * KD + cc], 1.17549435e-38f));
+                        acc[i] += x * sk[i] * __bfloat162float(c.k[rowi * KD + cc]) * exp2f(d);
+                        d += log2a(rowi, cc);
                     }
                 }
             }
@@ -368,6 +406,7 @@ __device__ __forceinline__ void wide_span_ap(const Ctx &c, int tid1, int t0, int
 // Builds the bf16 operands of every chunk into slot n & 1 as soon as the slot is free
 // (G3 and G4/G5 of chunk n-2 complete).  Warp w1 owns positions 16 w1 .. 16 w1 + 15, lane l
 // the channels 4l .. 4l+3; the positions are processed as two halves of 8.
+template <bool EDGES>
 __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
     unsigned char *sm = c.sm;
     float *vec = reinterpret_cast<float *>(sm + SM_VEC);
@@ -393,6 +432,28 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
             rq[p] = __ldg(reinterpret_cast<const uint2 *>(c.q + row * KD + c4));
             rk[p] = __ldg(reinterpret_cast<const uint2 *>(c.k + row * KD + c4));
             rb[p] = __ldg(reinterpret_cast<const uint2 *>(c.b + row * KD + c4));
+        }
+        if (EDGES) {
+            // q, k divided by their norms over the 128 channels (4 per lane: a warp holds a row),
+            // b = sigmoid(b logit), alpha = exp(-softplus(alpha logit))
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                const float2 qa = unpack2(rq[p].x), qb = unpack2(rq[p].y), ka = unpack2(rk[p].x), kb = unpack2(rk[p].y);
+                float sq = qa.x * qa.x + qa.y * qa.y + qb.x * qb.x + qb.y * qb.y;
+                float sk = ka.x * ka.x + ka.y * ka.y + kb.x * kb.x + kb.y * kb.y;
+#pragma unroll
+                for (int msk = 16; msk > 0; msk >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, msk);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, msk);
+                }
+                const float iq = rsqrtf(fmaxf(sq, EDGE_NORM_EPS * EDGE_NORM_EPS));
+                const float ik = rsqrtf(fmaxf(sk, EDGE_NORM_EPS * EDGE_NORM_EPS));
+                rq[p] = make_uint2(bscale2(rq[p].x, iq), bscale2(rq[p].y, iq));
+                rk[p] = make_uint2(bscale2(rk[p].x, ik), bscale2(rk[p].y, ik));
+                rb[p] = make_uint2(bsigmoid2(rb[p].x), bsigmoid2(rb[p].y));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) al[p][j] = alpha_of_logit(al[p][j]);
+            }
         }
         if (n + 1 < c.NC) {   // next chunk's rows of q, k, b, alpha into L2 (one 128-B line per request)
             const int r = tid1 & 63, half = tid1 >> 6;
@@ -545,7 +606,7 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                         make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
                 }
             }
-            wide_span_ap(c, tid1, t0, L);
+            wide_span_ap<EDGES>(c, tid1, t0, L);
         }
         fence_async_smem();
         fence_before();
@@ -822,6 +883,7 @@ __device__ __forceinline__ bool warp_wait(const Ctx &c, uint32_t mb, uint32_t pa
     return true;
 }
 
+template <bool EDGES>
 __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
     const int vw = tid2 >> 5, lane = tid2 & 31, c4 = lane * 4;
     const int T = c.T, H = c.H, bb = c.bb, h = c.h;
@@ -852,13 +914,16 @@ __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
 #pragma unroll
             for (int p = 0; p < 8; ++p)
                 *reinterpret_cast<uint2 *>(U + sw_off(p0 + p, c4, 64)) =
-                    p0 + p < Lw ? make_uint2(bmul2(rw[p].x, rv[p].x), bmul2(rw[p].y, rv[p].y)) : make_uint2(0u, 0u);
+                    p0 + p < Lw ? (EDGES ? make_uint2(bmul2(bsigmoid2(rw[p].x), rv[p].x), bmul2(bsigmoid2(rw[p].y), rv[p].y))
+                                         : make_uint2(bmul2(rw[p].x, rv[p].x), bmul2(rw[p].y, rv[p].y)))
+                                : make_uint2(0u, 0u);
         }
         fence_async_smem();
         mbar_arrive(mbar_slot(c, MB_U, n));
     }
 }
 
+template <bool EDGES>
 __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
     const int ow = tid2 >> 5, lane = tid2 & 31;   // this thread's row of O: TMEM lane 64 + tid2
     const uint32_t lrow = (uint32_t)(64 + ow * 32) << 16;
@@ -867,11 +932,28 @@ __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
     for (int n = 0; n < c.NC; ++n) {
         const int t0 = c.tb + n * C, L = store ? min(C, c.te - t0) : 0;
         if (!warp_wait(c, mbar_slot(c, MB_G45, n), slot_par(n))) return;
+        float rms_scale = 1.f;   // RMSNorm of the row (layer-edge variant): a first pass for mean(o^2)
+        if (EDGES && c.onorm) {
+            float ss = 0.f;
+#pragma unroll
+            for (int u2 = 0; u2 < 4; ++u2) {
+                uint32_t r32[32];
+                tmem_ld32(c.tmem + lrow + TM_D3 + 32 * u2, r32);
+                wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ss += __uint_as_float(r32[i]) * __uint_as_float(r32[i]);
+            }
+            rms_scale = rsqrtf(ss * (1.f / VD) + EDGE_RMS_EPS);
+        }
 #pragma unroll
         for (int u2 = 0; u2 < 4; ++u2) {
             uint32_t r32[32];
             tmem_ld32(c.tmem + lrow + TM_D3 + 32 * u2, r32);
             wait_ld();
+            if (EDGES && c.onorm)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    r32[i] = __float_as_uint(__uint_as_float(r32[i]) * rms_scale * __ldg(c.onorm + 32 * u2 + i));
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 uint4 pk;
@@ -896,12 +978,14 @@ __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
     }
 }
 
+template <bool EDGES>
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ alpha,
                     const __nv_bfloat16 *__restrict__ b, const __nv_bfloat16 *__restrict__ w,
                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST, int H,
-                    int T, int seg_len, int nseg, uint32_t flags, unsigned int *__restrict__ status) {
+                    int T, int seg_len, int nseg, uint32_t flags, const float *__restrict__ onorm,
+                    unsigned int *__restrict__ status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -913,6 +997,7 @@ __global__ void __launch_bounds__(NT, 1)
     c.T = T; c.H = H; c.bb = chain / H; c.h = chain % H;
     c.tb = seg * seg_len; c.te = min(T, c.tb + seg_len); c.NC = (c.te - c.tb + C - 1) / C;
     c.flags = flags;
+    c.onorm = onorm;
     float *st_dst = (flags & SEG_ST_LAST) ? (seg == nseg - 1 ? ST + (size_t)chain * KD * VD : nullptr)
                                           : ST + (size_t)blockIdx.x * KD * VD;
 
@@ -957,7 +1042,7 @@ __global__ void __launch_bounds__(NT, 1)
         regs_inc<128>();   // every warpgroup leaves its role with the launch budget
     } else if (warp < 8) {
         regs_inc<208>();
-        build_group(c, tid - 128);
+        build_group<EDGES>(c, tid - 128);
         regs_dec<128>();
     } else if (warp < 12) {
         regs_inc<128>();
@@ -966,9 +1051,9 @@ __global__ void __launch_bounds__(NT, 1)
     } else {
         regs_dec<72>();
         if (warp < 14)
-            u_group(c, tid - 384);
+            u_group<EDGES>(c, tid - 384);
         else
-            o_group(c, tid - 448);
+            o_group<EDGES>(c, tid - 448);
         regs_inc<128>();
     }
 
@@ -1052,17 +1137,16 @@ size_t tc_workspace_bytes(int B, int H, int T, int, int, int) {
 
 int launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
                     const float *S0, void *o, float *ST, int B, int H, int T, int K, int V, int C, void *ws,
-                    cudaStream_t st) {
+                    cudaStream_t st, int edges, const float *onorm) {
     if (!tc_supported(B, H, T, K, V, C, 1)) return -4;
     const int smem = (int)tcfwd::SM_BYTES;
-    if (cudaFuncSetAttribute(tcfwd::chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-        return -6;
+    auto kern = edges ? tcfwd::chunk_tc_kernel<true> : tcfwd::chunk_tc_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -6;
     auto run = [&](int nseg, int seg_len, uint32_t flags, const float *s0, float *st_out) {
-        tcfwd::chunk_tc_kernel<<<B * H * nseg, tcfwd::NT, smem, st>>>(
+        kern<<<B * H * nseg, tcfwd::NT, smem, st>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, alpha,
             (const __nv_bfloat16 *)b, (const __nv_bfloat16 *)w, s0, (__nv_bfloat16 *)o, st_out, H, T, seg_len, nseg,
-            flags, reinterpret_cast<unsigned int *>(ws));
+            flags, onorm, reinterpret_cast<unsigned int *>(ws));
     };
     const SegPlan sp = seg_plan(B, H, T);
     if (sp.nseg == 1) {

@@ -85,6 +85,28 @@ GDN2_API int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const f
                    int d_v, int C, int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The same prefill with the layer's input and output edges fused into the kernel (page
+ * "NVIDIA представила Gated DeltaNet-2 ...", the paragraph on the layer: q and k pass an L2
+ * norm, the gates are sigmoid projections, the output goes through RMSNorm).  Per (b, t, h):
+ *
+ *   q = q_raw / max(|q_raw|_2, 1e-6),   k = k_raw / max(|k_raw|_2, 1e-6)
+ *   b = sigmoid(b_logit),   w = sigmoid(w_logit),   alpha = exp(-softplus(a_logit))
+ *   o = recurrence output; if o_weight != NULL:  o <- o / sqrt(mean_v(o^2) + 1e-6) * o_weight
+ *
+ *   q_raw, k_raw, b_logit [B, T, H, d_k]  bf16
+ *   v, w_logit            [B, T, H, d_v]  bf16
+ *   a_logit               [B, T, H, d_k]  fp32
+ *   o_weight              [d_v] fp32 RMSNorm weight shared by the heads, or NULL (no norm)
+ * Everything else as gdn2_chunk_fwd (same workspace size).  Only bf16 tokens with
+ * d_k = d_v = 128 and C = 64 are supported (GDN2_ERR_UNSUPPORTED otherwise).
+ */
+GDN2_API int gdn2_chunk_fwd_edges(const void *q_raw, const void *k_raw, const void *v, const float *a_logit,
+                                  const void *b_logit, const void *w_logit, const float *S0,
+                                  const float *o_weight, void *o, float *S_T, int B, int H, int T, int d_k,
+                                  int d_v, int C, int dtype, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
  * One decode token per sequence, state updated in place (constant memory per token,
  * page "NVIDIA улучшила память LLM ...", section "Контекст").
  *

@@ -139,3 +139,41 @@ def rel_err(x, y):
     if den == 0.0:
         return num
     return num / den
+
+
+# ----------------------------------------------------------------------------- layer edges
+# The layer around the recurrence (page "NVIDIA представила Gated DeltaNet-2 ...", the paragraph on
+# the layer: q and k pass an L2 norm, the gates b and w are sigmoid projections, the output goes
+# through RMSNorm).  The pages fix neither the norms' epsilons nor how the decay is produced from
+# its projection; the readings taken: eps = 1e-6 in both norms, alpha = exp(-softplus(a)).  All fp64.
+
+NORM_EPS = 1e-6
+RMS_EPS = 1e-6
+
+
+def sigmoid(x):
+    x = _f64(x)
+    return 0.5 * (1.0 + np.tanh(0.5 * x))
+
+
+def softplus(x):
+    x = _f64(x)
+    return np.logaddexp(0.0, x)
+
+
+def l2_normalize(x, eps=NORM_EPS):
+    """x / max(|x|_2, eps) over the last axis."""
+    x = _f64(x)
+    return x / np.maximum(np.linalg.norm(x, axis=-1, keepdims=True), eps)
+
+
+def layer_edges(q_raw, k_raw, a_logit, b_logit, w_logit):
+    """Recurrence inputs (q, k, alpha, b, w) from the layer's raw inputs."""
+    return (l2_normalize(q_raw), l2_normalize(k_raw), np.exp(-softplus(a_logit)), sigmoid(b_logit),
+            sigmoid(w_logit))
+
+
+def rms_norm(o, weight, eps=RMS_EPS):
+    """o / sqrt(mean(o^2) + eps) * weight over the last axis."""
+    o = _f64(o)
+    return o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps) * _f64(weight)

@@ -1,0 +1,120 @@
+"""GPU parity of gdn2_chunk_fwd_edges (the prefill with the layer edges fused) against the fp64
+oracle: oracle.layer_edges on the stored raw inputs, the recurrence, oracle.rms_norm."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.gpu_util import TOL, assert_close, cuda_or_skip, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def raw_inputs(B, T, H, seed, chains=None, t_range=None):
+    """Seeded raw layer inputs ([B,T,H,d], or [n,T,d] for a list of (b, h) chains): unnormalised
+    q, k (scale 3), v ~ N(0,1), decay logits ~ N(1,1) (fp32), gate logits ~ N(0,1)."""
+    K = V = 128
+    t0, t1 = (0, T) if t_range is None else t_range
+    if chains is None:
+        idx = None
+        n = B * (t1 - t0) * H
+    else:
+        t = np.arange(t0, t1, dtype=np.uint64)
+        idx = np.concatenate([(np.uint64(b) * np.uint64(T) + t) * np.uint64(H) + np.uint64(h) for b, h in chains])
+        n = idx.size
+    r = lambda st, d, mu=0.0, scale=1.0, bf16=True: synth.rows(seed, st, synth.KIND_NORMAL, d, row_index=idx,
+                                                               nrows=n, mu=mu, scale=scale, bf16=bf16)
+    x = {"q": r(0, K, scale=3.0), "k": r(1, K, scale=3.0), "v": r(2, V), "a": r(3, K, mu=1.0, bf16=False),
+         "b": r(4, K), "w": r(5, V)}
+    shape = (B, t1 - t0, H) if chains is None else (len(chains), t1 - t0)
+    return {key: a.reshape(*shape, a.shape[-1]) for key, a in x.items()}
+
+
+def to_dev(torch, x):
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda().to(torch.float32 if k == "a" else torch.bfloat16)
+            for k, v in x.items()}
+
+
+def assert_normed_close(name, got, ref_o, weight, tol):
+    """RMSNorm output against the oracle: the norm turns each row's error relative to the largest
+    row of o into an error relative to that row, so row i may deviate by tol * max_j |o_j| / |o_i|
+    (relative to its own normalised size); this is the bf16 bound on o carried through the norm."""
+    ref = oracle.rms_norm(ref_o, weight)
+    rn_o = np.sqrt(np.mean(ref_o * ref_o, axis=-1))
+    rn = np.sqrt(np.mean(ref * ref, axis=-1))
+    err_row = np.sqrt(np.mean((got - ref) ** 2, axis=-1))
+    allow = tol * rn * np.maximum(1.0, rn_o.max() / np.maximum(rn_o, 1e-30))
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    worst = np.max(err_row / allow)
+    assert worst <= 1.0, f"{name}: row error {worst:.2f} x its allowance"
+
+
+def reference(x, S0):
+    q, k, alpha, b, w = oracle.layer_edges(x["q"], x["k"], x["a"], x["b"], x["w"])
+    return oracle.recurrence(q, k, x["v"], alpha, b, w, S0)
+
+
+def run(torch, g, xd, S0, weight):
+    B, T, H, K = xd["q"].shape
+    o = torch.full((B, T, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ST = torch.full((B, H, K, 128), float("nan"), dtype=torch.float32, device="cuda")
+    g.gdn2_chunk_fwd_edges(xd["q"], xd["k"], xd["v"], xd["a"], xd["b"], xd["w"], S0, weight, o, ST)
+    torch.cuda.synchronize()
+    return o, ST
+
+
+@pytest.mark.parametrize("norm", [False, True])
+@pytest.mark.parametrize("T", [1, 64, 200])
+def test_edges_small(norm, T):
+    torch, g = cuda_or_skip()
+    x = raw_inputs(2, T, 3, seed=91)
+    S0 = np.random.default_rng(7).normal(scale=0.05, size=(2, 3, 128, 128)).astype(np.float32)
+    weight = np.random.default_rng(8).normal(size=128).astype(np.float32) if norm else None
+    o, ST = run(torch, g, to_dev(torch, x), torch.from_numpy(S0).cuda(),
+                None if weight is None else torch.from_numpy(weight).cuda())
+    ref_o, ref_S = reference(x, S0)
+    if weight is None:
+        assert_close("o", f64(o), ref_o, TOL["bf16"])
+    else:
+        assert_normed_close("o", f64(o), ref_o, weight, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
+def test_edges_segmented_long_chain():
+    """Few chains, 41 chunks: the segmented path runs with the edges fused as well."""
+    torch, g = cuda_or_skip()
+    x = raw_inputs(1, 64 * 40 + 37, 2, seed=92)
+    S0 = np.random.default_rng(9).normal(scale=0.05, size=(1, 2, 128, 128)).astype(np.float32)
+    weight = np.random.default_rng(10).normal(size=128).astype(np.float32)
+    o, ST = run(torch, g, to_dev(torch, x), torch.from_numpy(S0).cuda(), torch.from_numpy(weight).cuda())
+    ref_o, ref_S = reference(x, S0)
+    assert_normed_close("o", f64(o), ref_o, weight, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
+def test_edges_full_size_sampled():
+    """The 1.3B-layer prefill shape (B8 H16 T4096) from raw inputs, four chains checked."""
+    torch, g = cuda_or_skip()
+    B, T, H = 8, 4096, 16
+    x = raw_inputs(B, T, H, seed=93)
+    weight = np.random.default_rng(11).normal(size=128).astype(np.float32)
+    o, ST = run(torch, g, to_dev(torch, x), None, torch.from_numpy(weight).cuda())
+    del x
+    chains = [(0, 0), (2, 9), (5, 4), (7, 15)]
+    xs = raw_inputs(B, T, H, seed=93, chains=chains)
+    q, k, alpha, b, w = oracle.layer_edges(xs["q"], xs["k"], xs["a"], xs["b"], xs["w"])
+    ref_o, ref_S = oracle.chain_recurrence(q, k, xs["v"], alpha, b, w)
+    for n, (bb, h) in enumerate(chains):
+        assert_normed_close(f"o chain {bb},{h}", f64(o[bb, :, h]), ref_o[n], weight, TOL["bf16"])
+        assert_close(f"S_T chain {bb},{h}", f64(ST[bb, h]), ref_S[n], TOL["bf16"])
+
+
+def test_edges_rejects_unsupported_shapes():
+    torch, g = cuda_or_skip()
+    x = to_dev(torch, raw_inputs(1, 64, 1, seed=94))
+    small = {k: v[..., :64].contiguous() for k, v in x.items()}
+    o = torch.empty((1, 64, 1, 64), dtype=torch.bfloat16, device="cuda")
+    ST = torch.empty((1, 1, 64, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(g.GDN2Error):
+        g.gdn2_chunk_fwd_edges(small["q"], small["k"], small["v"], small["a"], small["b"], small["w"], None, None,
+                               o, ST)
