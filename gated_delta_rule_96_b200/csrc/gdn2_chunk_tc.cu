@@ -133,29 +133,30 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
     return *reinterpret_cast<uint32_t *>(&r);
 }
-// tf32 operand of mma.sync: the fp32 bit pattern (the tensor core reads the top 19 bits, i.e.
-// truncates the mantissa to 10 bits; T ends up in bf16, far coarser)
 // Layer edges fused into the prefill (the layer around the recurrence: q and k L2-normalised per
 // token and head, b and w sigmoid gates, the decay from a logit, the output through RMSNorm).
 constexpr float EDGE_NORM_EPS = 1e-6f;   // q / max(|q|, eps), likewise k
 constexpr float EDGE_RMS_EPS = 1e-6f;    // o / sqrt(mean(o^2) + eps) * weight
-__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
-// alpha = exp(-softplus(a)) = 1 / (1 + e^a) (0 past fp32's range: the caller floors it)
-__device__ __forceinline__ float alpha_of_logit(float a) { return __fdividef(1.f, 1.f + __expf(a)); }
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// sigmoid(x) = 1 / (1 + 2^(-x log2 e)); the exponential saturates to +inf (result 0) or 0 (result 1)
+__device__ __forceinline__ float sigmoid_f(float x) { return fast_rcp(1.f + fast_exp2(-1.4426950408889634f * x)); }
+// alpha = exp(-softplus(a)) = 1 / (1 + e^a) = sigmoid(-a) (0 past fp32's range: the caller floors it)
+__device__ __forceinline__ float alpha_of_logit(float a) { return fast_rcp(1.f + fast_exp2(1.4426950408889634f * a)); }
 // log2 of alpha = exp(-softplus(a)), floored at log2 of the smallest normal float
 __device__ __forceinline__ float log2_alpha_of_logit(float a) {
     const float sp = a > 15.f ? a : __logf(1.f + __expf(a));
     return fmaxf(-sp * 1.4426950408889634f, -126.f);
 }
-// two bf16 values scaled by s, rounded to bf16
-__device__ __forceinline__ uint32_t bscale2(uint32_t a, float s) {
-    const float2 f = unpack2(a);
-    return pack_bf16(f.x * s, f.y * s);
-}
 __device__ __forceinline__ uint32_t bsigmoid2(uint32_t a) {
     const float2 f = unpack2(a);
     return pack_bf16(sigmoid_f(f.x), sigmoid_f(f.y));
 }
+// tf32 operand of mma.sync: the fp32 bit pattern (the tensor core reads the top 19 bits, i.e.
+// truncates the mantissa to 10 bits; T ends up in bf16, far coarser)
 __device__ __forceinline__ uint32_t tf32(float x) { return __float_as_uint(x); }
 // D(16x8) += A(16x8) B(8x8), tf32 inputs, fp32 accumulate (warp-level)
 __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -433,9 +434,11 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
             rk[p] = __ldg(reinterpret_cast<const uint2 *>(c.k + row * KD + c4));
             rb[p] = __ldg(reinterpret_cast<const uint2 *>(c.b + row * KD + c4));
         }
+        // layer edges: alpha = exp(-softplus(alpha logit)) here; q and k are divided by their norms
+        // over the 128 channels (4 per lane: a warp holds a row) and b = sigmoid(b logit) where they
+        // are used.  Lane l keeps the inverse norms of the warp's position l / 2.
+        float iq_l = 1.f, ik_l = 1.f;
         if (EDGES) {
-            // q, k divided by their norms over the 128 channels (4 per lane: a warp holds a row),
-            // b = sigmoid(b logit), alpha = exp(-softplus(alpha logit))
 #pragma unroll
             for (int p = 0; p < 16; ++p) {
                 const float2 qa = unpack2(rq[p].x), qb = unpack2(rq[p].y), ka = unpack2(rk[p].x), kb = unpack2(rk[p].y);
@@ -446,14 +449,12 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                     sq += __shfl_xor_sync(0xffffffffu, sq, msk);
                     sk += __shfl_xor_sync(0xffffffffu, sk, msk);
                 }
-                const float iq = rsqrtf(fmaxf(sq, EDGE_NORM_EPS * EDGE_NORM_EPS));
-                const float ik = rsqrtf(fmaxf(sk, EDGE_NORM_EPS * EDGE_NORM_EPS));
-                rq[p] = make_uint2(bscale2(rq[p].x, iq), bscale2(rq[p].y, iq));
-                rk[p] = make_uint2(bscale2(rk[p].x, ik), bscale2(rk[p].y, ik));
-                rb[p] = make_uint2(bsigmoid2(rb[p].x), bsigmoid2(rb[p].y));
+                if ((lane >> 1) == p) { iq_l = sq; ik_l = sk; }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) al[p][j] = alpha_of_logit(al[p][j]);
             }
+            iq_l = rsqrtf(fmaxf(iq_l, EDGE_NORM_EPS * EDGE_NORM_EPS));
+            ik_l = rsqrtf(fmaxf(ik_l, EDGE_NORM_EPS * EDGE_NORM_EPS));
         }
         if (n + 1 < c.NC) {   // next chunk's rows of q, k, b, alpha into L2 (one 128-B line per request)
             const int r = tid1 & 63, half = tid1 >> 6;
@@ -556,11 +557,22 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                     const int r = p0 + 8 * hf + p, pp = 8 * hf + p;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) f1[j] *= al[pp][j];
-                    const uint32_t F01 = pack_bf16(f1[0], f1[1]), F23 = pack_bf16(f1[2], f1[3]);
-                    *reinterpret_cast<uint2 *>(EQ + sw_off(r, c4, 128)) =
-                        make_uint2(bmul2(bmul2(rb[pp].x, rk[pp].x), F01), bmul2(bmul2(rb[pp].y, rk[pp].y), F23));
-                    *reinterpret_cast<uint2 *>(EQ + sw_off(64 + r, c4, 128)) =
-                        make_uint2(bmul2(rq[pp].x, F01), bmul2(rq[pp].y, F23));
+                    if (EDGES) {   // the inverse norms join the decay factors; b through its sigmoid
+                        const float iq = __shfl_sync(0xffffffffu, iq_l, 2 * pp), ik = __shfl_sync(0xffffffffu, ik_l, 2 * pp);
+                        const uint32_t b01 = bsigmoid2(rb[pp].x), b23 = bsigmoid2(rb[pp].y);
+                        *reinterpret_cast<uint2 *>(EQ + sw_off(r, c4, 128)) =
+                            make_uint2(bmul2(bmul2(b01, rk[pp].x), pack_bf16(f1[0] * ik, f1[1] * ik)),
+                                       bmul2(bmul2(b23, rk[pp].y), pack_bf16(f1[2] * ik, f1[3] * ik)));
+                        *reinterpret_cast<uint2 *>(EQ + sw_off(64 + r, c4, 128)) =
+                            make_uint2(bmul2(rq[pp].x, pack_bf16(f1[0] * iq, f1[1] * iq)),
+                                       bmul2(rq[pp].y, pack_bf16(f1[2] * iq, f1[3] * iq)));
+                    } else {
+                        const uint32_t F01 = pack_bf16(f1[0], f1[1]), F23 = pack_bf16(f1[2], f1[3]);
+                        *reinterpret_cast<uint2 *>(EQ + sw_off(r, c4, 128)) =
+                            make_uint2(bmul2(bmul2(rb[pp].x, rk[pp].x), F01), bmul2(bmul2(rb[pp].y, rk[pp].y), F23));
+                        *reinterpret_cast<uint2 *>(EQ + sw_off(64 + r, c4, 128)) =
+                            make_uint2(bmul2(rq[pp].x, F01), bmul2(rq[pp].y, F23));
+                    }
                 }
                 float f2[4];
 #pragma unroll
@@ -569,8 +581,10 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
 #pragma unroll
                 for (int p = 7; p >= 0; --p) {
                     const int r = p0 + 8 * hf + p, pp = 8 * hf + p;
+                    const float ik = EDGES ? __shfl_sync(0xffffffffu, ik_l, 2 * pp) : 1.f;
                     *reinterpret_cast<uint2 *>(KT + sw_off(r, c4, 64)) =
-                        make_uint2(bmul2(rk[pp].x, pack_bf16(f2[0], f2[1])), bmul2(rk[pp].y, pack_bf16(f2[2], f2[3])));
+                        make_uint2(bmul2(rk[pp].x, pack_bf16(EDGES ? f2[0] * ik : f2[0], EDGES ? f2[1] * ik : f2[1])),
+                                   bmul2(rk[pp].y, pack_bf16(EDGES ? f2[2] * ik : f2[2], EDGES ? f2[3] * ik : f2[3])));
 #pragma unroll
                     for (int j = 0; j < 4; ++j) f2[j] *= al[pp][j];
                 }
@@ -587,8 +601,14 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                     const float2 q01 = unpack2(rq[8 * hf + p].x), q23 = unpack2(rq[8 * hf + p].y);
                     const float2 k01 = unpack2(rk[8 * hf + p].x), k23 = unpack2(rk[8 * hf + p].y);
                     const float2 b01 = unpack2(rb[8 * hf + p].x), b23 = unpack2(rb[8 * hf + p].y);
-                    const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
-                    const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
+                    float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
+                    float bv[4] = {b01.x, b01.y, b23.x, b23.y};
+                    if (EDGES) {
+                        const float iq = __shfl_sync(0xffffffffu, iq_l, 2 * (8 * hf + p));
+                        const float ik = __shfl_sync(0xffffffffu, ik_l, 2 * (8 * hf + p));
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { qq[j] *= iq; kk[j] *= ik; bv[j] = sigmoid_f(bv[j]); }
+                    }
                     float E[4], Qh[4], Kt[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
