@@ -1,0 +1,124 @@
+"""Pins of the fp64 backward oracle (oracle/backward.py) to facts other than itself.
+
+The oracle gives the gradient of a scalar loss L through the recurrence of page
+"NVIDIA представила Gated DeltaNet-2 ...", section "Техническая схема".  Taking
+L = sum_t dO_t . o_t + sum dS_T ⊙ S_T makes dO and dS_T the loss's gradients
+at the outputs.  Pins:
+
+1. finite differences: central differences of L evaluated with the FORWARD
+   oracle (oracle/gdn2_oracle.c, itself pinned), along random directions, one
+   input at a time; the error of a central difference is O(eps^2);
+2. autograd: torch's reverse mode (fp64, CPU) through a step loop written here
+   from the update equation;
+3. closed form: alpha = 1 and b = 0 make the recurrence plain linear attention,
+   o_t = S_0^T q_t + sum_{i<=t} (k_i . q_t) u_i, whose gradients are textbook
+   sums over the causal mask.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import backward as ob
+from tests.test_oracle_pins import rand_inputs
+
+NAMES = ("q", "k", "v", "alpha", "b", "w", "S0")
+
+
+def loss(x, dO, dST):
+    o, ST = oracle.recurrence(*(x[n] for n in NAMES), threads=1)
+    return float(np.sum(dO * o) + np.sum(dST * ST))
+
+
+def problem(rng, B, T, H, K, V):
+    q, k, v, alpha, b, w, S0 = rand_inputs(rng, B, T, H, K, V, unit_k=False)
+    x = dict(zip(NAMES, (q, k, v, alpha, b, w, S0)))
+    dO = rng.standard_normal((B, T, H, V))
+    dST = rng.standard_normal((B, H, K, V))
+    return x, dO, dST
+
+
+def directional_errors(rng, x, dO, dST, grads, eps=1e-5):
+    """|central difference - <grad, d>| / scale for a random direction d per input."""
+    errs = {}
+    for name, g in zip(NAMES, grads):
+        d = rng.standard_normal(x[name].shape)
+        xp = dict(x)
+        xm = dict(x)
+        xp[name] = x[name] + eps * d
+        xm[name] = x[name] - eps * d
+        fd = (loss(xp, dO, dST) - loss(xm, dO, dST)) / (2 * eps)
+        an = float(np.sum(g * d))
+        errs[name] = abs(fd - an) / max(1.0, abs(an))
+    return errs
+
+
+@pytest.mark.parametrize("T,K,V", [(1, 3, 2), (4, 3, 5), (9, 5, 4)])
+def test_finite_differences(rng, T, K, V):
+    x, dO, dST = problem(rng, 1, T, 2, K, V)
+    grads = ob.recurrence_backward(*(x[n] for n in NAMES), dO, dST)
+    errs = directional_errors(rng, x, dO, dST, grads)
+    assert max(errs.values()) < 1e-8, errs
+
+
+def test_finite_differences_without_state_gradient(rng):
+    """dS_T = 0 and S_0 = 0 (the defaults): only the outputs o carry gradient."""
+    x, dO, _ = problem(rng, 1, 6, 1, 4, 3)
+    x["S0"] = np.zeros_like(x["S0"])
+    zero = np.zeros((1, 1, 4, 3))
+    grads = ob.recurrence_backward(*(x[n] for n in NAMES[:-1]), None, dO, None)
+    errs = directional_errors(rng, x, dO, zero, grads)
+    assert max(errs.values()) < 1e-8, errs
+
+
+def test_autograd(rng):
+    torch = pytest.importorskip("torch")
+    B, T, H, K, V = 1, 12, 2, 6, 5
+    x, dO, dST = problem(rng, B, T, H, K, V)
+    tx = {n: torch.tensor(x[n], dtype=torch.float64, requires_grad=True) for n in NAMES}
+    L = 0.0
+    for h in range(H):
+        S = tx["S0"][0, h]
+        for t in range(T):
+            kt, qt = tx["k"][0, t, h], tx["q"][0, t, h]
+            et = tx["b"][0, t, h] * kt
+            ut = tx["w"][0, t, h] * tx["v"][0, t, h]
+            M = torch.eye(K, dtype=torch.float64) - torch.outer(kt, et)
+            S = M @ (tx["alpha"][0, t, h][:, None] * S) + torch.outer(kt, ut)
+            L = L + torch.dot(torch.tensor(dO[0, t, h]), S.T @ qt)
+        L = L + torch.sum(torch.tensor(dST[0, h]) * S)
+    L.backward()
+    grads = ob.recurrence_backward(*(x[n] for n in NAMES), dO, dST)
+    for n, g in zip(NAMES, grads):
+        np.testing.assert_allclose(g, tx[n].grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=n)
+
+
+def test_linear_attention_closed_form(rng):
+    """alpha = 1, b = 0: o_t = S0^T q_t + sum_{i<=t} (q_t . k_i) u_i and S_T = S0 + sum_i k_i u_i^T."""
+    T, K, V = 7, 4, 3
+    x, dO, dST = problem(rng, 1, T, 1, K, V)
+    x["alpha"] = np.ones_like(x["alpha"])
+    x["b"] = np.zeros_like(x["b"])
+    g = ob.recurrence_backward(*(x[n] for n in NAMES), dO, dST)
+    q, k, v, w, S0 = (x[n][0, :, 0] if n != "S0" else x[n][0, 0] for n in ("q", "k", "v", "w", "S0"))
+    do, dst = dO[0, :, 0], dST[0, 0]
+    u = w * v
+    mask = np.tril(np.ones((T, T)))                 # mask[t, i] = 1 for i <= t
+    qk = (q @ k.T) * mask                            # (q_t . k_i) for i <= t
+    du_ref = qk.T @ do + k @ dst                     # du_i = sum_{t>=i} (q_t.k_i) dO_t + dS_T^T k_i
+    dk_ref = ((do @ u.T) * mask).T @ q + u @ dst.T   # dk_i = sum_{t>=i} (dO_t.u_i) q_t + dS_T u_i
+    dq_ref = ((do @ u.T) * mask) @ k + do @ S0.T     # dq_t = sum_{i<=t} (dO_t.u_i) k_i + S0 dO_t
+    dS0_ref = q.T @ do + dst
+    np.testing.assert_allclose(g[0][0, :, 0], dq_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g[1][0, :, 0], dk_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g[2][0, :, 0], w * du_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g[5][0, :, 0], v * du_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g[6][0, 0], dS0_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_empty_sequence(rng):
+    """T = 0: S_T = S_0, so dS0 = dS_T and there are no token gradients."""
+    x, dO, dST = problem(rng, 1, 1, 1, 3, 2)
+    g = ob.chain_backward(*(np.zeros((0, 3)) if n in ("q", "k", "alpha", "b") else np.zeros((0, 2))
+                            for n in NAMES[:-1]), x["S0"][0, 0], np.zeros((0, 2)), dST[0, 0])
+    assert all(a.shape[0] == 0 for a in g[:6])
+    np.testing.assert_array_equal(g[6], dST[0, 0])
