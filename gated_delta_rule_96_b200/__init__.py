@@ -18,7 +18,7 @@ __all__ = [
     "GDN2Error", "load_library", "library_path", "gdn2_chunk_fwd", "gdn2_chunk_fwd_edges", "gdn2_decode_step",
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
-    "chunk_fwd", "decode_step", "new_workspace",
+    "chunk_fwd", "decode_step", "new_workspace", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,6 +65,10 @@ def load_library():
     lib.gdn2_chunk_fwd_noalloc.restype = i
     lib.gdn2_chunk_fwd_edges.argtypes = [vp] * 10 + [i] * 7 + [vp, sz, vp]
     lib.gdn2_chunk_fwd_edges.restype = i
+    lib.gdn2_chunk_bwd_workspace_bytes.argtypes = [i] * 5
+    lib.gdn2_chunk_bwd_workspace_bytes.restype = sz
+    lib.gdn2_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
+    lib.gdn2_chunk_bwd.restype = i
     lib.gdn2_status_str.argtypes = [i]
     lib.gdn2_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -177,6 +181,40 @@ def gdn2_chunk_fwd_edges(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o_weigh
                                              workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_fwd_edges")
+
+
+def gdn2_chunk_bwd_workspace_bytes(B, H, T, d_k, d_v) -> int:
+    return int(load_library().gdn2_chunk_bwd_workspace_bytes(B, H, T, d_k, d_v))
+
+
+def gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, workspace=None,
+                   stream=None) -> None:
+    """Backward of the recurrence (include/gdn2.h, gdn2_chunk_bwd): fp32 gradients of every forward
+    input from dO (token dtype) and dS_T (fp32 or None); dS0 may be None."""
+    import torch
+    _check_cuda(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, workspace)
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    dt = _dtype_code(q)
+    for name, t in (("alpha", alpha), ("S0", S0), ("dS_T", dS_T), ("dq", dq), ("dk", dk), ("dv", dv),
+                    ("dalpha", dalpha), ("db", db), ("dw", dw), ("dS0", dS0)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    if dO.dtype != q.dtype:
+        raise TypeError("dO must have the token dtype")
+    tk, tv, st = (B, T, H, K), (B, T, H, V), (B, H, K, V)
+    for name, t, shp in (("k", k, tk), ("b", b, tk), ("alpha", alpha, tk), ("v", v, tv), ("w", w, tv),
+                         ("dO", dO, tv), ("S0", S0, st), ("dS_T", dS_T, st), ("dq", dq, tk), ("dk", dk, tk),
+                         ("dalpha", dalpha, tk), ("db", db, tk), ("dv", dv, tv), ("dw", dw, tv), ("dS0", dS0, st)):
+        if t is not None and tuple(t.shape) != shp:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    if workspace is None:
+        workspace = new_workspace(max(gdn2_chunk_bwd_workspace_bytes(B, H, T, K, V), 256), q.device)
+    rc = load_library().gdn2_chunk_bwd(*(_ptr(t) for t in (q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha,
+                                                           db, dw, dS0)), B, H, T, K, V, dt, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_chunk_bwd")
 
 
 def gdn2_chunk_fwd_noalloc(q, k, v, alpha, b, w, S0, o, S_T, C=64, stream=None) -> None:

@@ -28,4 +28,11 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
                     const void *w, const float *S0, void *o, float *ST, int B, int H, int T, int K, int V,
                     int C, void *ws, cudaStream_t st, int edges = 0, const float *onorm = nullptr);
 
+// Backward pass (three sequential passes per chain; fp32 gradients; d_k, d_v in {64, 128}).
+size_t bwd_workspace_bytes(int B, int H, int T, int K, int V);
+int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                     const float *S0, const void *dO, const float *dST, float *dq, float *dk, float *dv,
+                     float *dalpha, float *db, float *dw, float *dS0, int B, int H, int T, int K, int V, int bf16,
+                     void *ws, cudaStream_t st);
+
 }  // namespace gdn2

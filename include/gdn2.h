@@ -120,6 +120,37 @@ GDN2_API int gdn2_decode_step(const void *q, const void *k, const void *v, const
                      const void *w, float *S, void *o, int B, int H, int d_k, int d_v, int dtype,
                      void *stream);
 
+/* Bytes of device workspace gdn2_chunk_bwd needs (0 on bad sizes).  Depends only on its
+ * arguments: two fp32 [B, T, H, d_v] buffers, the fp32 state at every 64th step of every
+ * chain, and one fp32 d_k vector per 64 steps per chain. */
+GDN2_API size_t gdn2_chunk_bwd_workspace_bytes(int B, int H, int T, int d_k, int d_v);
+
+/*
+ * Backward pass of the recurrence: the gradients of a scalar loss L with respect to every
+ * input of gdn2_chunk_fwd, given the loss's gradients at its outputs (page "NVIDIA
+ * представила Gated DeltaNet-2 ...", the paragraph on the chunkwise kernels: the backward
+ * needs gradients that account for the per-channel gates).
+ *
+ *   q, k, v, alpha, b, w, S0   the forward's inputs, same layouts and dtypes (S0 may be NULL)
+ *   dO        [B, T, H, d_v]   token dtype, dL/do
+ *   dS_T      [B, H, d_k, d_v] fp32, dL/dS_T, or NULL for zero
+ *   dq, dk, db, dalpha (out)   [B, T, H, d_k] fp32
+ *   dv, dw             (out)   [B, T, H, d_v] fp32
+ *   dS0                (out)   [B, H, d_k, d_v] fp32, dL/dS0, or NULL if not wanted
+ *   workspace  device scratch of at least gdn2_chunk_bwd_workspace_bytes(...) bytes, 16-byte
+ *              aligned, no initialisation needed (no status header: these kernels never wait)
+ *
+ * Every gradient is computed and written in fp32 whatever the token dtype.  dalpha is
+ * formed as d(log alpha) / alpha with alpha floored at FLT_MIN.  T = 0 writes dS0 = dS_T
+ * (or zeros) and reads no token pointer.  d_k, d_v in {64, 128}.  The output buffers must
+ * not alias the inputs or each other.  Three kernel launches on `stream`.
+ */
+GDN2_API int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                            const void *w, const float *S0, const void *dO, const float *dS_T, float *dq,
+                            float *dk, float *dv, float *dalpha, float *db, float *dw, float *dS0, int B, int H,
+                            int T, int d_k, int d_v, int dtype, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
 /* Reads the device status word of a workspace (synchronises `stream` first).
  * *out receives 0 when every kernel that used this workspace finished normally, or a
  * nonzero code naming the first internal error.  With clear != 0 the word is reset.

@@ -118,3 +118,36 @@ def test_binding_refuses_cpu_tensors():
     a = torch.zeros((1, 4, 1, 64))
     with pytest.raises(ValueError, match="CUDA"):
         g.gdn2_chunk_fwd(x, x, x, a, x, x, None, x, torch.zeros(1, 1, 64, 64))
+
+
+def test_bwd_workspace_bytes():
+    a = lambda n: (n + 255) // 256 * 256
+    ntok, state = 8 * 4096 * 16, 4 * 128 * 128
+    # two fp32 [B,T,H,d_v] buffers, the state every 64 steps, one d_k vector every 64 steps
+    assert g.gdn2_chunk_bwd_workspace_bytes(8, 16, 4096, 128, 128) == \
+        2 * a(4 * ntok * 128) + a(128 * 64 * state) + a(128 * 64 * 4 * 128)
+    # a ragged tail costs a whole chunk of checkpoints
+    assert g.gdn2_chunk_bwd_workspace_bytes(1, 1, 65, 64, 128) == \
+        2 * a(4 * 65 * 128) + a(2 * 4 * 64 * 128) + a(2 * 4 * 64)
+    assert g.gdn2_chunk_bwd_workspace_bytes(1, 1, 8, 96, 128) == 0
+
+
+def call_bwd(lib, B=1, H=1, T=8, K=128, V=128, dtype=1, ptr=FAKE, grad=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return lib.gdn2_chunk_bwd(*(ptr,) * 6, None, ptr, None, *(grad,) * 6, None, B, H, T, K, V, dtype, ws,
+                              ws_bytes, None)
+
+
+def test_chunk_bwd_validation(lib):
+    assert call_bwd(lib, T=-1) == -2
+    assert call_bwd(lib, H=-1) == -2
+    assert call_bwd(lib, dtype=5) == -3
+    assert call_bwd(lib, K=32) == -4
+    assert call_bwd(lib, ptr=None) == -1
+    assert call_bwd(lib, grad=None) == -1
+    assert call_bwd(lib, ptr=P(0x10004)) == -7
+    assert call_bwd(lib, grad=P(0x10008)) == -7
+    assert call_bwd(lib, ws=None) == -5
+    assert call_bwd(lib, ws_bytes=64) == -5
+    assert call_bwd(lib, B=0) == 0
+    # no tokens and no dS0 wanted: nothing to do, no pointer read
+    assert call_bwd(lib, T=0, ptr=None, grad=None, ws=None, ws_bytes=0) == 0
