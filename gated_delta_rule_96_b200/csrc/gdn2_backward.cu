@@ -29,9 +29,12 @@
 //
 // Layout (one CTA per (b, h) chain, d_v / 8 warps): warp w owns the value columns
 // 8w .. 8w+7 of the carried matrix, lane l the key rows KR*l .. KR*l+KR-1 (KR = d_k / 32);
-// the matrix lives in registers.  Column sums over the key axis (feeding the recurrence)
-// stay inside the warp (a shuffle reduce-scatter); row sums over the value axis (outputs
-// only) go through shared memory and are flushed every NB steps.
+// the matrix lives in registers as column pairs, updated with the packed two-wide fp32
+// FMA of sm_100.  Column sums over the key axis (feeding the recurrence) stay inside the
+// warp (a shuffle reduce-scatter); row sums over the value axis (outputs only) go through
+// shared memory and are flushed every NB steps.  The token rows of each block of NB steps
+// are copied into shared memory with cp.async two blocks ahead, so the step loop reads
+// only registers and shared memory.
 #include <float.h>
 
 #include "gdn2_common.cuh"
@@ -40,58 +43,81 @@
 namespace gdn2 {
 namespace bwd {
 
-constexpr int C = 64;    // chunk length: checkpoint spacing and the span of the log-decay sums
-constexpr int NB = 16;   // steps per flush of the row sums (divides C)
-constexpr int PF = 16;   // steps of look-ahead for the L2 prefetch
-static_assert(C % NB == 0, "chunk ends must be flush ends");
+constexpr int C = 64;   // chunk length: checkpoint spacing and the span of the log-decay sums
+constexpr int NB = 8;   // steps per block: row-sum flush and cp.async staging unit (divides C)
+static_assert(C % NB == 0, "chunk ends must be block ends");
 
 __device__ __forceinline__ float2 bf2(uint32_t u) {
     __nv_bfloat162 p = *reinterpret_cast<__nv_bfloat162 *>(&u);
     return make_float2(__low2float(p), __high2float(p));
 }
 
-// KR consecutive token values (a lane's rows) as fp32
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// all but the most recent group complete (this thread's copies)
+__device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// n consecutive steps' rows of one token tensor (E elements per row, rows H apart) -> smem [n][E]
+template <int E, typename T>
+__device__ __forceinline__ void stage_rows(T *dst, const T *src, size_t row0, int H, int n, int tid, int NT) {
+    constexpr int PPR = E * (int)sizeof(T) / 16;   // 16-byte pieces per row
+    for (int p = tid; p < n * PPR; p += NT) {
+        const int s = p / PPR, c = p - s * PPR;
+        cp_async16(reinterpret_cast<char *>(dst + s * E) + 16 * c,
+                   reinterpret_cast<const char *>(src + (row0 + (size_t)s * H) * E) + 16 * c);
+    }
+}
+
+// a lane's KR consecutive values of a staged row, as fp32
 template <int KR>
-__device__ __forceinline__ void ld_rows(const float *p, float (&x)[KR]) {
+__device__ __forceinline__ void rows_of(const float *p, float (&x)[KR]) {
     if constexpr (KR == 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+        const float4 a = *reinterpret_cast<const float4 *>(p);
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
     } else {
-        const float2 a = __ldg(reinterpret_cast<const float2 *>(p));
+        const float2 a = *reinterpret_cast<const float2 *>(p);
         x[0] = a.x; x[1] = a.y;
     }
 }
 template <int KR>
-__device__ __forceinline__ void ld_rows(const __nv_bfloat16 *p, float (&x)[KR]) {
+__device__ __forceinline__ void rows_of(const __nv_bfloat16 *p, float (&x)[KR]) {
     if constexpr (KR == 4) {
-        const uint2 a = __ldg(reinterpret_cast<const uint2 *>(p));
+        const uint2 a = *reinterpret_cast<const uint2 *>(p);
         const float2 l = bf2(a.x), h = bf2(a.y);
         x[0] = l.x; x[1] = l.y; x[2] = h.x; x[3] = h.y;
     } else {
-        const float2 l = bf2(__ldg(reinterpret_cast<const unsigned int *>(p)));
+        const float2 l = bf2(*reinterpret_cast<const uint32_t *>(p));
         x[0] = l.x; x[1] = l.y;
     }
 }
-// 8 consecutive values (a warp's columns) as fp32; every lane reads the same address
-__device__ __forceinline__ void ld_cols8(const float *p, float (&x)[8]) {
+// a warp's 8 consecutive values (every lane reads the same address), as 4 column pairs
+__device__ __forceinline__ void cols_of(const float *p, float2 (&x)[4]) {
+    const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+    x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w); x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
+}
+__device__ __forceinline__ void cols_of(const __nv_bfloat16 *p, float2 (&x)[4]) {
+    const uint4 a = *reinterpret_cast<const uint4 *>(p);
+    x[0] = bf2(a.x); x[1] = bf2(a.y); x[2] = bf2(a.z); x[3] = bf2(a.w);
+}
+// global fp32 [8] at p (16-byte aligned) as column pairs
+__device__ __forceinline__ void cols_global(const float *p, float2 (&x)[4]) {
     const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w); x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
 }
-__device__ __forceinline__ void ld_cols8(const __nv_bfloat16 *p, float (&x)[8]) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
-    const float2 f0 = bf2(a.x), f1 = bf2(a.y), f2 = bf2(a.z), f3 = bf2(a.w);
-    x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y; x[4] = f2.x; x[5] = f2.y; x[6] = f3.x; x[7] = f3.y;
+__device__ __forceinline__ void store_cols(float *p, const float2 (&x)[4]) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
 }
-// fp32 values written by an earlier pass of the same call (plain loads: not read-only data)
-__device__ __forceinline__ void ld_ws8(const float *p, float (&x)[8]) {
-    const float4 a = *reinterpret_cast<const float4 *>(p), b = *(reinterpret_cast<const float4 *>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
+__device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
 
 // Sum over the 32 lanes of eight per-lane values p[0..7]; lane l receives the sum of
 // p[(l >> 2) & 7].  Lanes differing in bit 4, then 3, then 2 exchange half of what they
 // hold (4, 2, 1 values), then bits 1 and 0 finish: 9 shuffles instead of 40.
-__device__ __forceinline__ float warp_colsum8(const float (&p)[8], int lane) {
+__device__ __forceinline__ float warp_colsum8(const float2 (&p2)[4], int lane) {
+    const float p[8] = {p2[0].x, p2[0].y, p2[1].x, p2[1].y, p2[2].x, p2[2].y, p2[3].x, p2[3].y};
     const bool h4 = (lane & 16) != 0, h3 = (lane & 8) != 0, h2 = (lane & 4) != 0;
     float a[4], c[2];
 #pragma unroll
@@ -105,18 +131,16 @@ __device__ __forceinline__ float warp_colsum8(const float (&p)[8], int lane) {
     s += __shfl_xor_sync(0xffffffffu, s, 1);
     return s;
 }
-
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-// lane i of the calling warp prefetches the i-th 128-byte line of [p, p + bytes)
-__device__ __forceinline__ void prefetch_row(const void *p, int bytes, int lane) {
-    if (lane * 128 < bytes) prefetch_l2(static_cast<const char *>(p) + lane * 128);
+// the eight column values held by lanes 0, 4, ..., 28, as pairs in every lane
+__device__ __forceinline__ void broadcast8(float mine, float2 (&d)[4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        d[p] = make_float2(__shfl_sync(0xffffffffu, mine, 8 * p), __shfl_sync(0xffffffffu, mine, 8 * p + 4));
 }
 
 __device__ __forceinline__ bool chunk_end(int t, int T) { return t == T - 1 || (t + 1) % C == 0; }
 
-// Row sums of NB buffered steps: red[s][w][c] summed over the warps w.
+// Row sums of a block: red[s][w][c] summed over the warps w.
 template <int K, int NW>
 __device__ __forceinline__ float red_sum(const float *red, int s, int c) {
     float acc = 0.f;
@@ -124,13 +148,52 @@ __device__ __forceinline__ float red_sum(const float *red, int s, int c) {
     for (int w = 0; w < NW; ++w) acc += red[(s * NW + w) * K + c];
     return acc;
 }
-
 template <int KR>
-__device__ __forceinline__ void st_red(float *red, int slot, int NW, int K, int warp, int r0, const float (&x)[KR]) {
-    float *p = red + (slot * NW + warp) * K + r0;
+__device__ __forceinline__ void st_red(float *red, int s, int NW, int K, int warp, int r0, const float (&x)[KR]) {
+    float *p = red + (s * NW + warp) * K + r0;
     if constexpr (KR == 4) *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
     else *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
 }
+
+// The carried d_k x d_v matrix: a lane's KR rows x the warp's 8 columns, as column pairs.
+template <int KR>
+using Mat = float2[KR][4];
+
+template <int KR, int K, int V>
+__device__ __forceinline__ void load_mat(Mat<KR> &M, const float *src, int r0, int c0) {
+#pragma unroll
+    for (int i = 0; i < KR; ++i) {
+        if (src) cols_global(src + (size_t)(r0 + i) * V + c0, M[i]);
+        else
+#pragma unroll
+            for (int p = 0; p < 4; ++p) M[i][p] = make_float2(0.f, 0.f);
+    }
+}
+
+// Shared-memory staging areas of one block (per buffer), as byte offsets.
+template <int K, int V, typename Tok>
+struct Stage1 {   // pass 1: alpha, k, b | v, w, dO
+    static constexpr int al = 0, kk = al + NB * K * 4, bk = kk + NB * K * (int)sizeof(Tok);
+    static constexpr int vv = bk + NB * K * (int)sizeof(Tok), ww = vv + NB * V * (int)sizeof(Tok);
+    static constexpr int go = ww + NB * V * (int)sizeof(Tok), bytes = go + NB * V * (int)sizeof(Tok);
+};
+template <int K, int V, typename Tok>
+struct Stage2 {   // pass 2: alpha, k, b, q | v, w, dO, delta
+    static constexpr int al = 0, kk = al + NB * K * 4, bk = kk + NB * K * (int)sizeof(Tok);
+    static constexpr int qq = bk + NB * K * (int)sizeof(Tok), vv = qq + NB * K * (int)sizeof(Tok);
+    static constexpr int ww = vv + NB * V * (int)sizeof(Tok), go = ww + NB * V * (int)sizeof(Tok);
+    static constexpr int dl = go + NB * V * (int)sizeof(Tok), bytes = dl + NB * V * 4;
+};
+template <int K, int V, typename Tok>
+struct Stage3 {   // pass 3: alpha, k, b, q, dq, dk | delta, ddelta
+    static constexpr int al = 0, kk = al + NB * K * 4, bk = kk + NB * K * (int)sizeof(Tok);
+    static constexpr int qq = bk + NB * K * (int)sizeof(Tok), dq = qq + NB * K * (int)sizeof(Tok);
+    static constexpr int dk = dq + NB * K * 4, dl = dk + NB * K * 4, dd = dl + NB * V * 4;
+    static constexpr int bytes = dd + NB * V * 4;
+};
+
+template <typename T>
+__device__ __forceinline__ T *at(unsigned char *base, int off) { return reinterpret_cast<T *>(base + off); }
 
 // ------------------------------------------------------------------------------------ pass 1
 // Forward over S: delta_t -> workspace, dq_t = S_t dO_t -> dq, S at every chunk end -> ckpt.
@@ -141,99 +204,97 @@ pass_forward(const Tok *__restrict__ k, const Tok *__restrict__ v, const float *
              const Tok *__restrict__ dO, float *__restrict__ dq, float *__restrict__ delta,
              float *__restrict__ ckpt, int H, int T, int NC) {
     constexpr int K = 32 * KR, V = 8 * NW, NT = NW * 32;
-    extern __shared__ float red[];   // [NB][NW][K]
+    using L = Stage1<K, V, Tok>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    float *red = reinterpret_cast<float *>(smem);                       // [NB][NW][K]
+    unsigned char *stg = smem + NB * NW * K * 4;                         // [2][L::bytes]
     const int chain = blockIdx.x, bb = chain / H, h = chain % H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r0 = KR * lane, c0 = 8 * warp, jm = (lane >> 2) & 7;
+    const int nblk = (T + NB - 1) / NB;
 
-    float S[KR][8];
-#pragma unroll
-    for (int i = 0; i < KR; ++i) {
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (S0) ld_cols8(S0 + ((size_t)chain * K + r0 + i) * V + c0, x);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) S[i][j] = x[j];
-    }
-    struct In { float al[KR], kk[KR], e[KR], u, g[8]; };
-    auto load = [&](In &in, int t) {
-        const size_t row = ((size_t)bb * T + t) * H + h;
-        float bk[KR];
-        ld_rows<KR>(alpha + row * K + r0, in.al);
-        ld_rows<KR>(k + row * K + r0, in.kk);
-        ld_rows<KR>(b + row * K + r0, bk);
-#pragma unroll
-        for (int i = 0; i < KR; ++i) in.e[i] = bk[i] * in.kk[i];
-        in.u = to_f32(w[row * V + c0 + jm]) * to_f32(v[row * V + c0 + jm]);
-        ld_cols8(dO + row * V + c0, in.g);
+    auto stage = [&](int blk) {
+        const int t0 = blk * NB, n = min(NB, T - t0);
+        if (n <= 0) return;
+        unsigned char *sb = stg + (blk & 1) * L::bytes;
+        const size_t row0 = ((size_t)bb * T + t0) * H + h;
+        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT);
+        stage_rows<V>(at<Tok>(sb, L::vv), v, row0, H, n, tid, NT);
+        stage_rows<V>(at<Tok>(sb, L::ww), w, row0, H, n, tid, NT);
+        stage_rows<V>(at<Tok>(sb, L::go), dO, row0, H, n, tid, NT);
     };
-    In cur, nxt;
-    if (T > 0) load(cur, 0);
-    for (int t = 0; t < T; ++t) {
-        if (t + 1 < T) load(nxt, t + 1);
-        if (warp == 0 && t + PF < T) {
-            const size_t row = ((size_t)bb * T + t + PF) * H + h;
-            prefetch_row(alpha + row * K, K * 4, lane);
-            prefetch_row(k + row * K, K * (int)sizeof(Tok), lane);
-            prefetch_row(b + row * K, K * (int)sizeof(Tok), lane);
-            prefetch_row(v + row * V, V * (int)sizeof(Tok), lane);
-            prefetch_row(w + row * V, V * (int)sizeof(Tok), lane);
-            prefetch_row(dO + row * V, V * (int)sizeof(Tok), lane);
-        }
-        // Sbar = Diag(alpha) S; r = Sbar^T e (column sums); delta = u - r
-        float pr[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            pr[j] = 0.f;
-#pragma unroll
-            for (int i = 0; i < KR; ++i) {
-                S[i][j] *= cur.al[i];
-                pr[j] = fmaf(S[i][j], cur.e[i], pr[j]);
-            }
-        }
-        const float dmine = cur.u - warp_colsum8(pr, lane);
-        const size_t rowt = ((size_t)bb * T + t) * H + h;
-        if ((lane & 3) == 0) delta[rowt * V + c0 + jm] = dmine;
-        float d[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) d[j] = __shfl_sync(0xffffffffu, dmine, 4 * j);
-        // S_t = Sbar + k delta^T; row sums of S_t dO_t
-        float x[KR];
-#pragma unroll
-        for (int i = 0; i < KR; ++i) {
-            x[i] = 0.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                S[i][j] = fmaf(cur.kk[i], d[j], S[i][j]);
-                x[i] = fmaf(S[i][j], cur.g[j], x[i]);
-            }
-        }
-        const int slot = t % NB;
-        st_red<KR>(red, slot, NW, K, warp, r0, x);
-        if (chunk_end(t, T)) {
-            float *ck = ckpt + ((size_t)chain * NC + t / C) * K * V;
+    Mat<KR> S;
+    load_mat<KR, K, V>(S, S0 ? S0 + (size_t)chain * K * V : nullptr, r0, c0);
+    stage(0);
+    cp_commit();
+    stage(1);
+    cp_commit();
+    cp_wait_prev();
+    __syncthreads();
+    for (int blk = 0; blk < nblk; ++blk) {
+        const int t0 = blk * NB, n = min(NB, T - t0);
+        unsigned char *sb = stg + (blk & 1) * L::bytes;
+        for (int s = 0; s < n; ++s) {
+            const int t = t0 + s;
+            float al[KR], kk[KR], bk[KR];
+            rows_of<KR>(at<float>(sb, L::al) + s * K + r0, al);
+            rows_of<KR>(at<Tok>(sb, L::kk) + s * K + r0, kk);
+            rows_of<KR>(at<Tok>(sb, L::bk) + s * K + r0, bk);
+            float2 g[4];
+            cols_of(at<Tok>(sb, L::go) + s * V + c0, g);
+            const float u = to_f32(at<Tok>(sb, L::ww)[s * V + c0 + jm]) * to_f32(at<Tok>(sb, L::vv)[s * V + c0 + jm]);
+            // Sbar = Diag(alpha) S; r = Sbar^T e (column sums); delta = u - r
+            float2 pr[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
             for (int i = 0; i < KR; ++i) {
-                float4 *p = reinterpret_cast<float4 *>(ck + (size_t)(r0 + i) * V + c0);
-                p[0] = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
-                p[1] = make_float4(S[i][4], S[i][5], S[i][6], S[i][7]);
+                const float2 a2 = splat(al[i]), e2 = splat(bk[i] * kk[i]);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    S[i][p] = __fmul2_rn(S[i][p], a2);
+                    pr[p] = __ffma2_rn(S[i][p], e2, pr[p]);
+                }
+            }
+            const float dmine = u - warp_colsum8(pr, lane);
+            if ((lane & 3) == 0) delta[(((size_t)bb * T + t) * H + h) * V + c0 + jm] = dmine;
+            float2 d[4];
+            broadcast8(dmine, d);
+            // S_t = Sbar + k delta^T; row sums of S_t dO_t
+            float x[KR];
+#pragma unroll
+            for (int i = 0; i < KR; ++i) {
+                const float2 k2 = splat(kk[i]);
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    S[i][p] = __ffma2_rn(k2, d[p], S[i][p]);
+                    acc = __ffma2_rn(S[i][p], g[p], acc);
+                }
+                x[i] = acc.x + acc.y;
+            }
+            st_red<KR>(red, s, NW, K, warp, r0, x);
+            if (chunk_end(t, T)) {
+                float *ck = ckpt + ((size_t)chain * NC + t / C) * K * V;
+#pragma unroll
+                for (int i = 0; i < KR; ++i) store_cols(ck + (size_t)(r0 + i) * V + c0, S[i]);
             }
         }
-        if (slot == NB - 1 || t == T - 1) {
-            __syncthreads();
-            const int t0 = t - slot;
-            for (int idx = tid; idx < (slot + 1) * K; idx += NT) {
-                const int s = idx / K, c = idx % K;
-                dq[(((size_t)bb * T + t0 + s) * H + h) * K + c] = red_sum<K, NW>(red, s, c);
-            }
-            __syncthreads();
+        __syncthreads();   // block done: row sums complete, its staging buffer free
+        for (int idx = tid; idx < n * K; idx += NT) {
+            const int s = idx / K, c = idx - s * K;
+            dq[(((size_t)bb * T + t0 + s) * H + h) * K + c] = red_sum<K, NW>(red, s, c);
         }
-        cur = nxt;
+        stage(blk + 2);
+        cp_commit();
+        cp_wait_prev();
+        __syncthreads();
     }
 }
 
 // ------------------------------------------------------------------------------------ pass 2
 // Reverse over G: ddelta_t -> workspace, dv, dw, dk_t = G_t delta_t (completed by pass 3),
-// rowsum(G^fut ⊙ S) at every chunk end -> bnd, dS0 = G_0.
+// rowsum(G^fut ⊙ S) at every chunk end -> bnd, dS0 = G_0.  Blocks run from the end.
 template <int KR, int NW, typename Tok>
 __global__ void __launch_bounds__(NW * 32, 1)
 pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__restrict__ v,
@@ -243,119 +304,118 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
              float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dw, float *__restrict__ dS0,
              int H, int T, int NC) {
     constexpr int K = 32 * KR, V = 8 * NW, NT = NW * 32;
-    extern __shared__ float red[];   // [NB][NW][K], then [NW][K] for the chunk-end sums
-    float *rbnd = red + NB * NW * K;
+    using L = Stage2<K, V, Tok>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    float *red = reinterpret_cast<float *>(smem);                  // [NB][NW][K]
+    float *rbnd = red + NB * NW * K;                                // [NW][K]
+    unsigned char *stg = smem + (NB + 1) * NW * K * 4;              // [2][L::bytes]
     const int chain = blockIdx.x, bb = chain / H, h = chain % H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r0 = KR * lane, c0 = 8 * warp, jm = (lane >> 2) & 7;
-
-    float G[KR][8];
-#pragma unroll
-    for (int i = 0; i < KR; ++i) {
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (dST) ld_cols8(dST + ((size_t)chain * K + r0 + i) * V + c0, x);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) G[i][j] = x[j];
-    }
-    struct In { float al[KR], kk[KR], e[KR], qq[KR], g[8], dl[8], vm, wm; };
-    auto load = [&](In &in, int t) {
-        const size_t row = ((size_t)bb * T + t) * H + h;
-        float bk[KR];
-        ld_rows<KR>(alpha + row * K + r0, in.al);
-        ld_rows<KR>(k + row * K + r0, in.kk);
-        ld_rows<KR>(b + row * K + r0, bk);
-        ld_rows<KR>(q + row * K + r0, in.qq);
-#pragma unroll
-        for (int i = 0; i < KR; ++i) in.e[i] = bk[i] * in.kk[i];
-        ld_cols8(dO + row * V + c0, in.g);
-        ld_ws8(delta + row * V + c0, in.dl);
-        in.vm = to_f32(v[row * V + c0 + jm]);
-        in.wm = to_f32(w[row * V + c0 + jm]);
+    const int nblk = (T + NB - 1) / NB;
+    // reverse block r holds steps lo(r) .. hi(r), hi(r) = T - 1 - r NB; staged at s = t - lo
+    auto lo_of = [&](int r) { return max(T - (r + 1) * NB, 0); };
+    auto stage = [&](int r) {
+        if (r >= nblk) return;
+        const int lo = lo_of(r), n = T - r * NB - lo;
+        unsigned char *sb = stg + (r & 1) * L::bytes;
+        const size_t row0 = ((size_t)bb * T + lo) * H + h;
+        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::qq), q, row0, H, n, tid, NT);
+        stage_rows<V>(at<Tok>(sb, L::vv), v, row0, H, n, tid, NT);
+        stage_rows<V>(at<Tok>(sb, L::ww), w, row0, H, n, tid, NT);
+        stage_rows<V>(at<Tok>(sb, L::go), dO, row0, H, n, tid, NT);
+        stage_rows<V>(at<float>(sb, L::dl), delta, row0, H, n, tid, NT);
     };
-    In cur, nxt;
-    if (T > 0) load(cur, T - 1);
-    for (int t = T - 1; t >= 0; --t) {
-        if (t > 0) load(nxt, t - 1);
-        if (warp == 0 && t - PF >= 0) {
-            const size_t row = ((size_t)bb * T + t - PF) * H + h;
-            prefetch_row(alpha + row * K, K * 4, lane);
-            prefetch_row(k + row * K, K * (int)sizeof(Tok), lane);
-            prefetch_row(b + row * K, K * (int)sizeof(Tok), lane);
-            prefetch_row(q + row * K, K * (int)sizeof(Tok), lane);
-            prefetch_row(v + row * V, V * (int)sizeof(Tok), lane);
-            prefetch_row(w + row * V, V * (int)sizeof(Tok), lane);
-            prefetch_row(dO + row * V, V * (int)sizeof(Tok), lane);
-            prefetch_row(delta + row * V, V * 4, lane);
-        }
-        if (chunk_end(t, T)) {   // G here is dL/dS_t from the steps after t
-            const int ci = t / C;
-            const float *ck = ckpt + ((size_t)chain * NC + ci) * K * V;
-            float y[KR];
+    Mat<KR> G;
+    load_mat<KR, K, V>(G, dST ? dST + (size_t)chain * K * V : nullptr, r0, c0);
+    stage(0);
+    cp_commit();
+    stage(1);
+    cp_commit();
+    cp_wait_prev();
+    __syncthreads();
+    for (int r = 0; r < nblk; ++r) {
+        const int lo = lo_of(r), hi = T - 1 - r * NB;
+        unsigned char *sb = stg + (r & 1) * L::bytes;
+        for (int t = hi; t >= lo; --t) {
+            const int s = t - lo;
+            if (chunk_end(t, T)) {   // G here is dL/dS_t from the steps after t
+                const int ci = t / C;
+                const float *ck = ckpt + ((size_t)chain * NC + ci) * K * V;
+                float y[KR];
+#pragma unroll
+                for (int i = 0; i < KR; ++i) {
+                    float2 sv[4];
+                    cols_global(ck + (size_t)(r0 + i) * V + c0, sv);
+                    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) acc = __ffma2_rn(G[i][p], sv[p], acc);
+                    y[i] = acc.x + acc.y;
+                }
+                st_red<KR>(rbnd, 0, NW, K, warp, r0, y);
+                __syncthreads();
+                for (int c = tid; c < K; c += NT) bnd[((size_t)chain * NC + ci) * K + c] = red_sum<K, NW>(rbnd, 0, c);
+                __syncthreads();
+            }
+            float al[KR], kk[KR], bk[KR], qq[KR];
+            rows_of<KR>(at<float>(sb, L::al) + s * K + r0, al);
+            rows_of<KR>(at<Tok>(sb, L::kk) + s * K + r0, kk);
+            rows_of<KR>(at<Tok>(sb, L::bk) + s * K + r0, bk);
+            rows_of<KR>(at<Tok>(sb, L::qq) + s * K + r0, qq);
+            float2 g[4], dl[4];
+            cols_of(at<Tok>(sb, L::go) + s * V + c0, g);
+            cols_of(at<float>(sb, L::dl) + s * V + c0, dl);
+            // o_t = S_t^T q_t: G_t += q_t dO_t^T; ddelta = G_t^T k_t (column sums)
+            float2 pr[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
             for (int i = 0; i < KR; ++i) {
-                float s[8];
-                ld_ws8(ck + (size_t)(r0 + i) * V + c0, s);
-                y[i] = 0.f;
+                const float2 q2 = splat(qq[i]), k2 = splat(kk[i]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) y[i] = fmaf(G[i][j], s[j], y[i]);
+                for (int p = 0; p < 4; ++p) {
+                    G[i][p] = __ffma2_rn(q2, g[p], G[i][p]);
+                    pr[p] = __ffma2_rn(G[i][p], k2, pr[p]);
+                }
             }
-            st_red<KR>(rbnd, 0, NW, K, warp, r0, y);
-            __syncthreads();
-            for (int c = tid; c < K; c += NT) bnd[((size_t)chain * NC + ci) * K + c] = red_sum<K, NW>(rbnd, 0, c);
-            __syncthreads();
-        }
-        // o_t = S_t^T q_t: G_t += q_t dO_t^T; ddelta = G_t^T k_t (column sums)
-        float pr[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            pr[j] = 0.f;
+            const float ddm = warp_colsum8(pr, lane);
+            if ((lane & 3) == 0) {
+                const size_t e = (((size_t)bb * T + t) * H + h) * V + c0 + jm;
+                ddelta[e] = ddm;
+                dv[e] = ddm * to_f32(at<Tok>(sb, L::ww)[s * V + c0 + jm]);
+                dw[e] = ddm * to_f32(at<Tok>(sb, L::vv)[s * V + c0 + jm]);
+            }
+            float2 dd[4];
+            broadcast8(ddm, dd);
+            // row sums of G_t delta_t; G_{t-1} = Diag(alpha_t)(G_t - e_t ddelta_t^T)
+            float x[KR];
 #pragma unroll
             for (int i = 0; i < KR; ++i) {
-                G[i][j] = fmaf(cur.qq[i], cur.g[j], G[i][j]);
-                pr[j] = fmaf(G[i][j], cur.kk[i], pr[j]);
-            }
-        }
-        const float ddm = warp_colsum8(pr, lane);
-        const size_t rowt = ((size_t)bb * T + t) * H + h;
-        if ((lane & 3) == 0) {
-            ddelta[rowt * V + c0 + jm] = ddm;
-            dv[rowt * V + c0 + jm] = ddm * cur.wm;
-            dw[rowt * V + c0 + jm] = ddm * cur.vm;
-        }
-        float dd[8];
+                const float2 a2 = splat(al[i]), ne2 = splat(-bk[i] * kk[i]);
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dd[j] = __shfl_sync(0xffffffffu, ddm, 4 * j);
-        // row sums of G_t delta_t; G_{t-1} = Diag(alpha_t)(G_t - e_t ddelta_t^T)
-        float x[KR];
-#pragma unroll
-        for (int i = 0; i < KR; ++i) {
-            x[i] = 0.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                x[i] = fmaf(G[i][j], cur.dl[j], x[i]);
-                G[i][j] = cur.al[i] * fmaf(-cur.e[i], dd[j], G[i][j]);
+                for (int p = 0; p < 4; ++p) {
+                    acc = __ffma2_rn(G[i][p], dl[p], acc);
+                    G[i][p] = __fmul2_rn(a2, __ffma2_rn(ne2, dd[p], G[i][p]));
+                }
+                x[i] = acc.x + acc.y;
             }
+            st_red<KR>(red, hi - t, NW, K, warp, r0, x);
         }
-        const int slot = (T - 1 - t) % NB;
-        st_red<KR>(red, slot, NW, K, warp, r0, x);
-        if (slot == NB - 1 || t == 0) {
-            __syncthreads();
-            const int tf = t + slot;   // step of slot 0 (the latest of the group)
-            for (int idx = tid; idx < (slot + 1) * K; idx += NT) {
-                const int s = idx / K, c = idx % K;
-                dk[(((size_t)bb * T + tf - s) * H + h) * K + c] = red_sum<K, NW>(red, s, c);
-            }
-            __syncthreads();
+        __syncthreads();
+        for (int idx = tid; idx < (hi - lo + 1) * K; idx += NT) {
+            const int s = idx / K, c = idx - s * K;   // slot s holds step hi - s
+            dk[(((size_t)bb * T + hi - s) * H + h) * K + c] = red_sum<K, NW>(red, s, c);
         }
-        cur = nxt;
+        stage(r + 2);
+        cp_commit();
+        cp_wait_prev();
+        __syncthreads();
     }
     if (dS0) {
 #pragma unroll
-        for (int i = 0; i < KR; ++i) {
-            float4 *p = reinterpret_cast<float4 *>(dS0 + ((size_t)chain * K + r0 + i) * V + c0);
-            p[0] = make_float4(G[i][0], G[i][1], G[i][2], G[i][3]);
-            p[1] = make_float4(G[i][4], G[i][5], G[i][6], G[i][7]);
-        }
+        for (int i = 0; i < KR; ++i) store_cols(dS0 + ((size_t)chain * K + r0 + i) * V + c0, G[i]);
     }
 }
 
@@ -369,92 +429,114 @@ pass_gates(const Tok *__restrict__ q, const Tok *__restrict__ k, const float *__
            const float *__restrict__ ddelta, const float *__restrict__ bnd, const float *__restrict__ dq,
            float *__restrict__ dk, float *__restrict__ db, float *__restrict__ dalpha, int H, int T, int NC) {
     constexpr int K = 32 * KR, V = 8 * NW, NT = NW * 32;
-    extern __shared__ float red[];   // [NB][NW][K], then the chunk's dL/dg rows [C][K]
-    float *hbuf = red + NB * NW * K;
+    using L = Stage3<K, V, Tok>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    float *red = reinterpret_cast<float *>(smem);           // [NB][NW][K]
+    float *hbuf = red + NB * NW * K;                         // [C][K] dL/dg of the chunk's steps
+    float *abuf = hbuf + C * K;                              // [C][K] alpha of the chunk's steps
+    unsigned char *stg = reinterpret_cast<unsigned char *>(abuf + C * K);   // [2][L::bytes]
     const int chain = blockIdx.x, bb = chain / H, h = chain % H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r0 = KR * lane, c0 = 8 * warp;
+    const int nblk = (T + NB - 1) / NB;
 
-    float S[KR][8];
-#pragma unroll
-    for (int i = 0; i < KR; ++i) {
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (S0) ld_cols8(S0 + ((size_t)chain * K + r0 + i) * V + c0, x);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) S[i][j] = x[j];
-    }
-    struct In { float al[KR], kk[KR], dl[8], dd[8]; };
-    auto load = [&](In &in, int t) {
-        const size_t row = ((size_t)bb * T + t) * H + h;
-        ld_rows<KR>(alpha + row * K + r0, in.al);
-        ld_rows<KR>(k + row * K + r0, in.kk);
-        ld_ws8(delta + row * V + c0, in.dl);
-        ld_ws8(ddelta + row * V + c0, in.dd);
+    auto stage = [&](int blk) {
+        const int t0 = blk * NB, n = min(NB, T - t0);
+        if (n <= 0) return;
+        unsigned char *sb = stg + (blk & 1) * L::bytes;
+        const size_t row0 = ((size_t)bb * T + t0) * H + h;
+        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT);
+        stage_rows<K>(at<Tok>(sb, L::qq), q, row0, H, n, tid, NT);
+        stage_rows<K>(at<float>(sb, L::dq), dq, row0, H, n, tid, NT);
+        stage_rows<K>(at<float>(sb, L::dk), static_cast<const float *>(dk), row0, H, n, tid, NT);
+        stage_rows<V>(at<float>(sb, L::dl), delta, row0, H, n, tid, NT);
+        stage_rows<V>(at<float>(sb, L::dd), ddelta, row0, H, n, tid, NT);
     };
-    In cur, nxt;
-    if (T > 0) load(cur, 0);
-    for (int t = 0; t < T; ++t) {
-        if (t + 1 < T) load(nxt, t + 1);
-        if (warp == 0 && t + PF < T) {
-            const size_t row = ((size_t)bb * T + t + PF) * H + h;
-            prefetch_row(alpha + row * K, K * 4, lane);
-            prefetch_row(k + row * K, K * (int)sizeof(Tok), lane);
-            prefetch_row(delta + row * V, V * 4, lane);
-            prefetch_row(ddelta + row * V, V * 4, lane);
-        }
-        float x[KR];
+    Mat<KR> S;
+    load_mat<KR, K, V>(S, S0 ? S0 + (size_t)chain * K * V : nullptr, r0, c0);
+    stage(0);
+    cp_commit();
+    stage(1);
+    cp_commit();
+    cp_wait_prev();
+    __syncthreads();
+    for (int blk = 0; blk < nblk; ++blk) {
+        const int t0 = blk * NB, n = min(NB, T - t0);
+        unsigned char *sb = stg + (blk & 1) * L::bytes;
+        for (int s = 0; s < n; ++s) {
+            float al[KR], kk[KR];
+            rows_of<KR>(at<float>(sb, L::al) + s * K + r0, al);
+            rows_of<KR>(at<Tok>(sb, L::kk) + s * K + r0, kk);
+            float2 dl[4], dd[4];
+            cols_of(at<float>(sb, L::dl) + s * V + c0, dl);
+            cols_of(at<float>(sb, L::dd) + s * V + c0, dd);
+            float x[KR];
 #pragma unroll
-        for (int i = 0; i < KR; ++i) {
-            x[i] = 0.f;
+            for (int i = 0; i < KR; ++i) {
+                const float2 a2 = splat(al[i]), k2 = splat(kk[i]);
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                x[i] = fmaf(S[i][j], cur.dd[j], x[i]);                        // S_{t-1} ddelta_t
-                S[i][j] = fmaf(cur.kk[i], cur.dl[j], cur.al[i] * S[i][j]);   // S_t
-            }
-        }
-        const int slot = t % NB;
-        st_red<KR>(red, slot, NW, K, warp, r0, x);
-        if (slot == NB - 1 || t == T - 1) {
-            __syncthreads();
-            const int t0 = t - slot;
-            for (int idx = tid; idx < (slot + 1) * K; idx += NT) {
-                const int s = idx / K, c = idx % K;
-                const size_t e = (((size_t)bb * T + t0 + s) * H + h) * K + c;
-                const float a = alpha[e], kc = to_f32(k[e]), bc = to_f32(b[e]), qc = to_f32(q[e]);
-                const float de = -a * red_sum<K, NW>(red, s, c);
-                const float dkt = dk[e] + bc * de;
-                dk[e] = dkt;
-                db[e] = kc * de;
-                // dL/dg_t = q dq + e de - k (dk - b de)
-                hbuf[((t0 + s) % C) * K + c] = qc * dq[e] + 2.f * bc * kc * de - kc * dkt;
-            }
-            __syncthreads();
-            if (chunk_end(t, T)) {
-                const int ci = t / C, cs = ci * C;
-                for (int c = tid; c < K; c += NT) {
-                    float acc = bnd[((size_t)chain * NC + ci) * K + c];
-                    for (int s = t - cs; s >= 0; --s) {
-                        acc += hbuf[s * K + c];
-                        const size_t e = (((size_t)bb * T + cs + s) * H + h) * K + c;
-                        dalpha[e] = acc / fmaxf(alpha[e], FLT_MIN);
-                    }
+                for (int p = 0; p < 4; ++p) {
+                    acc = __ffma2_rn(S[i][p], dd[p], acc);                       // S_{t-1} ddelta_t
+                    S[i][p] = __ffma2_rn(k2, dl[p], __fmul2_rn(a2, S[i][p]));   // S_t
                 }
-                __syncthreads();
+                x[i] = acc.x + acc.y;
+            }
+            st_red<KR>(red, s, NW, K, warp, r0, x);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < n * K; idx += NT) {
+            const int s = idx / K, c = idx - s * K;
+            const size_t e = (((size_t)bb * T + t0 + s) * H + h) * K + c;
+            const float a = at<float>(sb, L::al)[s * K + c];
+            const float kc = to_f32(at<Tok>(sb, L::kk)[s * K + c]), bc = to_f32(at<Tok>(sb, L::bk)[s * K + c]);
+            const float qc = to_f32(at<Tok>(sb, L::qq)[s * K + c]);
+            const float de = -a * red_sum<K, NW>(red, s, c);
+            const float dkt = at<float>(sb, L::dk)[s * K + c] + bc * de;
+            dk[e] = dkt;
+            db[e] = kc * de;
+            // dL/dg_t = q dq + e de - k (dk - b de)
+            const int pos = (t0 + s) % C;
+            hbuf[pos * K + c] = qc * at<float>(sb, L::dq)[s * K + c] + 2.f * bc * kc * de - kc * dkt;
+            abuf[pos * K + c] = a;
+        }
+        __syncthreads();   // the staged rows of this block were read above: the buffer is free
+        stage(blk + 2);
+        cp_commit();
+        cp_wait_prev();
+        __syncthreads();
+        const int t = t0 + n - 1;
+        if (chunk_end(t, T)) {   // d log alpha summed back from the chunk end; its buffers are
+            const int ci = t / C, cs = ci * C;   // next written after the next block's first barrier
+            for (int c = tid; c < K; c += NT) {
+                float acc = bnd[((size_t)chain * NC + ci) * K + c];
+                for (int s = t - cs; s >= 0; --s) {
+                    acc += hbuf[s * K + c];
+                    dalpha[(((size_t)bb * T + cs + s) * H + h) * K + c] = acc / fmaxf(abuf[s * K + c], FLT_MIN);
+                }
             }
         }
-        cur = nxt;
     }
 }
+
+template <int K, int V, typename Tok>
+constexpr size_t smem1() { return (size_t)NB * (V / 8) * K * 4 + 2 * Stage1<K, V, Tok>::bytes; }
+template <int K, int V, typename Tok>
+constexpr size_t smem2() { return (size_t)(NB + 1) * (V / 8) * K * 4 + 2 * Stage2<K, V, Tok>::bytes; }
+template <int K, int V, typename Tok>
+constexpr size_t smem3() { return (size_t)NB * (V / 8) * K * 4 + 2 * (size_t)C * K * 4 + 2 * Stage3<K, V, Tok>::bytes; }
 
 template <int KR, int NW, typename Tok>
 int launch_all(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
                const float *S0, const void *dO, const float *dST, float *dq, float *dk, float *dv, float *dalpha,
                float *db, float *dw, float *dS0, int B, int H, int T, float *delta, float *ddelta, float *ckpt,
                float *bnd, cudaStream_t st) {
-    constexpr int K = 32 * KR;
+    constexpr int K = 32 * KR, V = 8 * NW;
+    constexpr size_t sm1 = smem1<K, V, Tok>(), sm2 = smem2<K, V, Tok>(), sm3 = smem3<K, V, Tok>();
+    static_assert(sm1 <= 227 * 1024 && sm2 <= 227 * 1024 && sm3 <= 227 * 1024, "shared memory");
     const int NC = (T + C - 1) / C, NT = NW * 32, grid = B * H;
-    const size_t red_bytes = sizeof(float) * NB * NW * K;
-    const size_t sm1 = red_bytes, sm2 = red_bytes + sizeof(float) * NW * K, sm3 = red_bytes + sizeof(float) * C * K;
     auto f1 = pass_forward<KR, NW, Tok>;
     auto f2 = pass_reverse<KR, NW, Tok>;
     auto f3 = pass_gates<KR, NW, Tok>;
@@ -474,6 +556,7 @@ int launch_all(const void *q, const void *k, const void *v, const float *alpha, 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace bwd
+
 
 size_t bwd_workspace_bytes(int B, int H, int T, int K, int V) {
     const size_t ntok = (size_t)B * T * H, NC = (size_t)(T + bwd::C - 1) / bwd::C;
