@@ -53,6 +53,18 @@ def prefill_flops(B, T, H, K, V, C=64):
     return n_chunks * per_chunk
 
 
+def backward_flops(B, T, H, K, V):
+    """fp32 arithmetic of the backward's three passes on the d_k x d_v carried matrix, per
+    token-head and state element: pass 1 (decay 1, erase read 2, write 2, S dO 2), pass 2
+    (q dO^T 2, G^T k 2, G delta 2, erase 2, decay 1), pass 3 (S ddelta 2, write 2, decay 1): 21."""
+    return 21 * B * T * H * K * V
+
+
+def fp32_alu_peak_tflops(n_sm, sm_mhz):
+    """Dense fp32 FMA peak from unit counts and clock: 128 fp32 lanes per SM, 2 flops per FMA."""
+    return n_sm * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def decode_bytes(B, H, K, V, tok_bytes=2):
     state = 4 * B * H * K * V
     return 2 * state + B * H * ((3 * K + 2 * V) * tok_bytes + 4 * K + V * tok_bytes)
@@ -438,6 +450,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
     e2e_value = tokens_all / (e2e_ms * 1e-3)
 
+    extras = None if (args.no_extras or world > 1) else run_next_rows(g, torch, dev, stream, pw, pre_ms, clocks)
+
     launches_per_step = (1 if path == 1 else 2) + 1
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -454,6 +468,8 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
+    if extras is not None:
+        out["next_rows"] = extras
     if parts != {"prefill", "decode"}:
         out["config"]["parts_only"] = sorted(parts)   # profiling run: not a bench line
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -467,6 +483,67 @@ def run_ours(args):
     return 0
 
 
+def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks):
+    """Timings of the rows beyond the step (not part of `value`): the backward pass of the
+    prefill workload and the prefill with the layer edges fused, both on that workload's sizes."""
+    import synth
+
+    def timed(fn, warm=2, reps=5):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    x = synth.make_inputs(wl)
+    B, T, H, K, V = wl.B, wl.T, wl.H, wl.K, wl.V
+    to = lambda a, dt: torch.from_numpy(a).to(dev).to(dt)
+    X = {k: to(a, torch.float32 if k == "alpha" else torch.bfloat16) for k, a in x.items()}
+    dO_np, dST_np = synth.make_output_grads(wl)
+    dO, dST = to(dO_np, torch.bfloat16), to(dST_np, torch.float32)
+    del x, dO_np, dST_np
+    grads = {n: torch.empty((B, T, H, K if n in ("dq", "dk", "dalpha", "db") else V), device=dev)
+             for n in ("dq", "dk", "dv", "dalpha", "db", "dw")}
+    dS0 = torch.empty((B, H, K, V), device=dev)
+    wsb = g.new_workspace(g.gdn2_chunk_bwd_workspace_bytes(B, H, T, K, V), dev)
+    bwd_ms = timed(lambda: g.gdn2_chunk_bwd(X["q"], X["k"], X["v"], X["alpha"], X["b"], X["w"], None, dO, dST,
+                                            grads["dq"], grads["dk"], grads["dv"], grads["dalpha"], grads["db"],
+                                            grads["dw"], dS0, workspace=wsb, stream=stream))
+    del grads, dS0, wsb, X, dO, dST
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    sm_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    peak = fp32_alu_peak_tflops(n_sm, sm_mhz)
+    flops = backward_flops(B, T, H, K, V)
+    achieved = flops / (bwd_ms * 1e-3) / 1e12
+    backward = {"ms": bwd_ms, "tokens_per_s": B * T / (bwd_ms * 1e-3), "launches": 3,
+                "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                             "frac": achieved / peak, "flops_per_launch": flops, "traffic": None,
+                             "peak_src": f"derived: {n_sm} SMs x 128 fp32 lanes x 2 flops x {sm_mhz:.0f} MHz"}}
+
+    r = synth.make_raw_inputs(wl)
+    R = {k: to(a, torch.float32 if k == "a" else torch.bfloat16) for k, a in r.items()}
+    del r
+    o = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((B, H, K, V), device=dev)
+    weight = torch.ones(V, device=dev)
+    ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_BF16), dev)
+    edge_ms = timed(lambda: g.gdn2_chunk_fwd_edges(R["q"], R["k"], R["v"], R["a"], R["b"], R["w"], None, weight, o,
+                                                   S_T, workspace=ws, stream=stream))
+    if g.gdn2_workspace_status(ws) != 0:
+        raise SystemExit("edge prefill kernel reported an internal error")
+    edges = {"ms": edge_ms, "tokens_per_s": B * T / (edge_ms * 1e-3), "launches": 1, "rmsnorm": True,
+             "plain_prefill_ms": plain_prefill_ms,
+             "inputs": "raw q, k ~ N(0, 9), decay logit ~ N(1, 1) (alpha = exp(-softplus(a)): the plain "
+                       "workload's alpha distribution), gate logits ~ N(0, 1)"}
+    return {"workload": f"{wl.name} (B{B} H{H} T{T} d_k=d_v={K}, bf16 tokens)", "backward": backward,
+            "edges_prefill": edges}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -474,6 +551,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-extras", action="store_true", help="skip the backward / fused-edge timings")
     ap.add_argument("--parts", default="prefill,decode",
                     help="profiling aid: run only some parts of the step (the default runs the whole step)")
     args = ap.parse_args(argv)

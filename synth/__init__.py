@@ -247,6 +247,44 @@ def make_state(wl: Workload, chains=None):
     return x.reshape(len(chains), K, V)
 
 
+RAW_QK_SCALE = 3.0   # raw (unnormalised) q, k rows of the layer-edge workloads: N(0, 3^2)
+
+
+def make_raw_inputs(wl: Workload, chains=None):
+    """The layer's raw inputs for the fused-edge prefill, same shapes as make_inputs: q, k ~ N(0, 9)
+    (not normalised), v ~ N(0, 1), the decay logit a ~ N(alpha_mu, 1) in fp32 (the recurrence's
+    alpha is exp(-softplus(a)), so its distribution matches make_inputs' alpha), the gate logits
+    b, w ~ N(0, 1).  Streams 10..15 of the workload's seed."""
+    T_full = wl.T
+    idx = _row_index(wl, T_full, chains, 0, T_full)
+    nrows = wl.B * T_full * wl.H if idx is None else idx.size
+    bf = wl.dtype == "bf16"
+
+    def tok(st, d, mu=0.0, scale=1.0, bf16=bf):
+        return rows(wl.seed, st, KIND_NORMAL, d, row_index=idx, nrows=nrows, mu=mu, scale=scale, bf16=bf16)
+
+    out = {"q": tok(10, wl.K, scale=RAW_QK_SCALE), "k": tok(11, wl.K, scale=RAW_QK_SCALE), "v": tok(12, wl.V),
+           "a": tok(13, wl.K, mu=wl.alpha_mu, bf16=False), "b": tok(14, wl.K), "w": tok(15, wl.V)}
+    shape = (wl.B, T_full, wl.H) if chains is None else (len(chains), T_full)
+    return {key: a.reshape(*shape, a.shape[-1]) for key, a in out.items()}
+
+
+def make_output_grads(wl: Workload, chains=None, dst_std: float = 0.05):
+    """Gradients at the recurrence's outputs for the backward workloads: dO ~ N(0, 1) in the token
+    dtype ([B,T,H,V] or [n,T,V]) and dS_T ~ N(0, dst_std^2) fp32 ([B,H,K,V] or [n,K,V]).
+    Streams 9 (dO) and 10 + 256 (dS_T) of the workload's seed."""
+    T_full = wl.T
+    idx = _row_index(wl, T_full, chains, 0, T_full)
+    nrows = wl.B * T_full * wl.H if idx is None else idx.size
+    dO = rows(wl.seed, 9, KIND_NORMAL, wl.V, row_index=idx, nrows=nrows, bf16=wl.dtype == "bf16")
+    if chains is None:
+        dST = rows(wl.seed, 266, KIND_NORMAL, wl.K * wl.V, nrows=wl.B * wl.H, scale=dst_std)
+        return dO.reshape(wl.B, T_full, wl.H, wl.V), dST.reshape(wl.B, wl.H, wl.K, wl.V)
+    sidx = np.array([b * wl.H + h for (b, h) in chains], dtype=np.uint64)
+    dST = rows(wl.seed, 266, KIND_NORMAL, wl.K * wl.V, row_index=sidx, scale=dst_std)
+    return dO.reshape(len(chains), T_full, wl.V), dST.reshape(len(chains), wl.K, wl.V)
+
+
 def as_f64(d: dict) -> dict:
     """fp64 copies (for the oracle) of a dict of float32 input arrays."""
     return {k: (None if v is None else np.asarray(v, dtype=np.float64)) for k, v in d.items()}

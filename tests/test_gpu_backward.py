@@ -23,23 +23,10 @@ pytestmark = pytest.mark.gpu
 
 TOL = 1e-4
 GRADS = ("dq", "dk", "dv", "dalpha", "db", "dw")
-ST_DO, ST_DST = 9, 10   # synth streams of the output gradients
 
 
-def output_grads(wl, chains=None, dst_std=0.05):
-    """dO ~ N(0,1) in the token dtype ([B,T,H,V], or [n,T,V] for chains), dS_T ~ N(0, dst_std^2)."""
-    bf = wl.dtype == "bf16"
-    if chains is None:
-        dO = synth.rows(wl.seed, ST_DO, synth.KIND_NORMAL, wl.V, nrows=wl.B * wl.T * wl.H, bf16=bf)
-        dO = dO.reshape(wl.B, wl.T, wl.H, wl.V)
-        dST = synth.rows(wl.seed, ST_DST, synth.KIND_NORMAL, wl.K * wl.V, nrows=wl.B * wl.H, scale=dst_std)
-        return dO, dST.reshape(wl.B, wl.H, wl.K, wl.V)
-    t = np.arange(wl.T, dtype=np.uint64)
-    idx = np.concatenate([(np.uint64(b) * np.uint64(wl.T) + t) * np.uint64(wl.H) + np.uint64(h) for b, h in chains])
-    dO = synth.rows(wl.seed, ST_DO, synth.KIND_NORMAL, wl.V, row_index=idx, bf16=bf).reshape(len(chains), wl.T, wl.V)
-    sidx = np.array([b * wl.H + h for b, h in chains], dtype=np.uint64)
-    dST = synth.rows(wl.seed, ST_DST, synth.KIND_NORMAL, wl.K * wl.V, row_index=sidx, scale=dst_std)
-    return dO, dST.reshape(len(chains), wl.K, wl.V)
+def output_grads(wl, chains=None):
+    return synth.make_output_grads(wl, chains)
 
 
 def run_bwd(torch, g, xd, S0, dO, dST, want_dS0=True):

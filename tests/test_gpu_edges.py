@@ -10,24 +10,11 @@ from tests.gpu_util import TOL, assert_close, cuda_or_skip, f64
 pytestmark = pytest.mark.gpu
 
 
-def raw_inputs(B, T, H, seed, chains=None, t_range=None):
-    """Seeded raw layer inputs ([B,T,H,d], or [n,T,d] for a list of (b, h) chains): unnormalised
-    q, k (scale 3), v ~ N(0,1), decay logits ~ N(1,1) (fp32), gate logits ~ N(0,1)."""
-    K = V = 128
-    t0, t1 = (0, T) if t_range is None else t_range
-    if chains is None:
-        idx = None
-        n = B * (t1 - t0) * H
-    else:
-        t = np.arange(t0, t1, dtype=np.uint64)
-        idx = np.concatenate([(np.uint64(b) * np.uint64(T) + t) * np.uint64(H) + np.uint64(h) for b, h in chains])
-        n = idx.size
-    r = lambda st, d, mu=0.0, scale=1.0, bf16=True: synth.rows(seed, st, synth.KIND_NORMAL, d, row_index=idx,
-                                                               nrows=n, mu=mu, scale=scale, bf16=bf16)
-    x = {"q": r(0, K, scale=3.0), "k": r(1, K, scale=3.0), "v": r(2, V), "a": r(3, K, mu=1.0, bf16=False),
-         "b": r(4, K), "w": r(5, V)}
-    shape = (B, t1 - t0, H) if chains is None else (len(chains), t1 - t0)
-    return {key: a.reshape(*shape, a.shape[-1]) for key, a in x.items()}
+def raw_inputs(B, T, H, seed, chains=None):
+    """Seeded raw layer inputs ([B,T,H,d], or [n,T,d] for a list of (b, h) chains), the recipe of
+    synth.make_raw_inputs: unnormalised q, k (scale 3), v ~ N(0,1), decay logits ~ N(1,1) (fp32),
+    gate logits ~ N(0,1)."""
+    return synth.make_raw_inputs(synth.Workload("edges", B, H, T, 128, 128, "bf16", 1.0, seed=seed), chains)
 
 
 def to_dev(torch, x):
