@@ -522,7 +522,8 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks):
     achieved = flops / (bwd_ms * 1e-3) / 1e12
     backward = {"ms": bwd_ms, "tokens_per_s": B * T / (bwd_ms * 1e-3), "launches": 3,
                 "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                             "frac": achieved / peak, "flops_per_launch": flops, "traffic": None,
+                             "frac": achieved / peak, "flops_per_launch": flops,
+                             "traffic": recorded_traffic("backward"),
                              "peak_src": f"derived: {n_sm} SMs x 128 fp32 lanes x 2 flops x {sm_mhz:.0f} MHz"}}
 
     r = synth.make_raw_inputs(wl)
