@@ -532,7 +532,7 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks):
     o = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((B, H, K, V), device=dev)
     weight = torch.ones(V, device=dev)
-    ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_BF16), dev)
+    ws = g.new_workspace(g.gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, K, V), dev)
     edge_ms = timed(lambda: g.gdn2_chunk_fwd_edges(R["q"], R["k"], R["v"], R["a"], R["b"], R["w"], None, weight, o,
                                                    S_T, workspace=ws, stream=stream))
     if g.gdn2_workspace_status(ws) != 0:

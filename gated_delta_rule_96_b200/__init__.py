@@ -19,6 +19,7 @@ __all__ = [
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
+    "gdn2_chunk_fwd_edges_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,6 +66,8 @@ def load_library():
     lib.gdn2_chunk_fwd_noalloc.restype = i
     lib.gdn2_chunk_fwd_edges.argtypes = [vp] * 10 + [i] * 7 + [vp, sz, vp]
     lib.gdn2_chunk_fwd_edges.restype = i
+    lib.gdn2_chunk_fwd_edges_workspace_bytes.argtypes = [i] * 6
+    lib.gdn2_chunk_fwd_edges_workspace_bytes.restype = sz
     lib.gdn2_chunk_bwd_workspace_bytes.argtypes = [i] * 5
     lib.gdn2_chunk_bwd_workspace_bytes.restype = sz
     lib.gdn2_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
@@ -153,6 +156,10 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, C=64, workspace=None, strea
         raise GDN2Error(rc, "gdn2_chunk_fwd")
 
 
+def gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, d_k, d_v, C=64) -> int:
+    return int(load_library().gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, d_k, d_v, C))
+
+
 def gdn2_chunk_fwd_edges(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o_weight, o, S_T, C=64, workspace=None,
                          stream=None) -> None:
     """Prefill with the layer edges fused (include/gdn2.h, gdn2_chunk_fwd_edges): q, k L2-normalised,
@@ -172,7 +179,7 @@ def gdn2_chunk_fwd_edges(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o_weigh
                          ("o_weight", o_weight, (V,))):
         if t is not None and tuple(t.shape) != shp:
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
-    need = gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, C, dt)
+    need = gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, K, V, C)
     if workspace is None:
         workspace = new_workspace(need, q_raw.device)
     rc = load_library().gdn2_chunk_fwd_edges(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_logit), _ptr(b_logit),

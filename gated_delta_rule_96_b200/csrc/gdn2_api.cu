@@ -36,6 +36,11 @@ size_t gdn2_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int
     return gdn2::simt_workspace_bytes(B, H, T, d_k, d_v, C);
 }
 
+size_t gdn2_chunk_fwd_edges_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C) {
+    if (B < 0 || H < 0 || T < 0 || !use_tc(B, H, T, d_k, d_v, C, GDN2_BF16)) return gdn2::kStatusBytes;
+    return gdn2::tc_workspace_bytes(B, H, T, d_k, d_v, C, 1);
+}
+
 int gdn2_chunk_fwd_path(int B, int H, int T, int d_k, int d_v, int C, int dtype) {
     return use_tc(B, H, T, d_k, d_v, C, dtype) ? 1 : 0;
 }
@@ -91,7 +96,7 @@ int gdn2_chunk_fwd_edges(const void *q_raw, const void *k_raw, const void *v, co
     if (!aligned16(S_T) || (S0 && !aligned16(S0)) || (o_weight && !aligned16(o_weight))) return GDN2_ERR_ALIGN;
     if (!workspace) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
-    if (workspace_bytes < gdn2_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, C, dtype)) return GDN2_ERR_WORKSPACE;
+    if (workspace_bytes < gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, d_k, d_v, C)) return GDN2_ERR_WORKSPACE;
     if (B == 0 || H == 0) return GDN2_OK;
     return gdn2::launch_chunk_tc(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o, S_T, B, H, T, d_k, d_v, C,
                                  workspace, reinterpret_cast<cudaStream_t>(stream), 1, o_weight);

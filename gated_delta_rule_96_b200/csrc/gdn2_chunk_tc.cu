@@ -95,6 +95,16 @@ enum : uint32_t {
     MB_G1 = 80, MB_READOUT = 88, MB_S1DONE = 96, MB_D3FREE = 104, MB_END = 112
 };
 constexpr uint32_t MISC_TSLOT = 160, MISC_ABORT = 164;
+// layer-edge ring: RING_SLOTS full / free barrier pairs, slot m % RING_SLOTS for chunk m
+constexpr uint32_t MB_RFULL = 168, MB_RFREE = 200;
+
+// Layer-edge ring (per block, in the workspace): the o warps write the decay rows of chunk m,
+// alpha = exp(-softplus(a)) in fp32, into slot m % RING_SLOTS, RING_SLOTS chunks ahead of the
+// build group, which reads them as it reads plain alpha.  q, k and b stay raw: the build group
+// folds the inverse norms of q and k into its decay factors and applies the sigmoid to b where
+// it uses it.
+constexpr int RING_SLOTS = 4;
+constexpr uint32_t RING_BYTES = C * KD * 4;   // 32 KB
 
 // Launch flags of the segmented (parallel-in-time) prefill.  A block owns segment
 // blockIdx.x % nseg of chain blockIdx.x / nseg; S0 and S_T are indexed by block.
@@ -150,6 +160,13 @@ __device__ __forceinline__ float alpha_of_logit(float a) { return fast_rcp(1.f +
 __device__ __forceinline__ float log2_alpha_of_logit(float a) {
     const float sp = a > 15.f ? a : __logf(1.f + __expf(a));
     return fmaxf(-sp * 1.4426950408889634f, -126.f);
+}
+// load of data that other warps of the block wrote earlier in this kernel (the layer-edge
+// ring): a plain global load, not the read-only path
+__device__ __forceinline__ float4 ld_f4(const float *p) {
+    float4 v;
+    asm volatile("ld.global.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p) : "memory");
+    return v;
 }
 __device__ __forceinline__ uint32_t bsigmoid2(uint32_t a) {
     const float2 f = unpack2(a);
@@ -249,6 +266,7 @@ struct Ctx {
     int T, H, bb, h, NC;
     int tb, te;        // token range of this block's segment: [tb, te)
     const float *onorm;   // RMSNorm weight of o (layer-edge variant; null: none)
+    unsigned char *ring;  // this block's layer-edge ring (layer-edge variant)
     uint32_t flags;    // SEG_* below
 };
 
@@ -339,55 +357,63 @@ __device__ __forceinline__ void issue_g45(const Ctx &c, int n) {
 }
 
 // ============================================================================ build group
+// Rows of one chunk's q, k, b (bf16) and alpha (fp32): row t of the chunk is at element
+// (base + t * stride) * KD.  Plain inputs: the token tensors; layer-edge variant: the ring slot.
+struct Src {
+    const __nv_bfloat16 *q, *k, *b;
+    const float *a;
+    size_t base, stride;       // rows of q and k
+    size_t base_ba, stride_ba; // rows of b and alpha
+    __device__ __forceinline__ size_t row(int t) const { return base + (size_t)t * stride; }
+    __device__ __forceinline__ size_t row_ba(int t) const { return base_ba + (size_t)t * stride_ba; }
+};
+
 // Wide-span chunk: A_ri = sum_c e_rc k_ic exp2(g_rc - g_ic) for i < r and P_ri likewise with
 // q for i <= r, one row per thread (rows of A on threads 0-63, of P on 64-127: the TMEM lane
 // of D1 that G1 would have written).  For each channel the exponent g_rc - g_ic is summed from
-// log2 alpha while i walks down from r, so it never leaves [-inf, 0]; tokens are re-read from
+// log2 alpha while i walks down from r, so it never leaves [-inf, 0]; rows are re-read from
 // global memory (resident in L2).
 template <bool EDGES>
-__device__ __forceinline__ void wide_span_ap(const Ctx &c, int tid1, int t0, int L) {
+__device__ __forceinline__ void wide_span_ap(const Ctx &c, const Src &src, int tid1, int L) {
     const int r = tid1 & 63;
     const bool isP = tid1 >= 64;
-    const int T = c.T, H = c.H, bb = c.bb, h = c.h;
     const uint32_t lane_base = c.tmem + ((uint32_t)((tid1 >> 5) * 32) << 16) + TM_D1;
-    const size_t rowr = ((size_t)bb * T + t0 + min(r, L - 1)) * H + h;
-    auto rownorm = [&](const __nv_bfloat16 *x, size_t row) {   // 1 / max(|x_row|, eps)
+    const int rc = min(r, L - 1);
+    const size_t rowr = src.row(rc), rowr_ba = src.row_ba(rc);
+    auto log2a = [&](int t, int cc) { return fast_log2(fmaxf(src.a[src.row_ba(t) * KD + cc], 1.17549435e-38f)); };
+    auto inv_norm = [&](const __nv_bfloat16 *x, size_t row) {   // layer edges: 1 / max(|x_row|, eps)
         float ss = 0.f;
         for (int cc = 0; cc < KD; ++cc) {
             const float v = __bfloat162float(x[row * KD + cc]);
             ss += v * v;
         }
-        return 1.f / fmaxf(sqrtf(ss), EDGE_NORM_EPS);
+        return rsqrtf(fmaxf(ss, EDGE_NORM_EPS * EDGE_NORM_EPS));
     };
-    auto log2a = [&](size_t row, int cc) {
-        const float a = c.alpha[row * KD + cc];
-        return EDGES ? log2_alpha_of_logit(a) : fast_log2(fmaxf(a, 1.17549435e-38f));
-    };
-    const float sr = EDGES ? (isP ? rownorm(c.q, rowr) : rownorm(c.k, rowr)) : 1.f;
+    const float sr = EDGES ? inv_norm(isP ? src.q : src.k, rowr) : 1.f;
 #pragma unroll 1
     for (int i0 = 0; i0 < 64; i0 += 16) {
         float acc[16], sk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             acc[i] = 0.f;
-            sk[i] = EDGES ? rownorm(c.k, ((size_t)bb * T + t0 + min(i0 + i, L - 1)) * H + h) : 1.f;
+            sk[i] = EDGES ? inv_norm(src.k, src.row(min(i0 + i, L - 1))) : 1.f;
         }
         if (r < L && i0 <= r) {
 #pragma unroll 1
             for (int cc = 0; cc < KD; ++cc) {
-                const float bg = EDGES ? sigmoid_f(__bfloat162float(c.b[rowr * KD + cc])) : __bfloat162float(c.b[rowr * KD + cc]);
-                const float x = sr * (isP ? __bfloat162float(c.q[rowr * KD + cc]) : bg * __bfloat162float(c.k[rowr * KD + cc]));
+                const float bg = EDGES ? sigmoid_f(__bfloat162float(src.b[rowr * KD + cc]))
+                                       : __bfloat162float(src.b[rowr * KD + cc]);
+                const float x = sr * (isP ? __bfloat162float(src.q[rowr * KD + cc]) : bg * __bfloat162float(src.k[rowr * KD + cc]));
                 // exponent at i = i0 + 15 (or r): log2 of alpha over positions i+1 .. r
                 const int itop = min(i0 + 15, r);
                 float d = 0.f;
 #pragma unroll 1
-                for (int j = r; j > itop; --j) d += log2a(((size_t)bb * T + t0 + j) * H + h, cc);
+                for (int jj = r; jj > itop; --jj) d += log2a(jj, cc);
 #pragma unroll
                 for (int i = 15; i >= 0; --i) {
                     if (i0 + i <= itop) {
-                        const size_t rowi = ((size_t)bb * T + t0 + i0 + i) * H + h;
-                        acc[i] += x * sk[i] * __bfloat162float(c.k[rowi * KD + cc]) * exp2f(d);
-                        d += log2a(rowi, cc);
+                        acc[i] += x * sk[i] * __bfloat162float(src.k[src.row(i0 + i) * KD + cc]) * exp2f(d);
+                        d += log2a(i0 + i, cc);
                     }
                 }
             }
@@ -422,21 +448,46 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
         unsigned char *EQ = sm + SM_EQ + (n & 1) * EQ_BYTES;
         unsigned char *KT = sm + SM_KT + (n & 1) * KT_BYTES;
         // ---------------------------------------------------------------- loads and log-decay prefix
+        // Layer-edge variant: b and alpha come mapped from the ring slot the o warps filled; q and k
+        // are raw, their inverse norms folded into the decay factors below.
+        const size_t row0 = ((size_t)bb * T + t0) * H + h;
+        Src src{c.q, c.k, c.b, c.alpha, row0, (size_t)H, row0, (size_t)H};
+        if (EDGES) {
+            src.a = reinterpret_cast<const float *>(c.ring + (n % RING_SLOTS) * RING_BYTES);
+            src.base_ba = 0;
+            src.stride_ba = 1;
+        }
         float al[16][4];   // alpha (1 past the end of the sequence)
         uint2 rq[16], rk[16], rb[16];
+        if (!EDGES) {
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-            const int t = min(p0 + p, L - 1);
-            const size_t row = ((size_t)bb * T + t0 + t) * H + h;
-            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(c.alpha + row * KD + c4));
-            al[p][0] = a4.x; al[p][1] = a4.y; al[p][2] = a4.z; al[p][3] = a4.w;
-            rq[p] = __ldg(reinterpret_cast<const uint2 *>(c.q + row * KD + c4));
-            rk[p] = __ldg(reinterpret_cast<const uint2 *>(c.k + row * KD + c4));
-            rb[p] = __ldg(reinterpret_cast<const uint2 *>(c.b + row * KD + c4));
+            for (int p = 0; p < 16; ++p) {
+                const size_t row = src.row(min(p0 + p, L - 1));
+                const float4 a4 = __ldg(reinterpret_cast<const float4 *>(src.a + row * KD + c4));
+                al[p][0] = a4.x; al[p][1] = a4.y; al[p][2] = a4.z; al[p][3] = a4.w;
+                rq[p] = __ldg(reinterpret_cast<const uint2 *>(src.q + row * KD + c4));
+                rk[p] = __ldg(reinterpret_cast<const uint2 *>(src.k + row * KD + c4));
+                rb[p] = __ldg(reinterpret_cast<const uint2 *>(src.b + row * KD + c4));
+            }
+        } else {   // raw q, k, b first; the decay rows once the producer has filled the ring slot
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                const size_t row = src.row(min(p0 + p, L - 1));
+                rq[p] = __ldg(reinterpret_cast<const uint2 *>(src.q + row * KD + c4));
+                rk[p] = __ldg(reinterpret_cast<const uint2 *>(src.k + row * KD + c4));
+                rb[p] = __ldg(reinterpret_cast<const uint2 *>(src.b + row * KD + c4));
+            }
+            if (!group_wait(c, mbar(c, MB_RFULL + 8 * (n % RING_SLOTS)), (uint32_t)((n / RING_SLOTS) & 1), BAR_BUILD,
+                            GROUP))
+                return;
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {   // the ring is written in this kernel: coherent loads
+                const float4 a4 = ld_f4(src.a + src.row_ba(min(p0 + p, L - 1)) * KD + c4);
+                al[p][0] = a4.x; al[p][1] = a4.y; al[p][2] = a4.z; al[p][3] = a4.w;
+            }
         }
-        // layer edges: alpha = exp(-softplus(alpha logit)) here; q and k are divided by their norms
-        // over the 128 channels (4 per lane: a warp holds a row) and b = sigmoid(b logit) where they
-        // are used.  Lane l keeps the inverse norms of the warp's position l / 2.
+        // layer edges: q and k are divided by their norms over the 128 channels (4 per lane: a warp
+        // holds a row) where they are used; lane l keeps the inverse norms of the warp's position l / 2
         float iq_l = 1.f, ik_l = 1.f;
         if (EDGES) {
 #pragma unroll
@@ -450,8 +501,6 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                     sk += __shfl_xor_sync(0xffffffffu, sk, msk);
                 }
                 if ((lane >> 1) == p) { iq_l = sq; ik_l = sk; }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) al[p][j] = alpha_of_logit(al[p][j]);
             }
             iq_l = rsqrtf(fmaxf(iq_l, EDGE_NORM_EPS * EDGE_NORM_EPS));
             ik_l = rsqrtf(fmaxf(ik_l, EDGE_NORM_EPS * EDGE_NORM_EPS));
@@ -460,11 +509,13 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
             const int r = tid1 & 63, half = tid1 >> 6;
             const int t = min(r, c.te - t0 - C - 1);
             const size_t row = ((size_t)bb * T + t0 + C + t) * H + h;
-            const char *base[3] = {(const char *)(c.q + row * KD), (const char *)(c.k + row * KD), (const char *)(c.b + row * KD)};
-#pragma unroll
-            for (int i = 0; i < 3; ++i) prefetch_l2(base[i] + 128 * half);
-            prefetch_l2((const char *)(c.alpha + row * KD) + 256 * half);
-            prefetch_l2((const char *)(c.alpha + row * KD) + 256 * half + 128);
+            prefetch_l2((const char *)(c.q + row * KD) + 128 * half);
+            prefetch_l2((const char *)(c.k + row * KD) + 128 * half);
+            prefetch_l2((const char *)(c.b + row * KD) + 128 * half);
+            if (!EDGES) {   // the producer reads the raw alpha rows of the layer-edge variant
+                prefetch_l2((const char *)(c.alpha + row * KD) + 256 * half);
+                prefetch_l2((const char *)(c.alpha + row * KD) + 256 * half + 128);
+            }
         }
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
@@ -557,7 +608,7 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                     const int r = p0 + 8 * hf + p, pp = 8 * hf + p;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) f1[j] *= al[pp][j];
-                    if (EDGES) {   // the inverse norms join the decay factors; b through its sigmoid
+                    if (EDGES) {   // the inverse norms join the decay factors before their one rounding
                         const float iq = __shfl_sync(0xffffffffu, iq_l, 2 * pp), ik = __shfl_sync(0xffffffffu, ik_l, 2 * pp);
                         const uint32_t b01 = bsigmoid2(rb[pp].x), b23 = bsigmoid2(rb[pp].y);
                         *reinterpret_cast<uint2 *>(EQ + sw_off(r, c4, 128)) =
@@ -626,11 +677,12 @@ __device__ __forceinline__ void build_group(const Ctx &c, int tid1) {
                         make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
                 }
             }
-            wide_span_ap<EDGES>(c, tid1, t0, L);
+            wide_span_ap<EDGES>(c, src, tid1, L);
         }
         fence_async_smem();
         fence_before();
         group_sync(BAR_BUILD, GROUP);
+        if (EDGES && tid1 == 0) mbar_arrive(mbar(c, MB_RFREE + 8 * (n % RING_SLOTS)));   // ring slot read
         if (tid1 == 0) issue_g1(c, n, slow);
     }
 }
@@ -903,6 +955,53 @@ __device__ __forceinline__ bool warp_wait(const Ctx &c, uint32_t mb, uint32_t pa
     return true;
 }
 
+// Layer-edge producer (o warps, 64 threads): the raw decay-logit rows of chunk m mapped into ring
+// slot m % RING_SLOTS, alpha = 1 / (1 + e^a) = exp(-softplus(a)).  Loads are issued eight at a
+// time before any is used.
+__device__ __forceinline__ void produce_a(const Ctx &c, int m, int tid2) {
+    const int t0 = c.tb + m * C, L = min(C, c.te - t0);
+    float *slot = reinterpret_cast<float *>(c.ring + (m % RING_SLOTS) * RING_BYTES);
+    const size_t base = ((size_t)c.bb * c.T + t0) * c.H + c.h;
+#pragma unroll 1
+    for (int j0 = 0; j0 < 32; j0 += 8) {   // 64 rows x 32 pieces of 4 fp32
+        float4 av[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int p = tid2 + 64 * (j0 + j), r = min(p >> 5, L - 1);
+            av[j] = __ldg(reinterpret_cast<const float4 *>(c.alpha + (base + (size_t)r * c.H) * KD) + (p & 31));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int p = tid2 + 64 * (j0 + j), r = p >> 5;
+            if (r < L)
+                reinterpret_cast<float4 *>(slot + (size_t)r * KD)[p & 31] =
+                    make_float4(alpha_of_logit(av[j].x), alpha_of_logit(av[j].y), alpha_of_logit(av[j].z),
+                                alpha_of_logit(av[j].w));
+        }
+    }
+}
+// raw decay-logit rows of chunk m into L2 ahead of their mapping
+__device__ __forceinline__ void prefetch_edges(const Ctx &c, int m, int tid2) {
+    if (m >= c.NC) return;
+    const int t0 = c.tb + m * C, L = min(C, c.te - t0);
+    const int r = tid2 & 63;
+    if (r >= L) return;
+    const size_t row = ((size_t)c.bb * c.T + t0 + r) * c.H + c.h;
+    const char *a = (const char *)(c.alpha + row * KD);
+    prefetch_l2(a); prefetch_l2(a + 128); prefetch_l2(a + 256); prefetch_l2(a + 384);
+}
+// chunk m's decay rows in its ring slot, once the build group has read the slot's previous chunk;
+// each of the 64 producer threads arrives on the slot's full barrier
+__device__ __forceinline__ bool fill_ring(const Ctx &c, int m, int tid2) {
+    if (m >= c.NC) return true;
+    if (m >= RING_SLOTS &&
+        !warp_wait(c, mbar(c, MB_RFREE + 8 * (m % RING_SLOTS)), (uint32_t)(((m - RING_SLOTS) / RING_SLOTS) & 1)))
+        return false;
+    produce_a(c, m, tid2);
+    mbar_arrive(mbar(c, MB_RFULL + 8 * (m % RING_SLOTS)));   // release: the rows above are visible
+    return true;
+}
+
 template <bool EDGES>
 __device__ __forceinline__ void u_group(const Ctx &c, int tid2) {
     const int vw = tid2 >> 5, lane = tid2 & 31, c4 = lane * 4;
@@ -949,6 +1048,11 @@ __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
     const uint32_t lrow = (uint32_t)(64 + ow * 32) << 16;
     unsigned char *stg = c.sm + SM_OST + ow * 2560;   // 32 rows x 80 B (64 B of data + 16 B pad)
     const bool store = !(c.flags & SEG_SKIP_O);
+    if (EDGES) {   // alpha of the first RING_SLOTS chunks, then each chunk's after the output of the one 4 earlier
+        for (int m = 0; m <= RING_SLOTS; ++m) prefetch_edges(c, m, tid2);
+        for (int m = 0; m < RING_SLOTS; ++m)
+            if (!fill_ring(c, m, tid2)) return;
+    }
     for (int n = 0; n < c.NC; ++n) {
         const int t0 = c.tb + n * C, L = store ? min(C, c.te - t0) : 0;
         if (!warp_wait(c, mbar_slot(c, MB_G45, n), slot_par(n))) return;
@@ -995,6 +1099,10 @@ __device__ __forceinline__ void o_group(const Ctx &c, int tid2) {
         }
         fence_before();
         mbar_arrive(mbar(c, MB_D3FREE));
+        if (EDGES) {
+            if (!fill_ring(c, n + RING_SLOTS, tid2)) return;
+            prefetch_edges(c, n + RING_SLOTS + 1, tid2);
+        }
     }
 }
 
@@ -1005,7 +1113,7 @@ __global__ void __launch_bounds__(NT, 1)
                     const __nv_bfloat16 *__restrict__ b, const __nv_bfloat16 *__restrict__ w,
                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST, int H,
                     int T, int seg_len, int nseg, uint32_t flags, const float *__restrict__ onorm,
-                    unsigned int *__restrict__ status) {
+                    unsigned char *ring, unsigned int *__restrict__ status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -1018,6 +1126,7 @@ __global__ void __launch_bounds__(NT, 1)
     c.tb = seg * seg_len; c.te = min(T, c.tb + seg_len); c.NC = (c.te - c.tb + C - 1) / C;
     c.flags = flags;
     c.onorm = onorm;
+    c.ring = EDGES ? ring + (size_t)blockIdx.x * RING_SLOTS * RING_BYTES : nullptr;
     float *st_dst = (flags & SEG_ST_LAST) ? (seg == nseg - 1 ? ST + (size_t)chain * KD * VD : nullptr)
                                           : ST + (size_t)blockIdx.x * KD * VD;
 
@@ -1026,6 +1135,11 @@ __global__ void __launch_bounds__(NT, 1)
         for (uint32_t off = 0; off < MB_END; off += 8)
             mbar_init(c.misc + off, (off == MB_VEC || off == MB_VEC + 8) ? 32u
                                      : (off == MB_U || off == MB_U + 8 || off == MB_D3FREE) ? 64u : 1u);
+        if (EDGES)
+            for (int i = 0; i < RING_SLOTS; ++i) {
+                mbar_init(c.misc + MB_RFULL + 8 * i, 64u);   // the 64 producer threads
+                mbar_init(c.misc + MB_RFREE + 8 * i, 1u);    // the build group's thread 0
+            }
         *reinterpret_cast<volatile uint32_t *>(sm + SM_MISC + MISC_ABORT) = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1149,10 +1263,11 @@ SegPlan seg_plan(int B, int H, int T) {
 
 }  // namespace
 
-size_t tc_workspace_bytes(int B, int H, int T, int, int, int) {
+size_t tc_workspace_bytes(int B, int H, int T, int, int, int, int edges) {
     const SegPlan sp = seg_plan(B, H, T);
-    if (sp.nseg == 1) return kStatusBytes;
-    return kStatusBytes + 3 * sizeof(float) * (size_t)B * H * sp.nseg * tcfwd::KD * tcfwd::VD;
+    const size_t seg = sp.nseg == 1 ? 0 : 3 * sizeof(float) * (size_t)B * H * sp.nseg * tcfwd::KD * tcfwd::VD;
+    const size_t ring = edges ? (size_t)B * H * sp.nseg * tcfwd::RING_SLOTS * tcfwd::RING_BYTES : 0;
+    return kStatusBytes + seg + ring;
 }
 
 int launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
@@ -1162,13 +1277,15 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
     const int smem = (int)tcfwd::SM_BYTES;
     auto kern = edges ? tcfwd::chunk_tc_kernel<true> : tcfwd::chunk_tc_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -6;
+    const SegPlan sp = seg_plan(B, H, T);
+    const size_t seg_bytes = sp.nseg == 1 ? 0 : 3 * sizeof(float) * (size_t)B * H * sp.nseg * tcfwd::KD * tcfwd::VD;
+    unsigned char *ring = edges ? static_cast<unsigned char *>(ws) + kStatusBytes + seg_bytes : nullptr;
     auto run = [&](int nseg, int seg_len, uint32_t flags, const float *s0, float *st_out) {
         kern<<<B * H * nseg, tcfwd::NT, smem, st>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, alpha,
             (const __nv_bfloat16 *)b, (const __nv_bfloat16 *)w, s0, (__nv_bfloat16 *)o, st_out, H, T, seg_len, nseg,
-            flags, onorm, reinterpret_cast<unsigned int *>(ws));
+            flags, onorm, ring, reinterpret_cast<unsigned int *>(ws));
     };
-    const SegPlan sp = seg_plan(B, H, T);
     if (sp.nseg == 1) {
         run(1, sp.seg_len, 0u, S0, ST);
         return launch_status();

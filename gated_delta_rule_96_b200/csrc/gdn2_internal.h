@@ -21,7 +21,8 @@ int launch_chunk_simt(const void *q, const void *k, const void *v, const float *
 
 // Fused tcgen05 prefill (bf16 tokens, d_k = d_v = 128, C = 64).
 bool tc_supported(int B, int H, int T, int K, int V, int C, int bf16);
-size_t tc_workspace_bytes(int B, int H, int T, int K, int V, int C);
+// edges != 0: the layer-edge variant's ring (RING_SLOTS x 80 KB per block) is included
+size_t tc_workspace_bytes(int B, int H, int T, int K, int V, int C, int edges = 0);
 // edges != 0: q, k, b, w, alpha are the layer's raw inputs (see gdn2_chunk_fwd_edges); onorm, if
 // not null, is the RMSNorm weight applied to o.
 int launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b,

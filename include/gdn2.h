@@ -97,9 +97,14 @@ GDN2_API int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const f
  *   v, w_logit            [B, T, H, d_v]  bf16
  *   a_logit               [B, T, H, d_k]  fp32
  *   o_weight              [d_v] fp32 RMSNorm weight shared by the heads, or NULL (no norm)
- * Everything else as gdn2_chunk_fwd (same workspace size).  Only bf16 tokens with
- * d_k = d_v = 128 and C = 64 are supported (GDN2_ERR_UNSUPPORTED otherwise).
+ * Everything else as gdn2_chunk_fwd, except the workspace: at least
+ * gdn2_chunk_fwd_edges_workspace_bytes(...) bytes (gdn2_chunk_fwd's plus 128 KB per thread
+ * block, B*H blocks, or B*H*segments when few long chains are split in time: the ring in which
+ * the kernel passes the decay rows of the next four chunks between its warps).  A workspace
+ * serves one call at a time.  Only bf16 tokens with d_k = d_v = 128 and C = 64 are supported
+ * (GDN2_ERR_UNSUPPORTED otherwise).
  */
+GDN2_API size_t gdn2_chunk_fwd_edges_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C);
 GDN2_API int gdn2_chunk_fwd_edges(const void *q_raw, const void *k_raw, const void *v, const float *a_logit,
                                   const void *b_logit, const void *w_logit, const float *S0,
                                   const float *o_weight, void *o, float *S_T, int B, int H, int T, int d_k,

@@ -151,3 +151,14 @@ def test_chunk_bwd_validation(lib):
     assert call_bwd(lib, B=0) == 0
     # no tokens and no dS0 wanted: nothing to do, no pointer read
     assert call_bwd(lib, T=0, ptr=None, grad=None, ws=None, ws_bytes=0) == 0
+
+
+def test_edges_workspace_bytes():
+    ring = 4 * 64 * 128 * 4   # four slots of a chunk's decay rows (fp32)
+    assert ring == 128 * 1024
+    assert g.gdn2_chunk_fwd_edges_workspace_bytes(8, 16, 4096, 128, 128) == 256 + 128 * ring
+    # segmented: the segment maps plus one ring per (chain, segment) block
+    state = 4 * 128 * 128
+    assert g.gdn2_chunk_fwd_edges_workspace_bytes(1, 16, 65536, 128, 128) == 256 + 3 * 16 * 8 * state + 16 * 8 * ring
+    # unsupported shapes need only the status header (the call itself is refused)
+    assert g.gdn2_chunk_fwd_edges_workspace_bytes(1, 1, 64, 64, 64) == 256
