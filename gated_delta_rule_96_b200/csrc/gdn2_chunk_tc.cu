@@ -156,11 +156,6 @@ __device__ __forceinline__ float fast_rcp(float x) {
 __device__ __forceinline__ float sigmoid_f(float x) { return fast_rcp(1.f + fast_exp2(-1.4426950408889634f * x)); }
 // alpha = exp(-softplus(a)) = 1 / (1 + e^a) = sigmoid(-a) (0 past fp32's range: the caller floors it)
 __device__ __forceinline__ float alpha_of_logit(float a) { return fast_rcp(1.f + fast_exp2(1.4426950408889634f * a)); }
-// log2 of alpha = exp(-softplus(a)), floored at log2 of the smallest normal float
-__device__ __forceinline__ float log2_alpha_of_logit(float a) {
-    const float sp = a > 15.f ? a : __logf(1.f + __expf(a));
-    return fmaxf(-sp * 1.4426950408889634f, -126.f);
-}
 // load of data that other warps of the block wrote earlier in this kernel (the layer-edge
 // ring): a plain global load, not the read-only path
 __device__ __forceinline__ float4 ld_f4(const float *p) {

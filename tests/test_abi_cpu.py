@@ -25,7 +25,9 @@ def lib():
 def test_header_declares_entry_points():
     syms = declared_symbols()
     for name in ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_fwd_workspace_bytes", "gdn2_status_str",
-                 "gdn2_workspace_status", "gdn2_chunk_fwd_path"):
+                 "gdn2_workspace_status", "gdn2_chunk_fwd_path", "gdn2_chunk_fwd_edges",
+                 "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
+                 "gdn2_chunk_fwd_noalloc"):
         assert name in syms
 
 
