@@ -44,6 +44,12 @@
 // chunk's loads in flight).
 // Every event that a waiter may see two chunks late has one mbarrier per buffer slot.
 // Every wait is bounded; on expiry the block sets the workspace status word and exits.
+//
+// The layer-edge instance (chunk_tc_kernel<true>) takes the layer's raw inputs: the o warps
+// also map the decay logits of chunk n + 4 into a four-slot ring in the workspace
+// (alpha = exp(-softplus(a))), the build group folds the inverse norms of q and k into its
+// decay factors and applies the sigmoid to b, the u group to w, and the o group applies
+// RMSNorm to o when given a weight.
 #include <algorithm>
 
 #include "gdn2_common.cuh"
