@@ -19,7 +19,7 @@ __all__ = [
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
-    "gdn2_chunk_fwd_edges_workspace_bytes",
+    "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_recurrence",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -282,3 +282,47 @@ def decode_step(q, k, v, alpha, b, w, S, stream=None):
     o = torch.empty((B, H, v.shape[-1]), dtype=q.dtype, device=q.device)
     gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=stream)
     return o
+
+
+def _recurrence_function():
+    """torch.autograd.Function over the C ABI: forward gdn2_chunk_fwd, backward gdn2_chunk_bwd."""
+    import torch
+
+    class GDN2Recurrence(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q, k, v, alpha, b, w, S0):
+            o, S_T = chunk_fwd(q, k, v, alpha, b, w, S0)
+            ctx.save_for_backward(q, k, v, alpha, b, w, S0)
+            ctx.has_s0 = S0 is not None
+            return o, S_T
+
+        @staticmethod
+        def backward(ctx, dO, dS_T):
+            q, k, v, alpha, b, w, S0 = ctx.saved_tensors
+            if not ctx.has_s0:
+                S0 = None
+            B, T, H, K = q.shape
+            V = v.shape[-1]
+            dO = torch.zeros_like(v) if dO is None else dO.to(q.dtype).contiguous()
+            dS_T = None if dS_T is None else dS_T.to(torch.float32).contiguous()
+            dev = q.device
+            gk = [torch.empty((B, T, H, K), dtype=torch.float32, device=dev) for _ in range(4)]   # dq dk dalpha db
+            gv = [torch.empty((B, T, H, V), dtype=torch.float32, device=dev) for _ in range(2)]   # dv dw
+            dS0 = torch.empty((B, H, K, V), dtype=torch.float32, device=dev) if ctx.has_s0 else None
+            gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T, gk[0], gk[1], gv[0], gk[2], gk[3], gv[1], dS0)
+            # the autograd engine casts each gradient to its input's dtype
+            return gk[0], gk[1], gv[0], gk[2], gk[3], gv[1], dS0
+
+    return GDN2Recurrence
+
+
+_GDN2_FN = None
+
+
+def gdn2_recurrence(q, k, v, alpha, b, w, S0=None):
+    """Differentiable prefill: (o, S_T) = recurrence(q, k, v, alpha, b, w, S0) with gradients of every
+    input through gdn2_chunk_bwd.  Same shapes and dtypes as gdn2_chunk_fwd (CUDA tensors only)."""
+    global _GDN2_FN
+    if _GDN2_FN is None:
+        _GDN2_FN = _recurrence_function()
+    return _GDN2_FN.apply(q, k, v, alpha, b, w, S0)

@@ -122,3 +122,28 @@ def test_full_size_sampled_chains():
         for name, r in zip(GRADS, ref[:6]):
             check(f"{name} chain {bb},{h}", got[name][bb, :, h], r, c["alpha"])
         assert_close(f"dS0 chain {bb},{h}", got["dS0"][bb, h], ref[6], TOL)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_autograd_function(dtype):
+    """gdn2_recurrence under torch.autograd: the gradients of L = sum(dO * o) + sum(dS_T * S_T) are the
+    oracle's (inputs leaf tensors of the token dtype; the engine casts the fp32 gradients to it)."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("bwa", 1, 2, 100, 64, 128, dtype, 1.0, s0_std=0.05, seed=2104)
+    x = synth.make_inputs(wl)
+    S0 = synth.make_state(wl)
+    dO, dST = output_grads(wl)
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    names = ("q", "k", "v", "alpha", "b", "w")
+    leaves = {n: torch.from_numpy(x[n]).cuda().to(torch.float32 if n == "alpha" else td).requires_grad_() for n in names}
+    S0t = torch.from_numpy(S0).cuda().requires_grad_()
+    o, ST = g.gdn2_recurrence(*(leaves[n] for n in names), S0t)
+    L = (o.float() * torch.from_numpy(dO).cuda().to(td).float()).sum() + (ST * torch.from_numpy(dST).cuda()).sum()
+    L.backward()
+    ref = ob.recurrence_backward(*(x[n] for n in names), S0, dO, dST)
+    a = x["alpha"].astype(np.float64)
+    # bf16 leaves receive gradients rounded to bf16: the bar is the bf16 one there
+    tol = TOL if dtype == "f32" else 2e-2
+    for n, r in zip(names, ref[:6]):
+        check("d" + n, f64(leaves[n].grad), r, a, tol if n != "alpha" else TOL)
+    assert_close("dS0", f64(S0t.grad), ref[6], TOL)
