@@ -60,14 +60,16 @@ __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_grou
 // all but the most recent group complete (this thread's copies)
 __device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// n consecutive steps' rows of one token tensor (E elements per row, rows H apart) -> smem [n][E]
+// n consecutive steps' rows of one token tensor -> smem [n][E]: E elements from each source row
+// (rows of `stride` elements, consecutive steps H rows apart)
 template <int E, typename T>
-__device__ __forceinline__ void stage_rows(T *dst, const T *src, size_t row0, int H, int n, int tid, int NT) {
+__device__ __forceinline__ void stage_rows(T *dst, const T *src, size_t row0, int H, int n, int tid, int NT,
+                                           int stride) {
     constexpr int PPR = E * (int)sizeof(T) / 16;   // 16-byte pieces per row
     for (int p = tid; p < n * PPR; p += NT) {
         const int s = p / PPR, c = p - s * PPR;
         cp_async16(reinterpret_cast<char *>(dst + s * E) + 16 * c,
-                   reinterpret_cast<const char *>(src + (row0 + (size_t)s * H) * E) + 16 * c);
+                   reinterpret_cast<const char *>(src + (row0 + (size_t)s * H) * stride) + 16 * c);
     }
 }
 
@@ -159,11 +161,11 @@ __device__ __forceinline__ void st_red(float *red, int s, int NW, int K, int war
 template <int KR>
 using Mat = float2[KR][4];
 
-template <int KR, int K, int V>
-__device__ __forceinline__ void load_mat(Mat<KR> &M, const float *src, int r0, int c0) {
+template <int KR>
+__device__ __forceinline__ void load_mat(Mat<KR> &M, const float *src, int r0, int col, int stride) {
 #pragma unroll
     for (int i = 0; i < KR; ++i) {
-        if (src) cols_global(src + (size_t)(r0 + i) * V + c0, M[i]);
+        if (src) cols_global(src + (size_t)(r0 + i) * stride + col, M[i]);
         else
 #pragma unroll
             for (int p = 0; p < 4; ++p) M[i][p] = make_float2(0.f, 0.f);
@@ -197,20 +199,23 @@ __device__ __forceinline__ T *at(unsigned char *base, int off) { return reinterp
 
 // ------------------------------------------------------------------------------------ pass 1
 // Forward over S: delta_t -> workspace, dq_t = S_t dO_t -> dq, S at every chunk end -> ckpt.
-template <int KR, int NW, typename Tok>
+template <int KR, int NW, typename Tok, bool SPLIT>
 __global__ void __launch_bounds__(NW * 32, 1)
 pass_forward(const Tok *__restrict__ k, const Tok *__restrict__ v, const float *__restrict__ alpha,
              const Tok *__restrict__ b, const Tok *__restrict__ w, const float *__restrict__ S0,
              const Tok *__restrict__ dO, float *__restrict__ dq, float *__restrict__ delta,
-             float *__restrict__ ckpt, int H, int T, int NC) {
+             float *__restrict__ ckpt, int H, int T, int NC, int Vt_arg, int ns_arg) {
     constexpr int K = 32 * KR, V = 8 * NW, NT = NW * 32;
+    // unsplit: one block holds all V columns of its chain (stride and slice count are constants)
+    const int Vt = SPLIT ? Vt_arg : V, ns = SPLIT ? ns_arg : 1;
     using L = Stage1<K, V, Tok>;
     extern __shared__ __align__(16) unsigned char smem[];
     float *red = reinterpret_cast<float *>(smem);                       // [NB][NW][K]
     unsigned char *stg = smem + NB * NW * K * 4;                         // [2][L::bytes]
-    const int chain = blockIdx.x, bb = chain / H, h = chain % H;
+    // block = (chain, slice of V columns); c0 is the warp's first column in the slice, cg in the state
+    const int chain = blockIdx.x / ns, bb = chain / H, h = chain % H, cb = (blockIdx.x % ns) * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r0 = KR * lane, c0 = 8 * warp, jm = (lane >> 2) & 7;
+    const int r0 = KR * lane, c0 = 8 * warp, cg = cb + c0, jm = (lane >> 2) & 7;
     const int nblk = (T + NB - 1) / NB;
 
     auto stage = [&](int blk) {
@@ -218,15 +223,15 @@ pass_forward(const Tok *__restrict__ k, const Tok *__restrict__ v, const float *
         if (n <= 0) return;
         unsigned char *sb = stg + (blk & 1) * L::bytes;
         const size_t row0 = ((size_t)bb * T + t0) * H + h;
-        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT);
-        stage_rows<V>(at<Tok>(sb, L::vv), v, row0, H, n, tid, NT);
-        stage_rows<V>(at<Tok>(sb, L::ww), w, row0, H, n, tid, NT);
-        stage_rows<V>(at<Tok>(sb, L::go), dO, row0, H, n, tid, NT);
+        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT, K);
+        stage_rows<V>(at<Tok>(sb, L::vv), v + cb, row0, H, n, tid, NT, Vt);
+        stage_rows<V>(at<Tok>(sb, L::ww), w + cb, row0, H, n, tid, NT, Vt);
+        stage_rows<V>(at<Tok>(sb, L::go), dO + cb, row0, H, n, tid, NT, Vt);
     };
     Mat<KR> S;
-    load_mat<KR, K, V>(S, S0 ? S0 + (size_t)chain * K * V : nullptr, r0, c0);
+    load_mat<KR>(S, S0 ? S0 + (size_t)chain * K * Vt : nullptr, r0, cg, Vt);
     stage(0);
     cp_commit();
     stage(1);
@@ -257,7 +262,7 @@ pass_forward(const Tok *__restrict__ k, const Tok *__restrict__ v, const float *
                 }
             }
             const float dmine = u - warp_colsum8(pr, lane);
-            if ((lane & 3) == 0) delta[(((size_t)bb * T + t) * H + h) * V + c0 + jm] = dmine;
+            if ((lane & 3) == 0) delta[(((size_t)bb * T + t) * H + h) * Vt + cg + jm] = dmine;
             float2 d[4];
             broadcast8(dmine, d);
             // S_t = Sbar + k delta^T; row sums of S_t dO_t
@@ -275,15 +280,17 @@ pass_forward(const Tok *__restrict__ k, const Tok *__restrict__ v, const float *
             }
             st_red<KR>(red, s, NW, K, warp, r0, x);
             if (chunk_end(t, T)) {
-                float *ck = ckpt + ((size_t)chain * NC + t / C) * K * V;
+                float *ck = ckpt + ((size_t)chain * NC + t / C) * K * Vt;
 #pragma unroll
-                for (int i = 0; i < KR; ++i) store_cols(ck + (size_t)(r0 + i) * V + c0, S[i]);
+                for (int i = 0; i < KR; ++i) store_cols(ck + (size_t)(r0 + i) * Vt + cg, S[i]);
             }
         }
         __syncthreads();   // block done: row sums complete, its staging buffer free
         for (int idx = tid; idx < n * K; idx += NT) {
             const int s = idx / K, c = idx - s * K;
-            dq[(((size_t)bb * T + t0 + s) * H + h) * K + c] = red_sum<K, NW>(red, s, c);
+            float *d = dq + (((size_t)bb * T + t0 + s) * H + h) * K + c;
+            if (ns > 1) atomicAdd(d, red_sum<K, NW>(red, s, c));   // the other slices' columns add in
+            else *d = red_sum<K, NW>(red, s, c);
         }
         stage(blk + 2);
         cp_commit();
@@ -295,23 +302,26 @@ pass_forward(const Tok *__restrict__ k, const Tok *__restrict__ v, const float *
 // ------------------------------------------------------------------------------------ pass 2
 // Reverse over G: ddelta_t -> workspace, dv, dw, dk_t = G_t delta_t (completed by pass 3),
 // rowsum(G^fut ⊙ S) at every chunk end -> bnd, dS0 = G_0.  Blocks run from the end.
-template <int KR, int NW, typename Tok>
+template <int KR, int NW, typename Tok, bool SPLIT>
 __global__ void __launch_bounds__(NW * 32, 1)
 pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__restrict__ v,
              const float *__restrict__ alpha, const Tok *__restrict__ b, const Tok *__restrict__ w,
              const Tok *__restrict__ dO, const float *__restrict__ dST, const float *__restrict__ delta,
              const float *__restrict__ ckpt, float *__restrict__ ddelta, float *__restrict__ bnd,
              float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dw, float *__restrict__ dS0,
-             int H, int T, int NC) {
+             int H, int T, int NC, int Vt_arg, int ns_arg) {
     constexpr int K = 32 * KR, V = 8 * NW, NT = NW * 32;
+    // unsplit: one block holds all V columns of its chain (stride and slice count are constants)
+    const int Vt = SPLIT ? Vt_arg : V, ns = SPLIT ? ns_arg : 1;
     using L = Stage2<K, V, Tok>;
     extern __shared__ __align__(16) unsigned char smem[];
     float *red = reinterpret_cast<float *>(smem);                  // [NB][NW][K]
     float *rbnd = red + NB * NW * K;                                // [NW][K]
     unsigned char *stg = smem + (NB + 1) * NW * K * 4;              // [2][L::bytes]
-    const int chain = blockIdx.x, bb = chain / H, h = chain % H;
+    // block = (chain, slice of V columns); c0 is the warp's first column in the slice, cg in the state
+    const int chain = blockIdx.x / ns, bb = chain / H, h = chain % H, cb = (blockIdx.x % ns) * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r0 = KR * lane, c0 = 8 * warp, jm = (lane >> 2) & 7;
+    const int r0 = KR * lane, c0 = 8 * warp, cg = cb + c0, jm = (lane >> 2) & 7;
     const int nblk = (T + NB - 1) / NB;
     // reverse block r holds steps lo(r) .. hi(r), hi(r) = T - 1 - r NB; staged at s = t - lo
     auto lo_of = [&](int r) { return max(T - (r + 1) * NB, 0); };
@@ -320,17 +330,17 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
         const int lo = lo_of(r), n = T - r * NB - lo;
         unsigned char *sb = stg + (r & 1) * L::bytes;
         const size_t row0 = ((size_t)bb * T + lo) * H + h;
-        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::qq), q, row0, H, n, tid, NT);
-        stage_rows<V>(at<Tok>(sb, L::vv), v, row0, H, n, tid, NT);
-        stage_rows<V>(at<Tok>(sb, L::ww), w, row0, H, n, tid, NT);
-        stage_rows<V>(at<Tok>(sb, L::go), dO, row0, H, n, tid, NT);
-        stage_rows<V>(at<float>(sb, L::dl), delta, row0, H, n, tid, NT);
+        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::qq), q, row0, H, n, tid, NT, K);
+        stage_rows<V>(at<Tok>(sb, L::vv), v + cb, row0, H, n, tid, NT, Vt);
+        stage_rows<V>(at<Tok>(sb, L::ww), w + cb, row0, H, n, tid, NT, Vt);
+        stage_rows<V>(at<Tok>(sb, L::go), dO + cb, row0, H, n, tid, NT, Vt);
+        stage_rows<V>(at<float>(sb, L::dl), delta + cb, row0, H, n, tid, NT, Vt);
     };
     Mat<KR> G;
-    load_mat<KR, K, V>(G, dST ? dST + (size_t)chain * K * V : nullptr, r0, c0);
+    load_mat<KR>(G, dST ? dST + (size_t)chain * K * Vt : nullptr, r0, cg, Vt);
     stage(0);
     cp_commit();
     stage(1);
@@ -344,12 +354,12 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
             const int s = t - lo;
             if (chunk_end(t, T)) {   // G here is dL/dS_t from the steps after t
                 const int ci = t / C;
-                const float *ck = ckpt + ((size_t)chain * NC + ci) * K * V;
+                const float *ck = ckpt + ((size_t)chain * NC + ci) * K * Vt;
                 float y[KR];
 #pragma unroll
                 for (int i = 0; i < KR; ++i) {
                     float2 sv[4];
-                    cols_global(ck + (size_t)(r0 + i) * V + c0, sv);
+                    cols_global(ck + (size_t)(r0 + i) * Vt + cg, sv);
                     float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int p = 0; p < 4; ++p) acc = __ffma2_rn(G[i][p], sv[p], acc);
@@ -357,7 +367,11 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
                 }
                 st_red<KR>(rbnd, 0, NW, K, warp, r0, y);
                 __syncthreads();
-                for (int c = tid; c < K; c += NT) bnd[((size_t)chain * NC + ci) * K + c] = red_sum<K, NW>(rbnd, 0, c);
+                for (int c = tid; c < K; c += NT) {
+                    float *d = bnd + ((size_t)chain * NC + ci) * K + c;
+                    if (ns > 1) atomicAdd(d, red_sum<K, NW>(rbnd, 0, c));
+                    else *d = red_sum<K, NW>(rbnd, 0, c);
+                }
                 __syncthreads();
             }
             float al[KR], kk[KR], bk[KR], qq[KR];
@@ -381,7 +395,7 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
             }
             const float ddm = warp_colsum8(pr, lane);
             if ((lane & 3) == 0) {
-                const size_t e = (((size_t)bb * T + t) * H + h) * V + c0 + jm;
+                const size_t e = (((size_t)bb * T + t) * H + h) * Vt + cg + jm;
                 ddelta[e] = ddm;
                 dv[e] = ddm * to_f32(at<Tok>(sb, L::ww)[s * V + c0 + jm]);
                 dw[e] = ddm * to_f32(at<Tok>(sb, L::vv)[s * V + c0 + jm]);
@@ -406,7 +420,9 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
         __syncthreads();
         for (int idx = tid; idx < (hi - lo + 1) * K; idx += NT) {
             const int s = idx / K, c = idx - s * K;   // slot s holds step hi - s
-            dk[(((size_t)bb * T + hi - s) * H + h) * K + c] = red_sum<K, NW>(red, s, c);
+            float *d = dk + (((size_t)bb * T + hi - s) * H + h) * K + c;
+            if (ns > 1) atomicAdd(d, red_sum<K, NW>(red, s, c));
+            else *d = red_sum<K, NW>(red, s, c);
         }
         stage(r + 2);
         cp_commit();
@@ -415,29 +431,31 @@ pass_reverse(const Tok *__restrict__ q, const Tok *__restrict__ k, const Tok *__
     }
     if (dS0) {
 #pragma unroll
-        for (int i = 0; i < KR; ++i) store_cols(dS0 + ((size_t)chain * K + r0 + i) * V + c0, G[i]);
+        for (int i = 0; i < KR; ++i) store_cols(dS0 + ((size_t)chain * K + r0 + i) * Vt + cg, G[i]);
     }
 }
 
 // ------------------------------------------------------------------------------------ pass 3
 // Forward over S with the kept delta: S_{t-1} ddelta_t gives de = -alpha ⊙ (S_{t-1} ddelta);
 // then db, the complete dk, and per chunk the log-decay sums -> dalpha.
-template <int KR, int NW, typename Tok>
+template <int KR, int NW, typename Tok, bool SPLIT>
 __global__ void __launch_bounds__(NW * 32, 1)
 pass_gates(const Tok *__restrict__ q, const Tok *__restrict__ k, const float *__restrict__ alpha,
            const Tok *__restrict__ b, const float *__restrict__ S0, const float *__restrict__ delta,
            const float *__restrict__ ddelta, const float *__restrict__ bnd, const float *__restrict__ dq,
-           float *__restrict__ dk, float *__restrict__ db, float *__restrict__ dalpha, int H, int T, int NC) {
+           float *__restrict__ dk, float *__restrict__ db, float *__restrict__ dalpha, float *__restrict__ X, int H,
+           int T, int NC, int Vt_arg, int ns_arg) {
     constexpr int K = 32 * KR, V = 8 * NW, NT = NW * 32;
+    const int Vt = SPLIT ? Vt_arg : V, ns = SPLIT ? ns_arg : 1;
     using L = Stage3<K, V, Tok>;
     extern __shared__ __align__(16) unsigned char smem[];
     float *red = reinterpret_cast<float *>(smem);           // [NB][NW][K]
     float *hbuf = red + NB * NW * K;                         // [C][K] dL/dg of the chunk's steps
     float *abuf = hbuf + C * K;                              // [C][K] alpha of the chunk's steps
     unsigned char *stg = reinterpret_cast<unsigned char *>(abuf + C * K);   // [2][L::bytes]
-    const int chain = blockIdx.x, bb = chain / H, h = chain % H;
+    const int chain = blockIdx.x / ns, bb = chain / H, h = chain % H, cb = (blockIdx.x % ns) * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r0 = KR * lane, c0 = 8 * warp;
+    const int r0 = KR * lane, c0 = 8 * warp, cg = cb + c0;
     const int nblk = (T + NB - 1) / NB;
 
     auto stage = [&](int blk) {
@@ -445,17 +463,19 @@ pass_gates(const Tok *__restrict__ q, const Tok *__restrict__ k, const float *__
         if (n <= 0) return;
         unsigned char *sb = stg + (blk & 1) * L::bytes;
         const size_t row0 = ((size_t)bb * T + t0) * H + h;
-        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT);
-        stage_rows<K>(at<Tok>(sb, L::qq), q, row0, H, n, tid, NT);
-        stage_rows<K>(at<float>(sb, L::dq), dq, row0, H, n, tid, NT);
-        stage_rows<K>(at<float>(sb, L::dk), static_cast<const float *>(dk), row0, H, n, tid, NT);
-        stage_rows<V>(at<float>(sb, L::dl), delta, row0, H, n, tid, NT);
-        stage_rows<V>(at<float>(sb, L::dd), ddelta, row0, H, n, tid, NT);
+        stage_rows<K>(at<float>(sb, L::al), alpha, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::kk), k, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::bk), b, row0, H, n, tid, NT, K);
+        stage_rows<K>(at<Tok>(sb, L::qq), q, row0, H, n, tid, NT, K);
+        if (ns == 1) {   // the complete row sums are formed here only when the block holds every column
+            stage_rows<K>(at<float>(sb, L::dq), dq, row0, H, n, tid, NT, K);
+            stage_rows<K>(at<float>(sb, L::dk), static_cast<const float *>(dk), row0, H, n, tid, NT, K);
+        }
+        stage_rows<V>(at<float>(sb, L::dl), delta + cb, row0, H, n, tid, NT, Vt);
+        stage_rows<V>(at<float>(sb, L::dd), ddelta + cb, row0, H, n, tid, NT, Vt);
     };
     Mat<KR> S;
-    load_mat<KR, K, V>(S, S0 ? S0 + (size_t)chain * K * V : nullptr, r0, c0);
+    load_mat<KR>(S, S0 ? S0 + (size_t)chain * K * Vt : nullptr, r0, cg, Vt);
     stage(0);
     cp_commit();
     stage(1);
@@ -487,6 +507,18 @@ pass_gates(const Tok *__restrict__ q, const Tok *__restrict__ k, const float *__
             st_red<KR>(red, s, NW, K, warp, r0, x);
         }
         __syncthreads();
+        if (ns > 1) {   // partial row sums S_{t-1} ddelta over this slice's columns; gates_finalize completes
+            for (int idx = tid; idx < n * K; idx += NT) {
+                const int s = idx / K, c = idx - s * K;
+                atomicAdd(X + (((size_t)bb * T + t0 + s) * H + h) * K + c, red_sum<K, NW>(red, s, c));
+            }
+            __syncthreads();
+            stage(blk + 2);
+            cp_commit();
+            cp_wait_prev();
+            __syncthreads();
+            continue;
+        }
         for (int idx = tid; idx < n * K; idx += NT) {
             const int s = idx / K, c = idx - s * K;
             const size_t e = (((size_t)bb * T + t0 + s) * H + h) * K + c;
@@ -521,6 +553,31 @@ pass_gates(const Tok *__restrict__ q, const Tok *__restrict__ k, const float *__
     }
 }
 
+// Column-sliced chains: completes pass 3 from the summed partial row sums X = S_{t-1} ddelta.
+// One block per (chain, chunk), one thread per key channel, walking the chunk backwards.
+template <typename Tok>
+__global__ void __launch_bounds__(128)
+gates_finalize(const Tok *__restrict__ q, const Tok *__restrict__ k, const float *__restrict__ alpha,
+               const Tok *__restrict__ b, const float *__restrict__ X, const float *__restrict__ bnd,
+               const float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ db,
+               float *__restrict__ dalpha, int H, int T, int NC, int K) {
+    const int chain = blockIdx.x, ci = blockIdx.y, bb = chain / H, h = chain % H;
+    const int cs = ci * C, ce = min(cs + C, T);
+    for (int c = threadIdx.x; c < K; c += blockDim.x) {
+        float acc = bnd[((size_t)chain * NC + ci) * K + c];
+        for (int t = ce - 1; t >= cs; --t) {
+            const size_t e = (((size_t)bb * T + t) * H + h) * K + c;
+            const float a = alpha[e], kc = to_f32(k[e]), bc = to_f32(b[e]), qc = to_f32(q[e]);
+            const float de = -a * X[e];
+            const float dkt = dk[e] + bc * de;
+            dk[e] = dkt;
+            db[e] = kc * de;
+            acc += qc * dq[e] + 2.f * bc * kc * de - kc * dkt;   // dL/dg_t, summed back from the chunk end
+            dalpha[e] = acc / fmaxf(a, FLT_MIN);
+        }
+    }
+}
+
 template <int K, int V, typename Tok>
 constexpr size_t smem1() { return (size_t)NB * (V / 8) * K * 4 + 2 * Stage1<K, V, Tok>::bytes; }
 template <int K, int V, typename Tok>
@@ -528,40 +585,60 @@ constexpr size_t smem2() { return (size_t)(NB + 1) * (V / 8) * K * 4 + 2 * Stage
 template <int K, int V, typename Tok>
 constexpr size_t smem3() { return (size_t)NB * (V / 8) * K * 4 + 2 * (size_t)C * K * 4 + 2 * Stage3<K, V, Tok>::bytes; }
 
-template <int KR, int NW, typename Tok>
+template <int KR, int NW, typename Tok, bool SPLIT>
 int launch_all(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
                const float *S0, const void *dO, const float *dST, float *dq, float *dk, float *dv, float *dalpha,
-               float *db, float *dw, float *dS0, int B, int H, int T, float *delta, float *ddelta, float *ckpt,
-               float *bnd, cudaStream_t st) {
-    constexpr int K = 32 * KR, V = 8 * NW;
+               float *db, float *dw, float *dS0, int B, int H, int T, int Vt, int ns, float *delta, float *ddelta,
+               float *ckpt, float *bnd, float *X, cudaStream_t st) {
+    constexpr int K = 32 * KR, V = 8 * NW;   // V: the columns of one block (Vt / ns)
     constexpr size_t sm1 = smem1<K, V, Tok>(), sm2 = smem2<K, V, Tok>(), sm3 = smem3<K, V, Tok>();
     static_assert(sm1 <= 227 * 1024 && sm2 <= 227 * 1024 && sm3 <= 227 * 1024, "shared memory");
-    const int NC = (T + C - 1) / C, NT = NW * 32, grid = B * H;
-    auto f1 = pass_forward<KR, NW, Tok>;
-    auto f2 = pass_reverse<KR, NW, Tok>;
-    auto f3 = pass_gates<KR, NW, Tok>;
+    const int NC = (T + C - 1) / C, NT = NW * 32, grid = B * H * ns;
+    if (ns > 1) {   // row sums accumulate over the slices
+        const size_t tokk = sizeof(float) * (size_t)B * T * H * K;
+        if (cudaMemsetAsync(dq, 0, tokk, st) != cudaSuccess || cudaMemsetAsync(dk, 0, tokk, st) != cudaSuccess ||
+            cudaMemsetAsync(X, 0, tokk, st) != cudaSuccess ||
+            cudaMemsetAsync(bnd, 0, sizeof(float) * (size_t)B * H * NC * K, st) != cudaSuccess)
+            return -6;
+    }
+    auto f1 = pass_forward<KR, NW, Tok, SPLIT>;
+    auto f2 = pass_reverse<KR, NW, Tok, SPLIT>;
+    auto f3 = pass_gates<KR, NW, Tok, SPLIT>;
     if (cudaFuncSetAttribute(f1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1) != cudaSuccess ||
         cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2) != cudaSuccess ||
         cudaFuncSetAttribute(f3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3) != cudaSuccess)
         return -6;
     const Tok *tq = static_cast<const Tok *>(q), *tk = static_cast<const Tok *>(k), *tv = static_cast<const Tok *>(v);
     const Tok *tb = static_cast<const Tok *>(b), *tw = static_cast<const Tok *>(w), *tdo = static_cast<const Tok *>(dO);
-    f1<<<grid, NT, sm1, st>>>(tk, tv, alpha, tb, tw, S0, tdo, dq, delta, ckpt, H, T, NC);
+    f1<<<grid, NT, sm1, st>>>(tk, tv, alpha, tb, tw, S0, tdo, dq, delta, ckpt, H, T, NC, Vt, ns);
     f2<<<grid, NT, sm2, st>>>(tq, tk, tv, alpha, tb, tw, tdo, dST, delta, ckpt, ddelta, bnd, dk, dv, dw, dS0, H, T,
-                              NC);
-    f3<<<grid, NT, sm3, st>>>(tq, tk, alpha, tb, S0, delta, ddelta, bnd, dq, dk, db, dalpha, H, T, NC);
+                              NC, Vt, ns);
+    f3<<<grid, NT, sm3, st>>>(tq, tk, alpha, tb, S0, delta, ddelta, bnd, dq, dk, db, dalpha, X, H, T, NC, Vt, ns);
+    if (ns > 1)
+        gates_finalize<Tok><<<dim3(B * H, NC), 128, 0, st>>>(tq, tk, alpha, tb, X, bnd, dq, dk, db, dalpha, H, T, NC,
+                                                              K);
     return launch_status();
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Column slices per chain: few chains would leave most of the 148 SMs idle, and the value columns
+// of every pass are independent, so a chain's columns are split over up to 8 blocks (at least 16
+// columns, two warps, each) while the blocks fit on the SMs.
+inline int slices(int chains, int V) {
+    int ns = 1;
+    while (ns * 2 * chains <= 148 && V / (8 * ns * 2) >= 2) ns *= 2;
+    return ns;
+}
 
 }  // namespace bwd
 
 
 size_t bwd_workspace_bytes(int B, int H, int T, int K, int V) {
     const size_t ntok = (size_t)B * T * H, NC = (size_t)(T + bwd::C - 1) / bwd::C;
+    const bool split = bwd::slices(B * H, V) > 1;   // + the partial row sums of pass 3
     return 2 * bwd::align256(sizeof(float) * ntok * V) + bwd::align256(sizeof(float) * B * H * NC * K * V) +
-           bwd::align256(sizeof(float) * B * H * NC * K);
+           bwd::align256(sizeof(float) * B * H * NC * K) + (split ? bwd::align256(sizeof(float) * ntok * K) : 0);
 }
 
 int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
@@ -577,20 +654,26 @@ int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *a
     float *ckpt = reinterpret_cast<float *>(p);
     p += bwd::align256(sizeof(float) * B * H * NC * K * V);
     float *bnd = reinterpret_cast<float *>(p);
-#define GDN2_BWD(KR, NW, TOK)                                                                                    \
-    return bwd::launch_all<KR, NW, TOK>(q, k, v, alpha, b, w, S0, dO, dST, dq, dk, dv, dalpha, db, dw, dS0, B, H, \
-                                        T, delta, ddelta, ckpt, bnd, st)
+    p += bwd::align256(sizeof(float) * B * H * NC * K);
+    float *X = reinterpret_cast<float *>(p);
+    const int ns = bwd::slices(B * H, V), nw = V / 8 / ns;   // warps per block
+#define GDN2_BWD(KR, NW, TOK, SPLIT)                                                                            \
+    return bwd::launch_all<KR, NW, TOK, SPLIT>(q, k, v, alpha, b, w, S0, dO, dST, dq, dk, dv, dalpha, db, dw, dS0, \
+                                               B, H, T, V, ns, delta, ddelta, ckpt, bnd, X, st)
+#define GDN2_BWD_NW(KR, TOK)                              \
+    if (ns == 1 && nw == 16) GDN2_BWD(KR, 16, TOK, false); \
+    if (ns == 1 && nw == 8) GDN2_BWD(KR, 8, TOK, false);   \
+    if (ns > 1 && nw == 8) GDN2_BWD(KR, 8, TOK, true);     \
+    if (ns > 1 && nw == 4) GDN2_BWD(KR, 4, TOK, true);     \
+    if (ns > 1 && nw == 2) GDN2_BWD(KR, 2, TOK, true);
     if (bf16) {
-        if (K == 128 && V == 128) GDN2_BWD(4, 16, __nv_bfloat16);
-        if (K == 128 && V == 64) GDN2_BWD(4, 8, __nv_bfloat16);
-        if (K == 64 && V == 128) GDN2_BWD(2, 16, __nv_bfloat16);
-        if (K == 64 && V == 64) GDN2_BWD(2, 8, __nv_bfloat16);
+        if (K == 128) { GDN2_BWD_NW(4, __nv_bfloat16) }
+        if (K == 64) { GDN2_BWD_NW(2, __nv_bfloat16) }
     } else {
-        if (K == 128 && V == 128) GDN2_BWD(4, 16, float);
-        if (K == 128 && V == 64) GDN2_BWD(4, 8, float);
-        if (K == 64 && V == 128) GDN2_BWD(2, 16, float);
-        if (K == 64 && V == 64) GDN2_BWD(2, 8, float);
+        if (K == 128) { GDN2_BWD_NW(4, float) }
+        if (K == 64) { GDN2_BWD_NW(2, float) }
     }
+#undef GDN2_BWD_NW
 #undef GDN2_BWD
     return -4;
 }

@@ -128,9 +128,10 @@ def test_bwd_workspace_bytes():
     # two fp32 [B,T,H,d_v] buffers, the state every 64 steps, one d_k vector every 64 steps
     assert g.gdn2_chunk_bwd_workspace_bytes(8, 16, 4096, 128, 128) == \
         2 * a(4 * ntok * 128) + a(128 * 64 * state) + a(128 * 64 * 4 * 128)
-    # a ragged tail costs a whole chunk of checkpoints
+    # a ragged tail costs a whole chunk of checkpoints; a single chain splits its value columns over
+    # several blocks, which adds the partial row sums of the last pass (fp32 [B,T,H,d_k])
     assert g.gdn2_chunk_bwd_workspace_bytes(1, 1, 65, 64, 128) == \
-        2 * a(4 * 65 * 128) + a(2 * 4 * 64 * 128) + a(2 * 4 * 64)
+        2 * a(4 * 65 * 128) + a(2 * 4 * 64 * 128) + a(2 * 4 * 64) + a(4 * 65 * 64)
     assert g.gdn2_chunk_bwd_workspace_bytes(1, 1, 8, 96, 128) == 0
 
 
