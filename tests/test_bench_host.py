@@ -94,3 +94,11 @@ def test_two_rank_plumbing_gloo():
     assert [r[0] for r in res] == [0, 1]
     assert all(r[2] == 20.0 and r[3] == 3.0 for r in res)     # max and sum over ranks
     assert res[0][4] != res[1][4]                              # distinct shards
+
+
+def test_backward_accounting():
+    import bench
+    # 21 fp32 flops per state element per token-head across the three passes
+    assert bench.backward_flops(8, 4096, 16, 128, 128) == 21 * 8 * 4096 * 16 * 128 * 128 == 180388626432
+    # 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz
+    assert abs(bench.fp32_alu_peak_tflops(148, 1965.0) - 74.44992) < 1e-9
