@@ -147,3 +147,10 @@ def test_autograd_function(dtype):
     for n, r in zip(names, ref[:6]):
         check("d" + n, f64(leaves[n].grad), r, a, tol if n != "alpha" else TOL)
     assert_close("dS0", f64(S0t.grad), ref[6], TOL)
+
+
+def test_few_long_chains_column_split():
+    """Two chains of 1,000 tokens (16 chunks): each chain's columns split over 8 blocks, so the row
+    sums and the 16 chunk-boundary terms accumulate from every slice."""
+    wl = synth.Workload("bwl", 1, 2, 1000, 128, 128, "bf16", 1.0, s0_std=0.05, seed=2105)
+    full_case(wl)
