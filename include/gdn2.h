@@ -148,7 +148,10 @@ GDN2_API size_t gdn2_chunk_bwd_workspace_bytes(int B, int H, int T, int d_k, int
  * Every gradient is computed and written in fp32 whatever the token dtype.  dalpha is
  * formed as d(log alpha) / alpha with alpha floored at FLT_MIN.  T = 0 writes dS0 = dS_T
  * (or zeros) and reads no token pointer.  d_k, d_v in {64, 128}.  The output buffers must
- * not alias the inputs or each other.  Three kernel launches on `stream`.
+ * not alias the inputs or each other.  Three kernel launches on `stream`; with few chains
+ * (2*B*H <= 148) each chain's value columns are split over several blocks, which adds zero fills of
+ * dq, dk and workspace buffers and a fourth, small kernel.  Results are deterministic in the
+ * unsplit case; in the split case the row sums are added in an unspecified order (fp32 rounding).
  */
 GDN2_API int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const void *b,
                             const void *w, const float *S0, const void *dO, const float *dS_T, float *dq,
