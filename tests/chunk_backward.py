@@ -1,0 +1,93 @@
+"""Test-only fp64 chunkwise restatement of the recurrence's gradient (the WY backward form).
+
+The forward chunk algebra is that of tests/chunk_algebra.py (page "NVIDIA представила
+Gated DeltaNet-2 ...", the chunkwise WY form).  Per chunk of L tokens with incoming state S,
+g = cumulative log alpha inside the chunk, Γ = exp(g), E = b ⊙ k, U = w ⊙ v:
+
+    Ê = Γ ⊙ E,  Q̂ = Γ ⊙ Q,  Ǩ = exp(-g) ⊙ K,  A = strict_lower(Ê Ǩ^T),  P = lower(Q̂ Ǩ^T)
+    R = U - Ê S,  Δ = (I + A)^-1 R,  O = Q̂ S + P Δ,  S' = Diag(γ) (S + Ǩ^T Δ),  γ = exp(g_{L-1})
+
+Given dO and dS' (the gradient at the chunk's outgoing state) the chunk's gradients are matrix
+products of the same shapes as the forward's:
+
+    dΔ = P^T dO + Ǩ (γ ⊙ dS'),          dR = (I + A)^-T dΔ
+    dA = -strict_lower(dR Δ^T),          dP = lower(dO Δ^T)
+    dÊ = -dR S^T + dA Ǩ,                 dQ̂ = dO S^T + dP Ǩ
+    dǨ = dA^T Ê + dP^T Q̂ + Δ (γ ⊙ dS')^T
+    dS = Q̂^T dO - Ê^T dR + γ ⊙ dS'      (to the previous chunk)
+
+then dq = Γ ⊙ dQ̂, de = Γ ⊙ dÊ, the key's own part exp(-g) ⊙ dǨ, and for the decay
+dL/dg_r = (Q̂ ⊙ dQ̂ + Ê ⊙ dÊ - Ǩ ⊙ dǨ)_r, summed from the chunk's end back to each position,
+plus rowsum(dS' ⊙ S') for the γ that scales the outgoing state.  This is the form a
+tensor-core backward would evaluate; here it pins the step-wise oracle (tests/test_chunk_backward.py).
+"""
+import numpy as np
+
+
+def chunk_grads(q, k, v, alpha, b, w, S, dO, dS_out):
+    """One chunk ([L, d] fp64 arrays, S and dS_out [K, V]).
+    Returns (dq, dk, dv, dalpha, db, dw, dS_in)."""
+    L = q.shape[0]
+    g = np.cumsum(np.log(alpha), axis=0)
+    Gam, Ginv = np.exp(g), np.exp(-g)
+    gam = Gam[-1]
+    e, u = b * k, w * v
+    Eh, Qh, Kc = Gam * e, Gam * q, Ginv * k
+    strict = np.tril(np.ones((L, L)), -1)
+    lower = np.tril(np.ones((L, L)), 0)
+    A = (Eh @ Kc.T) * strict
+    P = (Qh @ Kc.T) * lower
+    IA = np.eye(L) + A
+    R = u - Eh @ S
+    Delta = np.linalg.solve(IA, R)
+    S_out = gam[:, None] * (S + Kc.T @ Delta)
+
+    gdS = gam[:, None] * dS_out
+    dDelta = P.T @ dO + Kc @ gdS
+    dR = np.linalg.solve(IA.T, dDelta)
+    dA = -(dR @ Delta.T) * strict
+    dP = (dO @ Delta.T) * lower
+    dEh = -dR @ S.T + dA @ Kc
+    dQh = dO @ S.T + dP @ Kc
+    dKc = dA.T @ Eh + dP.T @ Qh + Delta @ gdS.T
+    dS_in = Qh.T @ dO - Eh.T @ dR + gdS
+
+    dq = Gam * dQh
+    de = Gam * dEh
+    dk = Ginv * dKc + b * de
+    db = k * de
+    dv = w * dR
+    dw = v * dR
+    h = Qh * dQh + Eh * dEh - Kc * dKc
+    dlog = np.cumsum(h[::-1], axis=0)[::-1] + np.sum(dS_out * S_out, axis=1)[None, :]
+    return dq, dk, dv, dlog / alpha, db, dw, dS_in
+
+
+def chunked_grads(q, k, v, alpha, b, w, S0, dO, dST, C):
+    """Whole chain ([T, d] arrays) in chunks of C (last one ragged): forward to collect each chunk's
+    incoming state, then the chunks in reverse."""
+    T, K = q.shape
+    V = v.shape[1]
+    S = np.zeros((K, V)) if S0 is None else np.array(S0, dtype=np.float64)
+    starts = []
+    for t0 in range(0, T, C):
+        t1 = min(T, t0 + C)
+        starts.append(S)
+        g = np.cumsum(np.log(alpha[t0:t1]), axis=0)
+        Gam = np.exp(g)
+        e, u = b[t0:t1] * k[t0:t1], w[t0:t1] * v[t0:t1]
+        Kc = np.exp(-g) * k[t0:t1]
+        A = ((Gam * e) @ Kc.T) * np.tril(np.ones((t1 - t0, t1 - t0)), -1)
+        Delta = np.linalg.solve(np.eye(t1 - t0) + A, u - (Gam * e) @ S)
+        S = Gam[-1][:, None] * (S + Kc.T @ Delta)
+    out = [np.zeros((T, K)), np.zeros((T, K)), np.zeros((T, V)), np.zeros((T, K)), np.zeros((T, K)),
+           np.zeros((T, V))]
+    dS = np.zeros((K, V)) if dST is None else np.array(dST, dtype=np.float64)
+    for ci in range(len(starts) - 1, -1, -1):
+        t0, t1 = ci * C, min(T, ci * C + C)
+        sl = slice(t0, t1)
+        g = chunk_grads(q[sl], k[sl], v[sl], alpha[sl], b[sl], w[sl], starts[ci], dO[sl], dS)
+        for i in range(6):
+            out[i][sl] = g[i]
+        dS = g[6]
+    return tuple(out) + (dS,)
