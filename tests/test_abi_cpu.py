@@ -165,3 +165,18 @@ def test_edges_workspace_bytes():
     assert g.gdn2_chunk_fwd_edges_workspace_bytes(1, 16, 65536, 128, 128) == 256 + 3 * 16 * 8 * state + 16 * 8 * ring
     # unsupported shapes need only the status header (the call itself is refused)
     assert g.gdn2_chunk_fwd_edges_workspace_bytes(1, 1, 64, 64, 64) == 256
+
+
+def test_bwd_column_split_threshold():
+    """The backward splits a chain's value columns while 2 x blocks still fit the 148 SMs: the split
+    adds the fp32 [B,T,H,d_k] partial row sums to the workspace."""
+    a = lambda n: (n + 255) // 256 * 256
+    T, K, V = 128, 128, 128
+
+    def base(chains):
+        ntok = chains * T
+        return 2 * a(4 * ntok * V) + a(chains * 2 * 4 * K * V) + a(chains * 2 * 4 * K)
+
+    for chains, split in ((74, True), (75, False), (128, False), (1, True)):
+        extra = a(4 * chains * T * K) if split else 0
+        assert g.gdn2_chunk_bwd_workspace_bytes(1, chains, T, K, V) == base(chains) + extra, chains
