@@ -35,6 +35,10 @@
 // shared memory and are flushed every NB steps.  The token rows of each block of NB steps
 // are copied into shared memory with cp.async two blocks ahead, so the step loop reads
 // only registers and shared memory.
+//
+// Few chains: the value columns are independent in all three passes, so a chain's columns are
+// split over up to 8 blocks (SPLIT instances); the row sums then accumulate with atomics and
+// gates_finalize completes de, db, dk and the decay sums per chunk.
 #include <float.h>
 
 #include "gdn2_common.cuh"
