@@ -37,7 +37,7 @@
 // only registers and shared memory.
 //
 // Few chains: the value columns are independent in all three passes, so a chain's columns are
-// split over up to 8 blocks (SPLIT instances); the row sums then accumulate with atomics and
+// split over up to 4 blocks (SPLIT instances); the row sums then accumulate with atomics and
 // gates_finalize completes de, db, dk and the decay sums per chunk.
 #include <float.h>
 
@@ -627,11 +627,11 @@ int launch_all(const void *q, const void *k, const void *v, const float *alpha, 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Column slices per chain: few chains would leave most of the 148 SMs idle, and the value columns
-// of every pass are independent, so a chain's columns are split over up to 8 blocks (at least 16
-// columns, two warps, each) while the blocks fit on the SMs.
+// of every pass are independent, so a chain's columns are split over up to 4 blocks (at least 32
+// columns, four warps, each: faster than 8 blocks of two warps) while the blocks fit on the SMs.
 inline int slices(int chains, int V) {
     int ns = 1;
-    while (ns * 2 * chains <= 148 && V / (8 * ns * 2) >= 2) ns *= 2;
+    while (ns * 2 * chains <= 148 && V / (8 * ns * 2) >= 4) ns *= 2;
     return ns;
 }
 
@@ -668,8 +668,7 @@ int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *a
     if (ns == 1 && nw == 16) GDN2_BWD(KR, 16, TOK, false); \
     if (ns == 1 && nw == 8) GDN2_BWD(KR, 8, TOK, false);   \
     if (ns > 1 && nw == 8) GDN2_BWD(KR, 8, TOK, true);     \
-    if (ns > 1 && nw == 4) GDN2_BWD(KR, 4, TOK, true);     \
-    if (ns > 1 && nw == 2) GDN2_BWD(KR, 2, TOK, true);
+    if (ns > 1 && nw == 4) GDN2_BWD(KR, 4, TOK, true);
     if (bf16) {
         if (K == 128) { GDN2_BWD_NW(4, __nv_bfloat16) }
         if (K == 64) { GDN2_BWD_NW(2, __nv_bfloat16) }

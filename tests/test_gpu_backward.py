@@ -150,7 +150,7 @@ def test_autograd_function(dtype):
 
 
 def test_few_long_chains_column_split():
-    """Two chains of 1,000 tokens (16 chunks): each chain's columns split over 8 blocks, so the row
+    """Two chains of 1,000 tokens (16 chunks): each chain's columns split over 4 blocks, so the row
     sums and the 16 chunk-boundary terms accumulate from every slice."""
     wl = synth.Workload("bwl", 1, 2, 1000, 128, 128, "bf16", 1.0, s0_std=0.05, seed=2105)
     full_case(wl)
