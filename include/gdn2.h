@@ -127,7 +127,8 @@ GDN2_API int gdn2_decode_step(const void *q, const void *k, const void *v, const
 
 /* Bytes of device workspace gdn2_chunk_bwd needs (0 on bad sizes).  Depends only on its
  * arguments: two fp32 [B, T, H, d_v] buffers, the fp32 state at every 64th step of every
- * chain, and one fp32 d_k vector per 64 steps per chain. */
+ * chain, one fp32 d_k vector per 64 steps per chain, and, when few chains split their value
+ * columns over blocks (2*B*H <= 148), one fp32 [B, T, H, d_k] buffer of partial row sums. */
 GDN2_API size_t gdn2_chunk_bwd_workspace_bytes(int B, int H, int T, int d_k, int d_v);
 
 /*
