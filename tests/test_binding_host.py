@@ -1,0 +1,101 @@
+"""Host-side checks of the Python binding's argument marshalling, on the CPU: the compute entry
+points of the library are replaced by a recorder (the workspace-size queries stay the real
+library's), the device checks by no-ops, and the recorded C arguments are compared with the
+tensors passed in: order of the pointers, sizes, dtype code, workspace size; shape and dtype
+errors are raised before any call."""
+import ctypes
+
+import pytest
+import torch
+
+import gated_delta_rule_96_b200 as g
+
+
+class Recorder:
+    def __init__(self, real):
+        self.real = real
+        self.calls = []
+
+    def __getattr__(self, name):
+        if name.endswith("_workspace_bytes") or name in ("gdn2_status_str", "gdn2_chunk_fwd_path"):
+            return getattr(self.real, name)
+
+        def record(*args):
+            self.calls.append((name, args))
+            return 0
+        return record
+
+
+@pytest.fixture
+def rec(monkeypatch):
+    r = Recorder(g.load_library())
+    monkeypatch.setattr(g, "load_library", lambda: r)
+    monkeypatch.setattr(g, "_check_cuda", lambda *ts: None)
+    monkeypatch.setattr(g, "_stream", lambda s: ctypes.c_void_p(0))
+    monkeypatch.setattr(g, "new_workspace", lambda n, device=None: torch.zeros(max(int(n), 256), dtype=torch.uint8))
+    return r
+
+
+def addr(p):
+    return None if p is None else p.value
+
+
+def test_bwd_marshalling(rec):
+    B, T, H, K, V = 2, 70, 3, 64, 128
+    tk = lambda dt=torch.bfloat16: torch.zeros(B, T, H, K, dtype=dt)
+    tv = lambda dt=torch.bfloat16: torch.zeros(B, T, H, V, dtype=dt)
+    st = lambda: torch.zeros(B, H, K, V)
+    ins = [tk(), tk(), tv(), tk(torch.float32), tk(), tv(), st(), tv(), st()]
+    outs = [tk(torch.float32), tk(torch.float32), tv(torch.float32), tk(torch.float32), tk(torch.float32),
+            tv(torch.float32), st()]
+    g.gdn2_chunk_bwd(*ins, *outs)
+    name, args = rec.calls[-1]
+    assert name == "gdn2_chunk_bwd"
+    assert [addr(a) for a in args[:16]] == [t.data_ptr() for t in ins + outs]
+    assert args[16:22] == (B, H, T, K, V, g.GDN2_BF16)
+    assert args[23] >= g.gdn2_chunk_bwd_workspace_bytes(B, H, T, K, V)
+    # optional S0, dS_T and dS0 travel as NULL
+    g.gdn2_chunk_bwd(*ins[:6], None, ins[7], None, *outs[:6], None)
+    _, args = rec.calls[-1]
+    assert args[6] is None and args[8] is None and args[15] is None
+
+
+def test_bwd_rejects_bad_arguments(rec):
+    B, T, H, K, V = 1, 8, 2, 64, 64
+    z = lambda *s, dt=torch.float32: torch.zeros(*s, dtype=dt)
+    tk, tv, st = (B, T, H, K), (B, T, H, V), (B, H, K, V)
+    good = [z(*tk), z(*tk), z(*tv), z(*tk), z(*tk), z(*tv), None, z(*tv), None,
+            z(*tk), z(*tk), z(*tv), z(*tk), z(*tk), z(*tv), None]
+    bad_shape = list(good)
+    bad_shape[9] = z(B, T, H, K + 1)
+    with pytest.raises(ValueError):
+        g.gdn2_chunk_bwd(*bad_shape)
+    bad_dtype = list(good)
+    bad_dtype[7] = z(*tv, dt=torch.bfloat16)      # dO must have the token dtype
+    with pytest.raises(TypeError):
+        g.gdn2_chunk_bwd(*bad_dtype)
+    bad_grad = list(good)
+    bad_grad[12] = z(*tk, dt=torch.bfloat16)      # gradients are fp32
+    with pytest.raises(TypeError):
+        g.gdn2_chunk_bwd(*bad_grad)
+    assert rec.calls == []
+
+
+def test_edges_marshalling(rec):
+    B, T, H, K, V = 1, 100, 2, 128, 128
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    q, k, b = bf(B, T, H, K), bf(B, T, H, K), bf(B, T, H, K)
+    v, w, o = bf(B, T, H, V), bf(B, T, H, V), bf(B, T, H, V)
+    a = torch.zeros(B, T, H, K)
+    weight, ST = torch.ones(V), torch.zeros(B, H, K, V)
+    g.gdn2_chunk_fwd_edges(q, k, v, a, b, w, None, weight, o, ST)
+    name, args = rec.calls[-1]
+    assert name == "gdn2_chunk_fwd_edges"
+    assert [addr(x) for x in args[:10]] == [q.data_ptr(), k.data_ptr(), v.data_ptr(), a.data_ptr(), b.data_ptr(),
+                                           w.data_ptr(), None, weight.data_ptr(), o.data_ptr(), ST.data_ptr()]
+    assert args[10:17] == (B, H, T, K, V, 64, g.GDN2_BF16)
+    assert args[18] >= g.gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, K, V)
+    with pytest.raises(ValueError):
+        g.gdn2_chunk_fwd_edges(q, k, v, a, b, w, None, torch.ones(V + 1), o, ST)
+    with pytest.raises(TypeError):
+        g.gdn2_chunk_fwd_edges(q, k, v, a.bfloat16(), b, w, None, weight, o, ST)
