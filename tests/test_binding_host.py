@@ -99,3 +99,44 @@ def test_edges_marshalling(rec):
         g.gdn2_chunk_fwd_edges(q, k, v, a, b, w, None, torch.ones(V + 1), o, ST)
     with pytest.raises(TypeError):
         g.gdn2_chunk_fwd_edges(q, k, v, a.bfloat16(), b, w, None, weight, o, ST)
+
+
+def test_fwd_and_decode_marshalling(rec):
+    B, T, H, K, V = 2, 65, 3, 128, 64
+    f = lambda *s, dt=torch.float32: torch.zeros(*s, dtype=dt)
+    q, k, b, a = f(B, T, H, K), f(B, T, H, K), f(B, T, H, K), f(B, T, H, K)
+    v, w, o = f(B, T, H, V), f(B, T, H, V), f(B, T, H, V)
+    S0, ST = f(B, H, K, V), f(B, H, K, V)
+    g.gdn2_chunk_fwd(q, k, v, a, b, w, S0, o, ST)
+    name, args = rec.calls[-1]
+    assert name == "gdn2_chunk_fwd"
+    assert [addr(x) for x in args[:9]] == [t.data_ptr() for t in (q, k, v, a, b, w, S0, o, ST)]
+    assert args[9:16] == (B, H, T, K, V, 64, g.GDN2_F32)
+    assert args[17] >= g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_F32)
+    qd, kd, bd, ad = f(B, H, K), f(B, H, K), f(B, H, K), f(B, H, K)
+    vd, wd, od = f(B, H, V), f(B, H, V), f(B, H, V)
+    g.gdn2_decode_step(qd, kd, vd, ad, bd, wd, S0, od)
+    name, args = rec.calls[-1]
+    assert name == "gdn2_decode_step"
+    assert [addr(x) for x in args[:8]] == [t.data_ptr() for t in (qd, kd, vd, ad, bd, wd, S0, od)]
+    assert args[8:13] == (B, H, K, V, g.GDN2_F32)
+
+
+def test_autograd_op_calls_backward_with_token_dtype_gradients(rec):
+    """gdn2_recurrence: the forward calls gdn2_chunk_fwd once; backward hands gdn2_chunk_bwd dO in the
+    token dtype and dS_T in fp32, fp32 gradient buffers, and the saved inputs."""
+    B, T, H, K, V = 1, 10, 2, 64, 64
+    leaf = lambda *s, dt=torch.bfloat16: torch.zeros(*s, dtype=dt).requires_grad_()
+    q, k, b, v, w = leaf(B, T, H, K), leaf(B, T, H, K), leaf(B, T, H, K), leaf(B, T, H, V), leaf(B, T, H, V)
+    a, S0 = leaf(B, T, H, K, dt=torch.float32), leaf(B, H, K, V, dt=torch.float32)
+    o, ST = g.gdn2_recurrence(q, k, v, a, b, w, S0)
+    assert [c[0] for c in rec.calls] == ["gdn2_chunk_fwd"]
+    (o.float().sum() + ST.sum()).backward()
+    name, args = rec.calls[-1]
+    assert name == "gdn2_chunk_bwd"
+    assert [addr(x) for x in args[:7]] == [t.data_ptr() for t in (q, k, v, a, b, w, S0)]
+    assert args[7] is not None and args[8] is not None and args[15] is not None
+    assert args[16:22] == (B, H, T, K, V, g.GDN2_BF16)
+    for t in (q, k, v, b, w):
+        assert t.grad is not None and t.grad.dtype == torch.bfloat16 and t.grad.shape == t.shape
+    assert a.grad.dtype == torch.float32 and S0.grad.shape == S0.shape
