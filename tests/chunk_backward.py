@@ -91,3 +91,73 @@ def chunked_grads(q, k, v, alpha, b, w, S0, dO, dST, C):
             out[i][sl] = g[i]
         dS = g[6]
     return tuple(out) + (dS,)
+
+
+def chunk_grads_framed(q, k, v, alpha, b, w, S, dO, dS_out):
+    """chunk_grads with every decay factor taken around the chunk's per-channel midpoint
+    m = (g_0 + g_{L-1}) / 2, as a tensor-core kernel must to keep its operands in range:
+    Ê_m = exp(g - m) ⊙ E, Q̂_m = exp(g - m) ⊙ Q, Ǩ_m = exp(m - g) ⊙ K (A, P unchanged), the state
+    in the frame Z = exp(m) ⊙ S, and dS entering as exp(g_{L-1} - m) ⊙ dS'.  The factors are then
+    bounded by exp(span / 2) instead of exp(span); the products above the diagonal of A and P, which
+    the masks drop, may still overflow and are selected away rather than multiplied by zero."""
+    L = q.shape[0]
+    g = np.cumsum(np.log(alpha), axis=0)
+    m = 0.5 * (g[0] + g[-1])
+    fm, fp = np.exp(g - m), np.exp(m - g)
+    e = b * k
+    Em, Qm, Km = fm * e, fm * q, fp * k
+    strict = np.tril(np.ones((L, L), dtype=bool), -1)
+    lower = np.tril(np.ones((L, L), dtype=bool), 0)
+    with np.errstate(over="ignore"):   # entries above the diagonal may overflow: they are not kept
+        A = np.where(strict, Em @ Km.T, 0.0)
+        P = np.where(lower, Qm @ Km.T, 0.0)
+    IA = np.eye(L) + A
+    Z = np.exp(m)[:, None] * S
+    Delta = np.linalg.solve(IA, w * v - Em @ Z)
+    S_out = np.exp(g[-1])[:, None] * S + np.exp(g[-1] - m)[:, None] * (Km.T @ Delta)
+
+    dSm = np.exp(g[-1] - m)[:, None] * dS_out
+    dDelta = P.T @ dO + Km @ dSm
+    dR = np.linalg.solve(IA.T, dDelta)
+    dA = np.where(strict, -(dR @ Delta.T), 0.0)
+    dP = np.where(lower, dO @ Delta.T, 0.0)
+    dEm = -dR @ Z.T + dA @ Km
+    dQm = dO @ Z.T + dP @ Km
+    dKm = dA.T @ Em + dP.T @ Qm + Delta @ dSm.T
+    dS_in = np.exp(m)[:, None] * (Qm.T @ dO - Em.T @ dR) + np.exp(g[-1])[:, None] * dS_out
+
+    dq = fm * dQm
+    de = fm * dEm
+    dk = fp * dKm + b * de
+    h = Qm * dQm + Em * dEm - Km * dKm       # frame-invariant: equals the unframed products
+    dlog = np.cumsum(h[::-1], axis=0)[::-1] + np.sum(dS_out * S_out, axis=1)[None, :]
+    return dq, dk, w * dR, dlog / alpha, k * de, v * dR, dS_in
+
+
+def chunked_grads_framed(q, k, v, alpha, b, w, S0, dO, dST, C):
+    """chunked_grads with chunk_grads_framed (the forward to each chunk's state is framed too)."""
+    T, K = q.shape
+    V = v.shape[1]
+    S = np.zeros((K, V)) if S0 is None else np.array(S0, dtype=np.float64)
+    starts = []
+    for t0 in range(0, T, C):
+        sl = slice(t0, min(T, t0 + C))
+        L = sl.stop - sl.start
+        starts.append(S)
+        g = np.cumsum(np.log(alpha[sl]), axis=0)
+        m = 0.5 * (g[0] + g[-1])
+        Em, Km = np.exp(g - m) * b[sl] * k[sl], np.exp(m - g) * k[sl]
+        with np.errstate(over="ignore"):
+            A = np.where(np.tril(np.ones((L, L), dtype=bool), -1), Em @ Km.T, 0.0)
+        Delta = np.linalg.solve(np.eye(L) + A, w[sl] * v[sl] - Em @ (np.exp(m)[:, None] * S))
+        S = np.exp(g[-1])[:, None] * S + np.exp(g[-1] - m)[:, None] * (Km.T @ Delta)
+    out = [np.zeros((T, K)), np.zeros((T, K)), np.zeros((T, V)), np.zeros((T, K)), np.zeros((T, K)),
+           np.zeros((T, V))]
+    dS = np.zeros((K, V)) if dST is None else np.array(dST, dtype=np.float64)
+    for ci in range(len(starts) - 1, -1, -1):
+        sl = slice(ci * C, min(T, ci * C + C))
+        gr = chunk_grads_framed(q[sl], k[sl], v[sl], alpha[sl], b[sl], w[sl], starts[ci], dO[sl], dS)
+        for i in range(6):
+            out[i][sl] = gr[i]
+        dS = gr[6]
+    return tuple(out) + (dS,)
