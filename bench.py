@@ -450,7 +450,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
     e2e_value = tokens_all / (e2e_ms * 1e-3)
 
-    extras = None if (args.no_extras or world > 1) else run_next_rows(g, torch, dev, stream, pw, pre_ms, clocks)
+    extras = None if (args.no_extras or world > 1) else run_next_rows(g, torch, dev, stream, pw, pre_ms, clocks,
+                                                                       with_cpu=not args.no_cpu_baseline)
 
     launches_per_step = (1 if path == 1 else 2) + 1
     out = {
@@ -483,7 +484,39 @@ def run_ours(args):
     return 0
 
 
-def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks):
+def oracle_next_rows_sample(wl):
+    """The fp64 oracles of the rows beyond the step, timed on one (b, h) chain of the workload with
+    one thread: the backward (oracle/backward.py) and the edge maps plus the recurrence.  Returns
+    {"backward": ..., "edges_prefill": ...} in tokens/s of the whole workload (B*T tokens over its
+    B*H chains run one after another)."""
+    import numpy as np
+    import threadpoolctl
+
+    import oracle
+    import synth
+    from oracle import backward as ob
+    chain = [(0, 0)]
+    scale = lambda sec: wl.B * wl.T / (sec * wl.B * wl.H)
+    x = {k: v[0].astype("float64") for k, v in synth.make_inputs(wl, chains=chain).items()}
+    dO, dST = synth.make_output_grads(wl, chains=chain)
+    with threadpoolctl.threadpool_limits(1):
+        t0 = time.perf_counter()
+        ob.chain_backward(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], None, dO[0].astype("float64"),
+                          dST[0].astype("float64"))
+        t_bwd = time.perf_counter() - t0
+        r = {k: v[0].astype("float64") for k, v in synth.make_raw_inputs(wl, chains=chain).items()}
+        t0 = time.perf_counter()
+        q, k, alpha, b, w = oracle.layer_edges(r["q"], r["k"], r["a"], r["b"], r["w"])
+        o, _ = oracle.chain_recurrence(q[None], k[None], r["v"][None], alpha[None], b[None], w[None], threads=1)
+        oracle.rms_norm(o, np.ones(wl.V))
+        t_edges = time.perf_counter() - t0
+    desc = f"one chain (b=0, h=0, T={wl.T}) of the {wl.B * wl.H}, one thread, scaled by the chain count"
+    return {"backward": {"value": scale(t_bwd), "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "edges_prefill": {"value": scale(t_edges), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                              "sample": desc}}
+
+
+def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=True):
     """Timings of the rows beyond the step (not part of `value`): the backward pass of the
     prefill workload and the prefill with the layer edges fused, both on that workload's sizes."""
     import synth
@@ -541,8 +574,15 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks):
              "plain_prefill_ms": plain_prefill_ms,
              "inputs": "raw q, k ~ N(0, 9), decay logit ~ N(1, 1) (alpha = exp(-softplus(a)): the plain "
                        "workload's alpha distribution), gate logits ~ N(0, 1)"}
-    return {"workload": f"{wl.name} (B{B} H{H} T{T} d_k=d_v={K}, bf16 tokens)", "backward": backward,
-            "edges_prefill": edges}
+    out = {"workload": f"{wl.name} (B{B} H{H} T{T} d_k=d_v={K}, bf16 tokens)", "backward": backward,
+           "edges_prefill": edges}
+    if with_cpu:
+        try:
+            cpu = oracle_next_rows_sample(wl)
+            backward["cpu_baseline"], edges["cpu_baseline"] = cpu["backward"], cpu["edges_prefill"]
+        except Exception as e:   # the CPU figures are context: never lose the GPU line over them
+            backward["cpu_baseline"] = edges["cpu_baseline"] = {"unavailable": repr(e)[:200]}
+    return out
 
 
 def main(argv=None):

@@ -102,3 +102,13 @@ def test_backward_accounting():
     assert bench.backward_flops(8, 4096, 16, 128, 128) == 21 * 8 * 4096 * 16 * 128 * 128 == 180388626432
     # 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz
     assert abs(bench.fp32_alu_peak_tflops(148, 1965.0) - 74.44992) < 1e-9
+
+
+def test_oracle_next_rows_sample_small():
+    import bench
+    import synth
+    wl = synth.Workload("nr", 2, 3, 96, 64, 64, "bf16", 1.0, seed=5)
+    out = bench.oracle_next_rows_sample(wl)
+    for key in ("backward", "edges_prefill"):
+        r = out[key]
+        assert r["kind"] == "oracle" and r["cores"] == 1 and r["unit"] == "tokens/s" and r["value"] > 0
