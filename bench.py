@@ -486,7 +486,8 @@ def run_ours(args):
 
 def oracle_next_rows_sample(wl):
     """The fp64 oracles of the rows beyond the step, timed on one (b, h) chain of the workload with
-    one thread: the backward (oracle/backward.py) and the edge maps plus the recurrence.  Returns
+    one thread: the backward (the C oracle's gdn2_oracle_backward) and the edge maps plus the
+    recurrence.  Returns
     {"backward": ..., "edges_prefill": ...} in tokens/s of the whole workload (B*T tokens over its
     B*H chains run one after another)."""
     import numpy as np
@@ -494,15 +495,15 @@ def oracle_next_rows_sample(wl):
 
     import oracle
     import synth
-    from oracle import backward as ob
     chain = [(0, 0)]
     scale = lambda sec: wl.B * wl.T / (sec * wl.B * wl.H)
     x = {k: v[0].astype("float64") for k, v in synth.make_inputs(wl, chains=chain).items()}
     dO, dST = synth.make_output_grads(wl, chains=chain)
+    r4 = lambda a: a.reshape(1, a.shape[0], 1, a.shape[-1])   # one chain as [B=1, T, H=1, d]
     with threadpoolctl.threadpool_limits(1):
         t0 = time.perf_counter()
-        ob.chain_backward(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], None, dO[0].astype("float64"),
-                          dST[0].astype("float64"))
+        oracle.recurrence_backward_c(*(r4(x[n]) for n in ("q", "k", "v", "alpha", "b", "w")), None,
+                                     r4(dO[0].astype("float64")), dST[0].astype("float64")[None, None], threads=1)
         t_bwd = time.perf_counter() - t0
         r = {k: v[0].astype("float64") for k, v in synth.make_raw_inputs(wl, chains=chain).items()}
         t0 = time.perf_counter()

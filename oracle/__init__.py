@@ -48,6 +48,8 @@ def _bind(lib):
     lib.gdn2_oracle_recurrence.restype = i
     lib.gdn2_oracle_decode_step.argtypes = [dp] * 8 + [i] * 5
     lib.gdn2_oracle_decode_step.restype = i
+    lib.gdn2_oracle_backward.argtypes = [dp] * 16 + [i] * 6
+    lib.gdn2_oracle_backward.restype = i
     return lib
 
 
@@ -118,6 +120,25 @@ def decode_step(q, k, v, alpha, b, w, S, threads=None, lib=None):
     if rc != 0:
         raise RuntimeError(f"oracle returned {rc}")
     return o
+
+
+def recurrence_backward_c(q, k, v, alpha, b, w, S0, dO, dST, threads=None, mem_budget=8 << 30, lib=None):
+    """The gradient of oracle/backward.py computed by the C oracle (gdn2_oracle_backward), chains in
+    parallel.  Same arguments and results ([B, T, H, d] tokens, [B, H, K, V] states, S0 / dST may be
+    None).  Each thread keeps its chain's T+1 states: threads are capped so that they fit mem_budget."""
+    lib = lib or load()
+    q, k, v, alpha, b, w, S0, dO, dST = map(_f64, (q, k, v, alpha, b, w, S0, dO, dST))
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    per_chain = 8 * (T + 1) * K * V
+    nt = max(1, min(_threads(threads), int(mem_budget // max(per_chain, 1))))
+    outs = [np.empty((B, T, H, K)), np.empty((B, T, H, K)), np.empty((B, T, H, V)), np.empty((B, T, H, K)),
+            np.empty((B, T, H, K)), np.empty((B, T, H, V)), np.empty((B, H, K, V))]
+    rc = lib.gdn2_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+                                  _ptr(dST), *(_ptr(o) for o in outs), B, H, T, K, V, nt)
+    if rc != 0:
+        raise RuntimeError(f"oracle backward returned {rc}")
+    return tuple(outs)
 
 
 def chain_recurrence(q, k, v, alpha, b, w, S0=None, threads=None):

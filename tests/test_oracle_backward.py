@@ -13,6 +13,8 @@ at the outputs.  Pins:
 3. closed form: alpha = 1 and b = 0 make the recurrence plain linear attention,
    o_t = S_0^T q_t + sum_{i<=t} (k_i . q_t) u_i, whose gradients are textbook
    sums over the causal mask.
+The C version of the same gradient (oracle/gdn2_oracle.c, gdn2_oracle_backward) passes the
+finite-difference pin and agrees with the numpy one to rounding.
 """
 import numpy as np
 import pytest
@@ -52,10 +54,14 @@ def directional_errors(rng, x, dO, dST, grads, eps=1e-5):
     return errs
 
 
+IMPLS = {"numpy": ob.recurrence_backward, "c": oracle.recurrence_backward_c}
+
+
+@pytest.mark.parametrize("impl", sorted(IMPLS))
 @pytest.mark.parametrize("T,K,V", [(1, 3, 2), (4, 3, 5), (9, 5, 4)])
-def test_finite_differences(rng, T, K, V):
+def test_finite_differences(rng, T, K, V, impl):
     x, dO, dST = problem(rng, 1, T, 2, K, V)
-    grads = ob.recurrence_backward(*(x[n] for n in NAMES), dO, dST)
+    grads = IMPLS[impl](*(x[n] for n in NAMES), dO, dST)
     errs = directional_errors(rng, x, dO, dST, grads)
     assert max(errs.values()) < 1e-8, errs
 
@@ -122,3 +128,23 @@ def test_empty_sequence(rng):
                             for n in NAMES[:-1]), x["S0"][0, 0], np.zeros((0, 2)), dST[0, 0])
     assert all(a.shape[0] == 0 for a in g[:6])
     np.testing.assert_array_equal(g[6], dST[0, 0])
+
+
+@pytest.mark.parametrize("B,T,H,K,V", [(1, 0, 2, 3, 2), (1, 1, 1, 4, 3), (2, 37, 3, 6, 5), (1, 70, 2, 16, 8)])
+@pytest.mark.parametrize("with_state", [True, False])
+def test_c_oracle_matches_numpy(rng, B, T, H, K, V, with_state):
+    """The C backward (oracle/gdn2_oracle.c) and the numpy one take the same steps in the same order:
+    they agree to rounding, threads or not."""
+    x, dO, dST = problem(rng, B, max(T, 1), H, K, V)
+    if T == 0:
+        x = {n: (a if n == "S0" else a[:, :0]) for n, a in x.items()}
+        dO = dO[:, :0]
+    if not with_state:
+        x["S0"] = None
+        dST = None
+    ref = ob.recurrence_backward(*(x[n] for n in NAMES), dO, dST)
+    for threads in (1, 3):
+        got = oracle.recurrence_backward_c(*(x[n] for n in NAMES), dO, dST, threads=threads)
+        for n, r, g in zip(("dq", "dk", "dv", "dalpha", "db", "dw", "dS0"), ref, got):
+            np.testing.assert_allclose(g, r, rtol=1e-12, atol=1e-13 * max(1.0, np.max(np.abs(r), initial=0.0)),
+                                       err_msg=n)

@@ -59,3 +59,34 @@ def test_unmutated_copy_passes(rng):
     errs = pins.directional_errors(rng, x, dO, dST, grads)
     assert max(errs.values()) < 1e-8, errs
     assert np.isfinite(list(errs.values())).all()
+
+
+# mistakes planted in the C version (oracle/gdn2_oracle.c, gdn2_oracle_backward)
+import oracle  # noqa: E402
+
+C_SRC = oracle._SRC
+C_MUTANTS = [
+    ("c_ddelta_uses_q", "dd[j] += G[(size_t)c * V + j] * kt[c];", "dd[j] += G[(size_t)c * V + j] * qt[c];"),
+    ("c_erase_sign", "de[c] = -s;", "de[c] = s;"),
+    ("c_erase_term_dropped", "dX[(size_t)c * V + j] = G[(size_t)c * V + j] - e * dd[j];",
+     "dX[(size_t)c * V + j] = G[(size_t)c * V + j];"),
+    ("c_decay_not_propagated", "G[(size_t)c * V + j] = at[c] * dX[(size_t)c * V + j];",
+     "G[(size_t)c * V + j] = dX[(size_t)c * V + j];"),
+    ("c_decay_reads_new_state", "s += dX[(size_t)c * V + j] * Sp[(size_t)c * V + j];",
+     "s += dX[(size_t)c * V + j] * Sn[(size_t)c * V + j];"),
+    ("c_readout_uses_previous_state", "s += Sn[(size_t)c * V + j] * gt[j];", "s += Sp[(size_t)c * V + j] * gt[j];"),
+    ("c_erase_gate_uses_b", "dbt[c] = kt[c] * de[c];", "dbt[c] = bt[c] * de[c];"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", C_MUTANTS, ids=[m[0] for m in C_MUTANTS])
+def test_c_mutant_is_caught(tmp_path, rng, name, old, new):
+    src = open(C_SRC).read()
+    assert src.count(old) == 1, name
+    path = tmp_path / f"oracle_{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.load(oracle.build(force=True, src=str(path), out=str(tmp_path / f"lib_{name}.so")))
+    x, dO, dST = pins.problem(rng, 1, 5, 1, 4, 3)
+    grads = oracle.recurrence_backward_c(*(x[n] for n in pins.NAMES), dO, dST, lib=lib)
+    errs = pins.directional_errors(rng, x, dO, dST, grads)
+    assert max(errs.values()) > 1e-4, f"{name} survived: {errs}"
