@@ -517,6 +517,55 @@ def oracle_next_rows_sample(wl):
                               "sample": desc}}
 
 
+def long_prefill_row(g, torch, dev, stream, timed, with_cpu):
+    """The prefill of few long chains (B1 H16 T65536, S0 given): segments in time, their state maps
+    composed along each chain (the transition scan), then every segment rerun from its start state."""
+    import numpy as np
+    import threadpoolctl
+
+    import oracle
+    import synth
+    lw = synth.WORKLOADS["prefill_long"]
+    x = synth.make_inputs(lw)
+    S0_np = synth.make_state(lw)
+    X = {k: torch.from_numpy(a).to(dev).to(torch.float32 if k == "alpha" else torch.bfloat16) for k, a in x.items()}
+    del x
+    S0 = torch.from_numpy(S0_np).to(dev)
+    B, T, H, K = X["q"].shape
+    V = X["v"].shape[-1]
+    o = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((B, H, K, V), device=dev)
+    ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_BF16), dev)
+    ms = timed(lambda: g.gdn2_chunk_fwd(X["q"], X["k"], X["v"], X["alpha"], X["b"], X["w"], S0, o, S_T,
+                                        workspace=ws, stream=stream))
+    if g.gdn2_workspace_status(ws) != 0:
+        raise RuntimeError("segmented prefill reported an internal error")
+    peaks = load_peaks()
+    nbytes = prefill_bytes(B, T, H, K, V, s0=True)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    row = {"workload": f"{lw.name} (B{B} H{H} T{T} d_k=d_v={K}, bf16 tokens, S0 given)", "ms": ms,
+           "tokens_per_s": B * T / (ms * 1e-3), "launches": 4,
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes, "traffic": None,
+                        "peak_src": peaks["src"],
+                        "note": "three passes over the segments plus the scan: about three times the bytes"}}
+    del X, o, S_T, ws, S0
+    if with_cpu:
+        try:
+            xs = synth.as_f64(synth.make_inputs(lw, chains=[(0, 0)]))
+            with threadpoolctl.threadpool_limits(1):
+                t0 = time.perf_counter()
+                oracle.chain_recurrence(*(xs[k] for k in ("q", "k", "v", "alpha", "b", "w")),
+                                        np.asarray(S0_np[0, :1], dtype=np.float64), threads=1)
+                sec = time.perf_counter() - t0
+            row["cpu_baseline"] = {"value": B * T / (sec * B * H), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                   "sample": f"one chain (b=0, h=0, T={T}) of the {B * H}, one thread, "
+                                             "scaled by the chain count"}
+        except Exception as e:
+            row["cpu_baseline"] = {"unavailable": repr(e)[:200]}
+    return row
+
+
 def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=True):
     """Timings of the rows beyond the step (not part of `value`): the backward pass of the
     prefill workload and the prefill with the layer edges fused, both on that workload's sizes."""
@@ -583,6 +632,10 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=
             backward["cpu_baseline"], edges["cpu_baseline"] = cpu["backward"], cpu["edges_prefill"]
         except Exception as e:   # the CPU figures are context: never lose the GPU line over them
             backward["cpu_baseline"] = edges["cpu_baseline"] = {"unavailable": repr(e)[:200]}
+    try:
+        out["segmented_prefill"] = long_prefill_row(g, torch, dev, stream, timed, with_cpu)
+    except Exception as e:   # likewise: this row must not cost the step's line
+        out["segmented_prefill"] = {"unavailable": repr(e)[:200]}
     return out
 
 
