@@ -148,3 +148,16 @@ def test_c_oracle_matches_numpy(rng, B, T, H, K, V, with_state):
         for n, r, g in zip(("dq", "dk", "dv", "dalpha", "db", "dw", "dS0"), ref, got):
             np.testing.assert_allclose(g, r, rtol=1e-12, atol=1e-13 * max(1.0, np.max(np.abs(r), initial=0.0)),
                                        err_msg=n)
+
+
+@pytest.mark.parametrize("impl", sorted(IMPLS))
+def test_gradients_linear_in_output_gradients(rng, impl):
+    """The gradient is a linear map of (dO, dS_T): grads(a*g1 + g2) = a*grads(g1) + grads(g2)."""
+    x, dO1, dST1 = problem(rng, 1, 11, 2, 5, 4)
+    _, dO2, dST2 = problem(rng, 1, 11, 2, 5, 4)
+    f = lambda dO, dST: IMPLS[impl](*(x[n] for n in NAMES), dO, dST)
+    a = 1.7
+    lhs = f(a * dO1 + dO2, a * dST1 + dST2)
+    g1, g2 = f(dO1, dST1), f(dO2, dST2)
+    for n, l, r1, r2 in zip(NAMES, lhs, g1, g2):
+        np.testing.assert_allclose(l, a * r1 + r2, rtol=1e-10, atol=1e-12, err_msg=n)
