@@ -33,16 +33,26 @@ def f32(x):
     return np.asarray(x, dtype=np.float32).astype(np.float64)
 
 
-def emulate_chain(q, k, v, alpha, b, w, S0, C=64):
+def ftz_exp2(x):
+    """2^x in fp32 with results below the smallest normal fp32 flushed to zero."""
+    y = f32(np.exp2(f32(x)))
+    return np.where(y < np.finfo(np.float32).tiny, 0.0, y)
+
+
+def emulate_chain(q, k, v, alpha, b, w, S0, C=64, combine_frame_factors=False):
     """One chain ([T, d] arrays holding the stored token values, alpha fp32; S0 [K, V] or None).
     Returns (o [T, V] as bf16 values, S_T [K, V] fp32 values).  Between chunks the state is the
     fp32 S the kernel forms as sPost * Z; per chunk sS scales its bf16 copy for G3 and sZ the fp32
     copy that G5 accumulates into (fast chunks: sS = sZ = 2^m, sPost = 2^(g_C - m); wide chunks:
-    sS = 1, sZ = 2^(g_C), sPost = 1)."""
+    sS = 1, sZ = 2^(g_C), sPost = 1).  combine_frame_factors=True instead takes sPost of one chunk
+    and sS / sZ of the next as ONE factor, 2 to the sum of their exponents, flushed to zero below
+    fp32's normal range as the GPU's ftz exp2 does: a design the kernel must not use, because at
+    long-context decay rates that sum falls below -126 while each exponent alone does not."""
     T, K = q.shape
     V = v.shape[1]
     S = np.zeros((K, V)) if S0 is None else f32(S0)
     o = np.zeros((T, V))
+    post = None   # combine_frame_factors: the previous chunk's sPost and accumulated Z
     tiny = np.finfo(np.float32).tiny
     for t0 in range(0, T, C):
         sl = slice(t0, min(T, t0 + C))
@@ -59,7 +69,7 @@ def emulate_chain(q, k, v, alpha, b, w, S0, C=64):
             dec = np.where(keep, np.exp2(np.where(keep, diff, 0.0)), 0.0)
             A = f32(np.einsum("rc,ic,ric->ri", b[sl] * k[sl], k[sl], dec)) * np.tril(np.ones((L, L)), -1)
             P = f32(np.einsum("rc,ic,ric->ri", q[sl], k[sl], dec))
-            sS, sZ, sPost = np.ones(K), f32(np.exp2(gC)), np.ones(K)
+            xS, xZ, xPost = np.zeros(K), gC, np.zeros(K)
         else:
             m = f32(0.5 * (g0 + gC))
             F = bf16(np.exp2(g - m))
@@ -69,16 +79,24 @@ def emulate_chain(q, k, v, alpha, b, w, S0, C=64):
                 Full = f32(np.vstack([Eh, Qh]) @ Kt.T)
             A = np.tril(Full[:L], -1)
             P = np.tril(Full[L:], 0)
-            sS = sZ = f32(np.exp2(m))
-            sPost = f32(np.exp2(gC - m))
+            xS = xZ = m
+            xPost = f32(gC - m)
+        sS, sZ, sPost = f32(np.exp2(xS)), f32(np.exp2(xZ)), f32(np.exp2(xPost))
         Tm = bf16(np.linalg.inv(np.eye(L) + A))
         Pb = bf16(P)
         Wp = f32(Tm @ Eh)
         Ut = f32(Tm @ U)
-        Zt = bf16(f32(sS[:, None] * S))
-        Z = f32(sZ[:, None] * S)
+        if post is None:
+            Zt = bf16(f32(sS[:, None] * S))
+            Z = f32(sZ[:, None] * S)
+        else:
+            x_prev, Z_prev = post
+            Zt = bf16(f32(ftz_exp2(x_prev + xS)[:, None] * Z_prev))
+            Z = f32(ftz_exp2(x_prev + xZ)[:, None] * Z_prev)
         Delta = bf16(f32(Ut - bf16(Wp) @ Zt))
         o[sl] = bf16(f32(Qh @ Zt + Pb @ Delta))
         Z = f32(Z + Kt.T @ Delta)
         S = f32(sPost[:, None] * Z)
+        if combine_frame_factors:
+            post = (xPost, Z)
     return o, S

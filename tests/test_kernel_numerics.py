@@ -40,3 +40,26 @@ def test_wide_span_chunks(rng):
     o_ref, S_ref = oracle.chain_recurrence(*(c[k][None] for k in ("q", "k", "v", "alpha", "b", "w")))
     o, S = emulate_chain(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], None)
     assert rel(o, o_ref[0]) <= 2e-2 and rel(S, S_ref[0]) <= 2e-2, (rel(o, o_ref[0]), rel(S, S_ref[0]))
+
+
+def test_combined_frame_factors_fail_on_long_context():
+    """Why the two frame factors between chunks are applied in turn: taken as one factor, 2 to the sum
+    of their exponents flushes to zero on the channels whose chunk spans reach the long workload's
+    typical ~150 log2, and the state those channels carry into the next chunk is lost (o errors of
+    0.13-0.18 here against 0.006-0.01 for the kernel's order)."""
+    wl0 = synth.WORKLOADS["prefill_long"]
+    wl = synth.Workload(wl0.name, wl0.B, wl0.H, 2048, wl0.K, wl0.V, wl0.dtype, wl0.alpha_mu, s0_std=wl0.s0_std,
+                        seed=wl0.seed)
+    errs = []
+    for h in range(4):
+        x = synth.make_inputs(wl, chains=[(0, h)])
+        S0 = synth.make_state(wl, chains=[(0, h)])
+        c = {k: a[0].astype(np.float64) for k, a in x.items()}
+        o_ref, _ = oracle.chain_recurrence(*(x[k].astype(np.float64) for k in ("q", "k", "v", "alpha", "b", "w")),
+                                           S0.astype(np.float64))
+        args = (c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], S0[0].astype(np.float64))
+        good, _ = emulate_chain(*args)
+        bad, _ = emulate_chain(*args, combine_frame_factors=True)
+        errs.append((rel(good, o_ref[0]), rel(bad, o_ref[0])))
+    assert all(g <= 2e-2 for g, _ in errs), errs
+    assert max(b for _, b in errs) > 2e-2, errs
