@@ -450,8 +450,12 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
     e2e_value = tokens_all / (e2e_ms * 1e-3)
 
-    extras = None if (args.no_extras or world > 1) else run_next_rows(g, torch, dev, stream, pw, pre_ms, clocks,
-                                                                       with_cpu=not args.no_cpu_baseline)
+    extras = None
+    if not (args.no_extras or world > 1):
+        try:   # timed after the step's region: a failure here must not cost the step's line
+            extras = run_next_rows(g, torch, dev, stream, pw, pre_ms, clocks, with_cpu=not args.no_cpu_baseline)
+        except Exception as e:
+            extras = {"unavailable": repr(e)[:200]}
 
     launches_per_step = (1 if path == 1 else 2) + 1
     out = {
@@ -619,7 +623,7 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=
     edge_ms = timed(lambda: g.gdn2_chunk_fwd_edges(R["q"], R["k"], R["v"], R["a"], R["b"], R["w"], None, weight, o,
                                                    S_T, workspace=ws, stream=stream))
     if g.gdn2_workspace_status(ws) != 0:
-        raise SystemExit("edge prefill kernel reported an internal error")
+        raise RuntimeError("edge prefill kernel reported an internal error")
     edges = {"ms": edge_ms, "tokens_per_s": B * T / (edge_ms * 1e-3), "launches": 1, "rmsnorm": True,
              "plain_prefill_ms": plain_prefill_ms,
              "inputs": "raw q, k ~ N(0, 9), decay logit ~ N(1, 1) (alpha = exp(-softplus(a)): the plain "

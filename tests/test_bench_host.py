@@ -7,6 +7,7 @@ import socket
 import pytest
 
 import bench
+from tests.test_binding_host import rec  # noqa: F401  (fixture)
 
 
 def test_prefill_bytes_per_token_head():
@@ -112,3 +113,52 @@ def test_oracle_next_rows_sample_small():
     for key in ("backward", "edges_prefill"):
         r = out[key]
         assert r["kind"] == "oracle" and r["cores"] == 1 and r["unit"] == "tokens/s" and r["value"] > 0
+
+
+def test_next_rows_run_on_cpu_through_the_binding(rec, monkeypatch):
+    """The bench's extra rows (backward, edge-fused prefill, segmented long prefill) driven on the CPU:
+    the library's compute calls are recorded instead of launched and CUDA events return 1 ms per 5 timed calls, so the
+    host code of each row (tensor shapes, binding arguments, accounting, the oracle baselines) runs
+    end to end and every row comes back complete."""
+    import types
+
+    import torch
+
+    import bench
+    import gated_delta_rule_96_b200 as g
+    import synth
+
+    class Event:
+        def __init__(self, enable_timing=False):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+
+    cuda = types.SimpleNamespace(Event=Event, synchronize=lambda dev=None: None,
+                                 get_device_properties=lambda dev: types.SimpleNamespace(multi_processor_count=148))
+
+    class FakeTorch:
+        def __getattr__(self, name):
+            return cuda if name == "cuda" else getattr(torch, name)
+
+    monkeypatch.setitem(synth.WORKLOADS, "prefill_long",
+                        synth.Workload("prefill_long", 1, 2, 200, 128, 128, "bf16", 1.0, s0_std=0.01, seed=7))
+    wl = synth.Workload("nr", 1, 2, 96, 128, 128, "bf16", 1.0, seed=5)
+    out = bench.run_next_rows(g, FakeTorch(), "cpu", None, wl, 0.5, {"sm_max_mhz": 1965.0})
+    names = [c[0] for c in rec.calls]
+    assert names.count("gdn2_chunk_bwd") == 7 and names.count("gdn2_chunk_fwd_edges") == 7
+    assert names.count("gdn2_chunk_fwd") == 7
+    bw, ed, sp = out["backward"], out["edges_prefill"], out["segmented_prefill"]
+    ms = 1.0 / 5
+    assert bw["ms"] == ms and bw["tokens_per_s"] == pytest.approx(96 / (ms * 1e-3))
+    assert bw["roofline"]["bound"] == "alu" and bw["roofline"]["flops_per_launch"] == bench.backward_flops(
+        1, 96, 2, 128, 128)
+    assert ed["ms"] == ms and ed["plain_prefill_ms"] == 0.5 and sp["ms"] == ms
+    assert sp["roofline"]["algorithmic_bytes_per_launch"] == bench.prefill_bytes(1, 200, 2, 128, 128, s0=True)
+    for row in (bw, ed, sp):
+        c = row["cpu_baseline"]
+        assert "unavailable" not in c and c["kind"] == "oracle" and c["value"] > 0, c
