@@ -161,3 +161,67 @@ def chunked_grads_framed(q, k, v, alpha, b, w, S0, dO, dST, C):
             out[i][sl] = gr[i]
         dS = gr[6]
     return tuple(out) + (dS,)
+
+
+def _f32(x):
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+def tf32(x):
+    """Round to tf32 (10 explicit mantissa bits, nearest, ties to even) through fp32; fp64 result."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0xFFF + ((u >> 13) & 1)) & 0xFFFFE000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def chunked_grads_rounded(q, k, v, alpha, b, w, S0, dO, dST, C, rnd):
+    """chunked_grads_framed with the number formats of a tensor-core kernel: every operand of a matrix
+    product rounded by `rnd` (bf16 or tf32), every product accumulated and every other quantity held
+    in fp32, the state carried in fp32, T = (I + A)^-1 formed in fp32.  Used to predict the accuracy
+    such a kernel can reach, not as a reference."""
+    mm = lambda x, y: _f32(rnd(x) @ rnd(y))
+    T, K = q.shape
+    V = v.shape[1]
+    strict = lambda L: np.tril(np.ones((L, L), dtype=bool), -1)
+    lower = lambda L: np.tril(np.ones((L, L), dtype=bool), 0)
+    S = np.zeros((K, V)) if S0 is None else _f32(S0)
+    saved = []
+    for t0 in range(0, T, C):   # forward: each chunk's operands and its incoming state
+        sl = slice(t0, min(T, t0 + C))
+        L = sl.stop - sl.start
+        g = _f32(np.cumsum(_f32(np.log(alpha[sl])), axis=0))
+        m = _f32(0.5 * (g[0] + g[-1]))
+        fm, fp = _f32(np.exp(g - m)), _f32(np.exp(m - g))
+        Em, Qm, Km = _f32(fm * _f32(b[sl] * k[sl])), _f32(fm * q[sl]), _f32(fp * k[sl])
+        with np.errstate(over="ignore", invalid="ignore"):
+            A = np.where(strict(L), mm(Em, Km.T), 0.0)
+            P = np.where(lower(L), mm(Qm, Km.T), 0.0)
+        Tm = _f32(np.linalg.inv(np.eye(L) + A))
+        Z = _f32(np.exp(m)[:, None] * S)
+        Delta = mm(Tm, _f32(_f32(w[sl] * v[sl]) - mm(Em, Z)))
+        S_out = _f32(_f32(np.exp(g[-1]))[:, None] * S + _f32(np.exp(g[-1] - m))[:, None] * mm(Km.T, Delta))
+        saved.append((sl, L, g, m, fm, fp, Em, Qm, Km, P, Tm, Z, Delta, S_out))
+        S = S_out
+    out = [np.zeros((T, K)), np.zeros((T, K)), np.zeros((T, V)), np.zeros((T, K)), np.zeros((T, K)),
+           np.zeros((T, V))]
+    dS = np.zeros((K, V)) if dST is None else _f32(dST)
+    for sl, L, g, m, fm, fp, Em, Qm, Km, P, Tm, Z, Delta, S_out in reversed(saved):
+        dSm = _f32(_f32(np.exp(g[-1] - m))[:, None] * dS)
+        dDelta = _f32(mm(P.T, dO[sl]) + mm(Km, dSm))
+        dR = mm(Tm.T, dDelta)
+        dA = np.where(strict(L), -mm(dR, Delta.T), 0.0)
+        dP = np.where(lower(L), mm(dO[sl], Delta.T), 0.0)
+        dEm = _f32(-mm(dR, Z.T) + mm(dA, Km))
+        dQm = _f32(mm(dO[sl], Z.T) + mm(dP, Km))
+        dKm = _f32(mm(dA.T, Em) + mm(dP.T, Qm) + mm(Delta, dSm.T))
+        h = _f32(Qm * dQm + Em * dEm - Km * dKm)
+        dlog = _f32(np.cumsum(h[::-1], axis=0)[::-1] + np.sum(dS * S_out, axis=1)[None, :])
+        de = _f32(fm * dEm)
+        out[0][sl] = _f32(fm * dQm)
+        out[1][sl] = _f32(fp * dKm + b[sl] * de)
+        out[2][sl] = _f32(w[sl] * dR)
+        out[3][sl] = _f32(dlog / alpha[sl])
+        out[4][sl] = _f32(k[sl] * de)
+        out[5][sl] = _f32(v[sl] * dR)
+        dS = _f32(_f32(np.exp(m))[:, None] * (mm(Qm.T, dO[sl]) - mm(Em.T, dR)) + _f32(np.exp(g[-1]))[:, None] * dS)
+    return tuple(out) + (dS,)

@@ -49,3 +49,41 @@ def test_framed_chunkwise_gradient(rng, log_alpha_range):
         with np.errstate(over="ignore", invalid="ignore"):
             plain = chunked_grads(q, k, v, alpha, b, w, S0, dO, dST, C)
         assert not all(np.all(np.isfinite(x)) for x in plain)
+
+
+@pytest.mark.parametrize("wl_name", ["prefill_1p3b", "prefill_slow_decay"])
+def test_rounded_chunkwise_gradient_accuracy(wl_name):
+    """What a tensor-core chunkwise backward can reach: the framed WY gradient with every product's
+    operands rounded to tf32 or bf16 (fp32 accumulation and state), on the bench workloads' value
+    distributions (d = 128, T = 512), against the fp64 step-wise oracle.  dq, dk, dv, db, dw, dS0 and
+    the gradient of log alpha stay within 2e-2 (bf16 operands) and 2e-3 (tf32); neither reaches the
+    1e-4 of the fp32 passes.  The gradient of alpha itself is d log alpha / alpha: at the bench
+    workload's smallest decays (alpha ~ 3e-3) that division lifts the absolute error of d log alpha
+    above 2e-2 of max |d alpha| with bf16 operands, so such a kernel would hand out d log alpha (what
+    a decay produced from a logit needs) or form d alpha in fp32.  Unrounded fp32 operands check the
+    emulation itself."""
+    import synth
+    from tests.chunk_backward import chunked_grads_rounded, tf32
+    from tests.kernel_numerics import bf16
+    wl0 = synth.WORKLOADS[wl_name]
+    wl = synth.Workload(wl0.name, 1, 2, 512, wl0.K, wl0.V, wl0.dtype, wl0.alpha_mu, gates=wl0.gates,
+                        seed=wl0.seed, alpha_scale=wl0.alpha_scale)
+    x = synth.as_f64(synth.make_inputs(wl, chains=[(0, 1)]))
+    dO, dST = synth.make_output_grads(wl, chains=[(0, 1)])
+    args = [x[n][0] for n in ("q", "k", "v", "alpha", "b", "w")]
+    alpha = args[3]
+    dO, dST = dO[0].astype(np.float64), dST[0].astype(np.float64)
+    ref = ob.chain_backward(*args, None, dO, dST)
+    rel = lambda a, r: np.max(np.abs(a - r)) / np.max(np.abs(r))
+    worst, dalpha = {}, {}
+    for name, rnd in (("fp32", lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)), ("tf32", tf32),
+                      ("bf16", bf16)):
+        got = chunked_grads_rounded(*args, None, dO, dST, 64, rnd)
+        errs = [rel(g, r) for i, (g, r) in enumerate(zip(got, ref)) if i != 3]
+        worst[name] = max(errs + [rel(got[3] * alpha, ref[3] * alpha)])
+        dalpha[name] = rel(got[3], ref[3])
+    assert worst["fp32"] <= 1e-5 and dalpha["fp32"] <= 1e-4, (worst, dalpha)
+    assert worst["tf32"] <= 2e-3, worst
+    assert worst["bf16"] <= 2e-2, worst
+    if wl_name == "prefill_1p3b":
+        assert dalpha["bf16"] > 2e-2, dalpha
