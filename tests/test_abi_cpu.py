@@ -180,3 +180,52 @@ def test_bwd_column_split_threshold():
     for chains, split in ((74, True), (75, False), (128, False), (1, True)):
         extra = a(4 * chains * T * K) if split else 0
         assert g.gdn2_chunk_bwd_workspace_bytes(1, chains, T, K, V) == base(chains) + extra, chains
+
+
+def call_edges(lib, B=1, H=1, T=100, K=128, V=128, C=64, dtype=1, ptr=FAKE, weight=None, ST=FAKE, ws=FAKE,
+               ws_bytes=1 << 30, o=FAKE):
+    return lib.gdn2_chunk_fwd_edges(ptr, ptr, ptr, ptr, ptr, ptr, None, weight, o, ST, B, H, T, K, V, C, dtype, ws,
+                                    ws_bytes, None)
+
+
+def test_chunk_fwd_edges_validation(lib):
+    assert call_edges(lib, T=-1) == -2
+    assert call_edges(lib, B=-1) == -2
+    assert call_edges(lib, dtype=9) == -3
+    assert call_edges(lib, ptr=None) == -1
+    assert call_edges(lib, o=None) == -1
+    assert call_edges(lib, ST=None) == -1
+    # the edges are fused into the tensor-core kernel only: bf16 tokens, d_k = d_v = 128, C = 64
+    assert call_edges(lib, K=64) == -4
+    assert call_edges(lib, V=64) == -4
+    assert call_edges(lib, C=32) == -4
+    assert call_edges(lib, dtype=0) == -4
+    assert call_edges(lib, ptr=P(0x10004)) == -7
+    assert call_edges(lib, weight=P(0x10008)) == -7
+    assert call_edges(lib, ws=None) == -5
+    assert call_edges(lib, ws=P(0x10004)) == -7
+    # the ring (128 KB per block) is part of the workspace: the plain prefill's size is too small
+    plain = g.gdn2_chunk_fwd_workspace_bytes(1, 1, 100, 128, 128, 64, g.GDN2_BF16)
+    assert plain < g.gdn2_chunk_fwd_edges_workspace_bytes(1, 1, 100, 128, 128)
+    assert call_edges(lib, ws_bytes=plain) == -5
+    assert call_edges(lib, B=0) == 0
+    assert call_edges(lib, H=0, weight=FAKE) == 0
+
+
+def call_noalloc(lib, B=1, H=1, T=8, K=128, V=128, C=64, dtype=1, ptr=FAKE, ST=FAKE, o=FAKE):
+    return lib.gdn2_chunk_fwd_noalloc(ptr, ptr, ptr, ptr, ptr, ptr, None, o, ST, B, H, T, K, V, C, dtype, None)
+
+
+def test_chunk_fwd_noalloc_validation(lib):
+    assert call_noalloc(lib, T=-1) == -2
+    assert call_noalloc(lib, H=-1) == -2
+    assert call_noalloc(lib, dtype=4) == -3
+    assert call_noalloc(lib, K=32) == -4
+    assert call_noalloc(lib, C=128) == -4
+    assert call_noalloc(lib, ST=None) == -1
+    assert call_noalloc(lib, ptr=None) == -1
+    assert call_noalloc(lib, o=None) == -1
+    assert call_noalloc(lib, ST=P(0x10004)) == -7
+    assert call_noalloc(lib, ptr=P(0x10002)) == -7
+    # more scratch than the fixed array holds is refused before any device call
+    assert call_noalloc(lib, B=64, H=64, T=1 << 16) == -9
