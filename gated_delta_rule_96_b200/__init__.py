@@ -111,6 +111,7 @@ def _stream(stream):
 
 
 def _check_cuda(*ts):
+    dev = None
     for t in ts:
         if t is None:
             continue
@@ -118,6 +119,33 @@ def _check_cuda(*ts):
             raise ValueError("all tensors must be CUDA tensors (no CPU path)")
         if not t.is_contiguous():
             raise ValueError("all tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"all tensors must be on one device ({dev} and {t.device} given)")
+
+
+def _check_dtypes(ref, named):
+    """Every (name, tensor) in `named` (None skipped) has the dtype of `ref`: the library reads all
+    token tensors of a call in one dtype, so a mismatch would read the wrong number of bytes."""
+    for name, t in named:
+        if t is not None and t.dtype != ref.dtype:
+            raise TypeError(f"{name} must have the token dtype {ref.dtype}, got {t.dtype}")
+
+
+def _check_shapes(named):
+    for name, t, shp in named:
+        if t is not None and tuple(t.shape) != tuple(shp):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shp)}")
+
+
+def _on_device(t):
+    """Make t's device current for the call: the library launches on the current device and on the
+    given (or that device's current) stream."""
+    import contextlib
+
+    import torch
+    return torch.cuda.device(t.device) if getattr(t, "is_cuda", False) else contextlib.nullcontext()
 
 
 def new_workspace(nbytes: int, device=None):
@@ -138,20 +166,17 @@ def gdn2_chunk_fwd(q, k, v, alpha, b, w, S0, o, S_T, C=64, workspace=None, strea
     dt = _dtype_code(q)
     if alpha.dtype != torch.float32 or S_T.dtype != torch.float32 or (S0 is not None and S0.dtype != torch.float32):
         raise TypeError("alpha and the states must be float32")
-    for name, t in (("k", k), ("b", b), ("v", v), ("w", w), ("o", o)):
-        if t.dtype != q.dtype:
-            raise TypeError(f"{name} must have the dtype of q ({q.dtype})")
-    for name, t, shp in (("k", k, (B, T, H, K)), ("b", b, (B, T, H, K)), ("alpha", alpha, (B, T, H, K)),
-                         ("w", w, (B, T, H, V)), ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)),
-                         ("S0", S0, (B, H, K, V))):
-        if t is not None and tuple(t.shape) != shp:
-            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    _check_dtypes(q, (("k", k), ("b", b), ("v", v), ("w", w), ("o", o)))
+    _check_shapes((("k", k, (B, T, H, K)), ("b", b, (B, T, H, K)), ("alpha", alpha, (B, T, H, K)),
+                   ("w", w, (B, T, H, V)), ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)),
+                   ("S0", S0, (B, H, K, V))))
     need = gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, C, dt)
     if workspace is None:
         workspace = new_workspace(need, q.device)
-    rc = load_library().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
-                                       _ptr(o), _ptr(S_T), B, H, T, K, V, C, dt, _ptr(workspace),
-                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    with _on_device(q):
+        rc = load_library().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                           _ptr(o), _ptr(S_T), B, H, T, K, V, C, dt, _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_fwd")
 
@@ -173,19 +198,19 @@ def gdn2_chunk_fwd_edges(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o_weigh
     for name, t in (("a_logit", a_logit), ("S_T", S_T), ("S0", S0), ("o_weight", o_weight)):
         if t is not None and t.dtype != torch.float32:
             raise TypeError(f"{name} must be float32")
-    for name, t, shp in (("k_raw", k_raw, (B, T, H, K)), ("b_logit", b_logit, (B, T, H, K)),
-                         ("a_logit", a_logit, (B, T, H, K)), ("w_logit", w_logit, (B, T, H, V)),
-                         ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)), ("S0", S0, (B, H, K, V)),
-                         ("o_weight", o_weight, (V,))):
-        if t is not None and tuple(t.shape) != shp:
-            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    _check_dtypes(q_raw, (("k_raw", k_raw), ("v", v), ("b_logit", b_logit), ("w_logit", w_logit), ("o", o)))
+    _check_shapes((("k_raw", k_raw, (B, T, H, K)), ("b_logit", b_logit, (B, T, H, K)),
+                   ("a_logit", a_logit, (B, T, H, K)), ("v", v, (B, T, H, V)), ("w_logit", w_logit, (B, T, H, V)),
+                   ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)), ("S0", S0, (B, H, K, V)),
+                   ("o_weight", o_weight, (V,))))
     need = gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, K, V, C)
     if workspace is None:
         workspace = new_workspace(need, q_raw.device)
-    rc = load_library().gdn2_chunk_fwd_edges(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_logit), _ptr(b_logit),
-                                             _ptr(w_logit), _ptr(S0), _ptr(o_weight), _ptr(o), _ptr(S_T), B, H, T,
-                                             K, V, C, dt, _ptr(workspace),
-                                             workspace.numel() * workspace.element_size(), _stream(stream))
+    with _on_device(q_raw):
+        rc = load_library().gdn2_chunk_fwd_edges(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_logit), _ptr(b_logit),
+                                                 _ptr(w_logit), _ptr(S0), _ptr(o_weight), _ptr(o), _ptr(S_T), B, H,
+                                                 T, K, V, C, dt, _ptr(workspace),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_fwd_edges")
 
@@ -207,19 +232,18 @@ def gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, d
                     ("dalpha", dalpha), ("db", db), ("dw", dw), ("dS0", dS0)):
         if t is not None and t.dtype != torch.float32:
             raise TypeError(f"{name} must be float32")
-    if dO.dtype != q.dtype:
-        raise TypeError("dO must have the token dtype")
+    _check_dtypes(q, (("k", k), ("v", v), ("b", b), ("w", w), ("dO", dO)))
     tk, tv, st = (B, T, H, K), (B, T, H, V), (B, H, K, V)
-    for name, t, shp in (("k", k, tk), ("b", b, tk), ("alpha", alpha, tk), ("v", v, tv), ("w", w, tv),
-                         ("dO", dO, tv), ("S0", S0, st), ("dS_T", dS_T, st), ("dq", dq, tk), ("dk", dk, tk),
-                         ("dalpha", dalpha, tk), ("db", db, tk), ("dv", dv, tv), ("dw", dw, tv), ("dS0", dS0, st)):
-        if t is not None and tuple(t.shape) != shp:
-            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    _check_shapes((("k", k, tk), ("b", b, tk), ("alpha", alpha, tk), ("v", v, tv), ("w", w, tv),
+                   ("dO", dO, tv), ("S0", S0, st), ("dS_T", dS_T, st), ("dq", dq, tk), ("dk", dk, tk),
+                   ("dalpha", dalpha, tk), ("db", db, tk), ("dv", dv, tv), ("dw", dw, tv), ("dS0", dS0, st)))
     if workspace is None:
         workspace = new_workspace(max(gdn2_chunk_bwd_workspace_bytes(B, H, T, K, V), 256), q.device)
-    rc = load_library().gdn2_chunk_bwd(*(_ptr(t) for t in (q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha,
-                                                           db, dw, dS0)), B, H, T, K, V, dt, _ptr(workspace),
-                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    with _on_device(q):
+        rc = load_library().gdn2_chunk_bwd(*(_ptr(t) for t in (q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv,
+                                                               dalpha, db, dw, dS0)), B, H, T, K, V, dt,
+                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_bwd")
 
@@ -228,12 +252,21 @@ def gdn2_chunk_fwd_noalloc(q, k, v, alpha, b, w, S0, o, S_T, C=64, stream=None) 
     """Prefill for callers that cannot allocate device memory: no workspace argument; the
     library's fixed scratch array is used instead (see include/gdn2.h for the size limit
     and for the rule that overlapping calls race on the shared array)."""
+    import torch
     _check_cuda(q, k, v, alpha, b, w, S0, o, S_T)
     B, T, H, K = q.shape
     V = v.shape[-1]
-    rc = load_library().gdn2_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
-                                               _ptr(S0), _ptr(o), _ptr(S_T), B, H, T, K, V, C, _dtype_code(q),
-                                               _stream(stream))
+    dt = _dtype_code(q)
+    if alpha.dtype != torch.float32 or S_T.dtype != torch.float32 or (S0 is not None and S0.dtype != torch.float32):
+        raise TypeError("alpha and the states must be float32")
+    _check_dtypes(q, (("k", k), ("b", b), ("v", v), ("w", w), ("o", o)))
+    _check_shapes((("k", k, (B, T, H, K)), ("b", b, (B, T, H, K)), ("alpha", alpha, (B, T, H, K)),
+                   ("w", w, (B, T, H, V)), ("o", o, (B, T, H, V)), ("S_T", S_T, (B, H, K, V)),
+                   ("S0", S0, (B, H, K, V))))
+    with _on_device(q):
+        rc = load_library().gdn2_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                                                   _ptr(S0), _ptr(o), _ptr(S_T), B, H, T, K, V, C, dt,
+                                                   _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_fwd_noalloc")
 
@@ -247,18 +280,21 @@ def gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=None) -> None:
     dt = _dtype_code(q)
     if alpha.dtype != torch.float32 or S.dtype != torch.float32:
         raise TypeError("alpha and S must be float32")
-    if tuple(S.shape) != (B, H, K, V) or tuple(o.shape) != (B, H, V):
-        raise ValueError("S must be [B,H,d_k,d_v] and o [B,H,d_v]")
-    rc = load_library().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S),
-                                         _ptr(o), B, H, K, V, dt, _stream(stream))
+    _check_dtypes(q, (("k", k), ("b", b), ("v", v), ("w", w), ("o", o)))
+    _check_shapes((("k", k, (B, H, K)), ("b", b, (B, H, K)), ("alpha", alpha, (B, H, K)), ("v", v, (B, H, V)),
+                   ("w", w, (B, H, V)), ("o", o, (B, H, V)), ("S", S, (B, H, K, V))))
+    with _on_device(q):
+        rc = load_library().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S),
+                                             _ptr(o), B, H, K, V, dt, _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_decode_step")
 
 
 def gdn2_workspace_status(workspace, clear=False, stream=None) -> int:
     out = ctypes.c_int(0)
-    rc = load_library().gdn2_workspace_status(_ptr(workspace), 1 if clear else 0, ctypes.byref(out),
-                                              _stream(stream))
+    with _on_device(workspace):
+        rc = load_library().gdn2_workspace_status(_ptr(workspace), 1 if clear else 0, ctypes.byref(out),
+                                                  _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_workspace_status")
     return out.value

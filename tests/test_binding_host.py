@@ -140,3 +140,61 @@ def test_autograd_op_calls_backward_with_token_dtype_gradients(rec):
     for t in (q, k, v, b, w):
         assert t.grad is not None and t.grad.dtype == torch.bfloat16 and t.grad.shape == t.shape
     assert a.grad.dtype == torch.float32 and S0.grad.shape == S0.shape
+
+
+def test_token_dtype_mismatch_refused_before_any_call(rec):
+    """The library reads every token tensor of a call in q's dtype: a tensor of another dtype would be
+    read with the wrong element size, so the binding refuses it for every entry point."""
+    B, T, H, K, V = 1, 8, 2, 64, 64
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    f = lambda *s: torch.zeros(*s)
+    tk, tv, st = (B, T, H, K), (B, T, H, V), (B, H, K, V)
+    with pytest.raises(TypeError):     # v fp32 with bf16 q
+        g.gdn2_chunk_fwd(bf(*tk), bf(*tk), f(*tv), f(*tk), bf(*tk), bf(*tv), None, bf(*tv), f(*st))
+    with pytest.raises(TypeError):
+        g.gdn2_chunk_fwd_noalloc(bf(*tk), f(*tk), bf(*tv), f(*tk), bf(*tk), bf(*tv), None, bf(*tv), f(*st))
+    with pytest.raises(TypeError):     # w_logit fp32 with bf16 q_raw
+        g.gdn2_chunk_fwd_edges(bf(*tk), bf(*tk), bf(*tv), f(*tk), bf(*tk), f(*tv), None, None, bf(*tv), f(*st))
+    with pytest.raises(TypeError):     # k bf16 with fp32 q
+        g.gdn2_chunk_bwd(f(*tk), bf(*tk), f(*tv), f(*tk), f(*tk), f(*tv), None, f(*tv), None,
+                         f(*tk), f(*tk), f(*tv), f(*tk), f(*tk), f(*tv), None)
+    with pytest.raises(TypeError):     # decode: b fp32 with bf16 q
+        g.gdn2_decode_step(bf(B, H, K), bf(B, H, K), bf(B, H, V), f(B, H, K), f(B, H, K), bf(B, H, V), f(*st),
+                           bf(B, H, V))
+    assert rec.calls == []
+
+
+def test_shape_mismatch_refused_before_any_call(rec):
+    B, T, H, K, V = 1, 8, 2, 64, 64
+    f = lambda *s: torch.zeros(*s)
+    tk, tv, st = (B, T, H, K), (B, T, H, V), (B, H, K, V)
+    with pytest.raises(ValueError):    # decode: k of another head count
+        g.gdn2_decode_step(f(B, H, K), f(B, H + 1, K), f(B, H, V), f(B, H, K), f(B, H, K), f(B, H, V), f(*st),
+                           f(B, H, V))
+    with pytest.raises(ValueError):    # no-alloc prefill: alpha one token short
+        g.gdn2_chunk_fwd_noalloc(f(*tk), f(*tk), f(*tv), f(B, T - 1, H, K), f(*tk), f(*tv), None, f(*tv), f(*st))
+    with pytest.raises(ValueError):    # edges: v with another time length
+        g.gdn2_chunk_fwd_edges(f(*tk).bfloat16(), f(*tk).bfloat16(), f(B, T + 1, H, V).bfloat16(), f(*tk),
+                               f(*tk).bfloat16(), f(*tv).bfloat16(), None, None, f(*tv).bfloat16(), f(*st))
+    assert rec.calls == []
+
+
+class FakeTensor:
+    def __init__(self, device, is_cuda=True, contiguous=True):
+        self.device, self.is_cuda, self._c = device, is_cuda, contiguous
+
+    def is_contiguous(self):
+        return self._c
+
+
+def test_check_cuda_rules():
+    """CUDA tensors only, contiguous, all on one device (a kernel launched on one device must not be
+    handed another device's pointers)."""
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    g._check_cuda(FakeTensor(d0), None, FakeTensor(d0))
+    with pytest.raises(ValueError, match="one device"):
+        g._check_cuda(FakeTensor(d0), FakeTensor(d1))
+    with pytest.raises(ValueError, match="CUDA"):
+        g._check_cuda(FakeTensor(torch.device("cpu"), is_cuda=False))
+    with pytest.raises(ValueError, match="contiguous"):
+        g._check_cuda(FakeTensor(d0, contiguous=False))
