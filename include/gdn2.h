@@ -18,6 +18,8 @@
  *   - All tensor pointers are DEVICE pointers to contiguous, row-major buffers, each
  *     16-byte aligned.  The caller owns every buffer; the library allocates nothing
  *     and keeps no state between calls.
+ *   - Kernels launch on the calling thread's current CUDA device, which must own every
+ *     pointer of the call (and `stream`, if given).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
  *     legacy default stream).  The return value reports argument checking and launch
  *     errors only; device-side errors are read with gdn2_workspace_status().
