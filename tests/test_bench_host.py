@@ -162,3 +162,27 @@ def test_next_rows_run_on_cpu_through_the_binding(rec, monkeypatch):
     for row in (bw, ed, sp):
         c = row["cpu_baseline"]
         assert "unavailable" not in c and c["kind"] == "oracle" and c["value"] > 0, c
+
+
+def test_clock_sampler_without_nvidia_smi(monkeypatch):
+    """No nvidia-smi (or no GPU): the sampler reports 'unavailable' instead of failing the run."""
+    monkeypatch.setenv("PATH", "/nonexistent")
+    with bench.ClockSampler(0) as c:
+        pass
+    s = c.summary()
+    assert s["reasons"] == ["unavailable"] and s["samples"] == 0
+
+
+def test_clock_sampler_summary(tmp_path):
+    """Median SM clock under load, the max clock, and the throttle reasons seen Active."""
+    p = tmp_path / "clocks.csv"
+    p.write_text("0, 1965, 1965, 700.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+                 "0, 1800, 1965, 1000.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+                 "0, 1900, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+                 "garbage line\n")
+    c = bench.ClockSampler(0)
+    c.path = str(p)
+    s = c.summary()
+    assert s["sm_mhz"] == 1900 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 1000.1
+    assert not p.exists()
