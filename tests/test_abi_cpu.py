@@ -229,3 +229,18 @@ def test_chunk_fwd_noalloc_validation(lib):
     assert call_noalloc(lib, ptr=P(0x10002)) == -7
     # more scratch than the fixed array holds is refused before any device call
     assert call_noalloc(lib, B=64, H=64, T=1 << 16) == -9
+
+
+def test_library_is_standalone():
+    """libgdn2.so depends on no Python or torch library (the CUDA runtime is linked statically): the
+    boundary is plain C, usable from any host program."""
+    import shutil
+    import subprocess
+    readelf = shutil.which("readelf")
+    if readelf is None:
+        pytest.skip("readelf not available")
+    out = subprocess.run([readelf, "-d", g.library_path()], capture_output=True, text=True, check=True).stdout
+    needed = re.findall(r"\(NEEDED\).*\[(.+?)\]", out)
+    assert needed, out
+    for lib_name in needed:
+        assert not re.search(r"torch|c10|python|cudart", lib_name), lib_name
