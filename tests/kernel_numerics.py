@@ -39,7 +39,7 @@ def ftz_exp2(x):
     return np.where(y < np.finfo(np.float32).tiny, 0.0, y)
 
 
-def emulate_chain(q, k, v, alpha, b, w, S0, C=64, combine_frame_factors=False):
+def emulate_chain(q, k, v, alpha, b, w, S0, C=64, combine_frame_factors=False, stored_u_bf16=False):
     """One chain ([T, d] arrays holding the stored token values, alpha fp32; S0 [K, V] or None).
     Returns (o [T, V] as bf16 values, S_T [K, V] fp32 values).  Between chunks the state is the
     fp32 S the kernel forms as sPost * Z; per chunk sS scales its bf16 copy for G3 and sZ the fp32
@@ -47,7 +47,10 @@ def emulate_chain(q, k, v, alpha, b, w, S0, C=64, combine_frame_factors=False):
     sS = 1, sZ = 2^(g_C), sPost = 1).  combine_frame_factors=True instead takes sPost of one chunk
     and sS / sZ of the next as ONE factor, 2 to the sum of their exponents, flushed to zero below
     fp32's normal range as the GPU's ftz exp2 does: a design the kernel must not use, because at
-    long-context decay rates that sum falls below -126 while each exponent alone does not."""
+    long-context decay rates that sum falls below -126 while each exponent alone does not.
+    stored_u_bf16=True rounds Ũ = T U to bf16 as well, as a prefill split into a parallel build/solve
+    kernel and a state walk would when it passes Ũ through HBM in bf16 (the fused kernel keeps it
+    in fp32 in TMEM)."""
     T, K = q.shape
     V = v.shape[1]
     S = np.zeros((K, V)) if S0 is None else f32(S0)
@@ -86,6 +89,8 @@ def emulate_chain(q, k, v, alpha, b, w, S0, C=64, combine_frame_factors=False):
         Pb = bf16(P)
         Wp = f32(Tm @ Eh)
         Ut = f32(Tm @ U)
+        if stored_u_bf16:
+            Ut = bf16(Ut)
         if post is None:
             Zt = bf16(f32(sS[:, None] * S))
             Z = f32(sZ[:, None] * S)

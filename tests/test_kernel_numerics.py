@@ -63,3 +63,18 @@ def test_combined_frame_factors_fail_on_long_context():
         errs.append((rel(good, o_ref[0]), rel(bad, o_ref[0])))
     assert all(g <= 2e-2 for g, _ in errs), errs
     assert max(b for _, b in errs) > 2e-2, errs
+
+
+def test_bf16_intermediates_of_a_split_prefill():
+    """A prefill split into a parallel build/solve kernel and a state walk would pass W', Ũ, Q̂, K̃ and P
+    through HBM; in bf16, Ũ is the one operand the fused kernel keeps wider (fp32 in TMEM).  Rounding
+    it too keeps the bench workload's o within the bf16 bar."""
+    wl0 = synth.WORKLOADS["prefill_1p3b"]
+    wl = synth.Workload(wl0.name, 1, 4, 1024, wl0.K, wl0.V, wl0.dtype, wl0.alpha_mu, seed=wl0.seed)
+    for h in range(2):
+        x = synth.make_inputs(wl, chains=[(0, h)])
+        c = {k: a[0].astype(np.float64) for k, a in x.items()}
+        o_ref, S_ref = oracle.chain_recurrence(*(x[k].astype(np.float64) for k in ("q", "k", "v", "alpha", "b", "w")))
+        args = (c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], None)
+        o, S = emulate_chain(*args, stored_u_bf16=True)
+        assert rel(o, o_ref[0]) <= 2e-2 and rel(S, S_ref[0]) <= 2e-2, (rel(o, o_ref[0]), rel(S, S_ref[0]))
