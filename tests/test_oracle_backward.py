@@ -161,3 +161,22 @@ def test_gradients_linear_in_output_gradients(rng, impl):
     g1, g2 = f(dO1, dST1), f(dO2, dST2)
     for n, l, r1, r2 in zip(NAMES, lhs, g1, g2):
         np.testing.assert_allclose(l, a * r1 + r2, rtol=1e-10, atol=1e-12, err_msg=n)
+
+
+@pytest.mark.parametrize("impl", sorted(IMPLS))
+@pytest.mark.parametrize("T,K,V", [(1, 3, 2), (9, 5, 4), (30, 4, 6)])
+def test_euler_identities(rng, impl, T, K, V):
+    """Homogeneity pins.  L = sum dO.o + sum dS_T⊙S_T is linear in (S0, v) jointly and, through the
+    readout alone, in q; by Euler's theorem for degree-1 functions
+        <dS0, S0> + <dv, v> = <dS0, S0> + <dw, w> = L      and      <dq, q> = sum dO.o,
+    and dq does not depend on dS_T (q never feeds the state)."""
+    x, dO, dST = problem(rng, 1, T, 2, K, V)
+    g = IMPLS[impl](*(x[n] for n in NAMES), dO, dST)
+    o, ST = oracle.recurrence(*(x[n] for n in NAMES), threads=1)
+    L_o, L = float(np.sum(dO * o)), float(np.sum(dO * o) + np.sum(dST * ST))
+    for grad, name in ((g[2], "v"), (g[5], "w")):   # u = w ⊙ v is linear in each of them
+        euler = float(np.sum(g[6] * x["S0"]) + np.sum(grad * x[name]))
+        assert abs(euler - L) <= 1e-11 * (1 + abs(L)), (name, euler, L)
+    assert abs(float(np.sum(g[0] * x["q"])) - L_o) <= 1e-11 * (1 + abs(L_o))
+    g0 = IMPLS[impl](*(x[n] for n in NAMES), dO, np.zeros_like(dST))
+    np.testing.assert_allclose(g0[0], g[0], rtol=1e-13, atol=1e-14)
