@@ -231,8 +231,9 @@ def oracle_sample_time(prefill_wl, decode_wl, budget_s=12.0, max_chains=None):
 
     Prefill: whole (b, h) chains of the prefill workload (full T), as many as fit the
     budget (at least 2*cores, capped by the workload); decode: one decode step of a
-    slice of the heads.  Returns (seconds for a FULL step extrapolated by work share,
-    description, threads used)."""
+    slice of the heads.  Returns a dict: the seconds actually measured, the work share
+    of one full step that the sample covers, the seconds of a FULL step extrapolated by
+    that share, a description and the threads used."""
     import numpy as np
 
     import oracle
@@ -268,8 +269,12 @@ def oracle_sample_time(prefill_wl, decode_wl, budget_s=12.0, max_chains=None):
     t_dec = time.perf_counter() - t0
     full_dec = t_dec * (decode_wl.B * decode_wl.H) / len(heads)
     desc = (f"fp64 oracle on {n} of {len(all_chains)} prefill chains (full T={T}) and one decode step of "
-            f"{len(heads)} of {decode_wl.B * decode_wl.H} heads, scaled to one full step by work share")
-    return full_pre + full_dec, desc, cores
+            f"{len(heads)} of {decode_wl.B * decode_wl.H} heads")
+    # tokens of the metric covered by the sample: a chain is 1/H of a prefill token row, a decode
+    # head 1/H of a decode token
+    tokens = n * T / H + len(heads) / decode_wl.H
+    return {"measured_s": t_pre + t_dec, "tokens": tokens, "full_step_s": full_pre + full_dec, "desc": desc,
+            "cores": cores}
 
 
 def bench_config(world):
@@ -287,27 +292,34 @@ def bench_config(world):
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
+    """The oracle arm: each step times the fp64 oracle on a bounded sample of the step's work
+    (whole prefill chains and a slice of the decode heads).  `ms_per_step` is the time of the
+    sampled work actually run; `value` is the tokens that sample covers per second; the time a
+    full step would take at that rate is reported on its own under `full_step_ms_extrapolated`."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import synth
     pw, dw = synth.WORKLOADS[PREFILL], synth.WORKLOADS[DECODE]
-    tokens_step = pw.B * pw.T + dw.B
     cores = os.cpu_count() or 1
-    times, desc = [], ""
+    meas, toks, full, desc = [], [], [], ""
     for i in range(args.warmup + args.steps):
-        t_full, desc, cores = oracle_sample_time(pw, dw, budget_s=4.0, max_chains=max(2, cores))
+        r = oracle_sample_time(pw, dw, budget_s=4.0, max_chains=max(2, cores))
+        desc, cores = r["desc"], r["cores"]
         if i >= args.warmup:
-            times.append(t_full)
-    sec = statistics.mean(times)
-    value = tokens_step / sec
+            meas.append(r["measured_s"])
+            toks.append(r["tokens"])
+            full.append(r["full_step_s"])
+    sec = statistics.mean(meas)
+    value = sum(toks) / sum(meas)
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": bench_config(args.gpus),
+        "full_step_ms_extrapolated": statistics.mean(full) * 1e3,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": desc + " (each step)"},
+                         "sample": desc + " per step; ms_per_step is that sample's time"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -402,6 +414,27 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     value = tokens_all / (ms_per_step * 1e-3)
 
+    # ---- steady state: the same step back to back for >= 1.5 s, clocks sampled throughout
+    steady = None
+    if args.steady_s > 0:
+        n_steady = max(args.steps, int(args.steady_s * 1e3 / max(ms_per_step, 1e-3)) + 1)
+        s0_, s1_ = ev(), ev()
+        barrier(pg)
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clk2:
+            s0_.record(stream)
+            for _ in range(n_steady):
+                prefill()
+                decode()
+            s1_.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier(pg)
+        st_ms = max_over_ranks(s0_.elapsed_time(s1_), pg, dev) / n_steady
+        steady = {"steps": n_steady, "ms_per_step": st_ms, "value": tokens_all / (st_ms * 1e-3),
+                  "timed_s": st_ms * n_steady * 1e-3, "clocks": clk2.summary()}
+        if g.gdn2_workspace_status(ws) != 0:
+            raise SystemExit("prefill kernel reported an internal error in the steady-state region")
+
     peaks = load_peaks()
     pb = prefill_bytes(B, T, H, K, V)
     db = decode_bytes(dw.B, dw.H, dw.K, dw.V)
@@ -478,14 +511,16 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
+    if steady is not None:
+        out["steady"] = steady
     if extras is not None:
         out["next_rows"] = extras
     if parts != {"prefill", "decode"}:
         out["config"]["parts_only"] = sorted(parts)   # profiling run: not a bench line
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sec, desc, cores = oracle_sample_time(pw, dw)
-        out["cpu_baseline"] = {"value": tokens_rank / sec, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                               "sample": desc}
+        r = oracle_sample_time(pw, dw)
+        out["cpu_baseline"] = {"value": r["tokens"] / r["measured_s"], "unit": "tokens/s", "cores": r["cores"],
+                               "kind": "oracle", "sample": r["desc"] + f" ({r['measured_s']:.1f} s)"}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if pg is not None:
@@ -656,6 +691,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--no-extras", action="store_true", help="skip the backward / fused-edge timings")
+    ap.add_argument("--steady-s", type=float, default=1.5,
+                    help="length of the extra back-to-back region reported under 'steady' (0: skip)")
     ap.add_argument("--parts", default="prefill,decode",
                     help="profiling aid: run only some parts of the step (the default runs the whole step)")
     args = ap.parse_args(argv)

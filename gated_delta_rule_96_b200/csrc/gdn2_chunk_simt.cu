@@ -183,8 +183,8 @@ __global__ void __launch_bounds__(256) intra_kernel(const Tok *__restrict__ q, c
 
 // ---------------------------------------------------------------- stage 2
 template <typename Tok, int K, int V>
-__global__ void __launch_bounds__(128) inter_kernel(const float *__restrict__ ws, const float *__restrict__ S0,
-                                                    Tok *__restrict__ o, float *__restrict__ ST, int H, int T,
+__global__ void __launch_bounds__(128) inter_kernel(const float *__restrict__ ws, const float *S0,
+                                                    Tok *__restrict__ o, float *ST, int H, int T,
                                                     int NC) {
     extern __shared__ float sm[];
     float *sS = sm;                  // [K][VT]

@@ -1112,7 +1112,7 @@ __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ alpha,
                     const __nv_bfloat16 *__restrict__ b, const __nv_bfloat16 *__restrict__ w,
-                    const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST, int H,
+                    const float *S0, __nv_bfloat16 *__restrict__ o, float *ST, int H,
                     int T, int seg_len, int nseg, uint32_t flags, const float *__restrict__ onorm,
                     unsigned char *ring, unsigned int *__restrict__ status) {
     extern __shared__ unsigned char smem_raw[];
@@ -1204,7 +1204,7 @@ __global__ void __launch_bounds__(NT, 1)
 // S_g = M_(g-1) S_(g-1) + N_(g-1) along the segments of each chain (g = 1 .. nseg-1), S_0 = S0.
 // One block per (chain, 16-column slice of S); fp32.
 __global__ void __launch_bounds__(256) segment_scan_kernel(const float *__restrict__ M, const float *__restrict__ N,
-                                                           const float *__restrict__ S0, float *__restrict__ Sg,
+                                                           const float *S0, float *__restrict__ Sg,
                                                            int nseg) {
     __shared__ float sprev[KD][16];
     const int chain = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;

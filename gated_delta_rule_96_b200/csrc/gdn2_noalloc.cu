@@ -11,6 +11,8 @@
 // GDN2_NOALLOC_SCRATCH_BYTES for the array until the process exits, and all calls
 // share the one array, so calls that overlap on the GPU (other streams, other host
 // threads) race on it and corrupt each other's results.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "gdn2.h"
@@ -24,20 +26,51 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN2_NOALLOC_SC
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+// Per device: the array's address and the id of the context it was looked up in.  A device
+// reset (cudaDeviceReset) replaces the context and reloads the module, so an address from
+// the old context is never reused: a new context id triggers a new lookup.
+struct Cached {
+    unsigned long long ctx_id;
+    void *addr;
+};
+Cached g_cache[kMaxDevices] = {};
 
-// Device address of the array on the current device, looked up once per device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Id of the calling thread's current context (driver entry points fetched through the
+// runtime, so the library does not link libcuda).  False when no context is current yet.
+bool current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *f1 = nullptr, *f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault) != cudaSuccess || !f1) return false;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault) != cudaSuccess || !f2) return false;
+        get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the array on the current device: looked up with that device current,
+// once per device and context (cudaGetSymbolAddress allocates nothing).
 int scratch_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GDN2_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
+    unsigned long long id = 0;
+    const bool known = current_context_id(&id);
+    if (!known || !g_cache[dev].addr || g_cache[dev].ctx_id != id) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN2_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        if (!current_context_id(&id)) return GDN2_ERR_CUDA;   // the lookup made the context current
+        g_cache[dev] = {id, p};
     }
-    *out = g_scratch_addr[dev];
+    *out = g_cache[dev].addr;
     return GDN2_OK;
 }
 

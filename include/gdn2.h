@@ -17,7 +17,8 @@
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers to contiguous, row-major buffers, each
  *     16-byte aligned.  The caller owns every buffer; the library allocates nothing
- *     and keeps no state between calls.
+ *     and keeps no state between calls, except gdn2_chunk_fwd_noalloc, whose fixed
+ *     scratch array (below) is library-owned device memory shared by all its calls.
  *   - Kernels launch on the calling thread's current CUDA device, which must own every
  *     pointer of the call (and `stream`, if given).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
@@ -189,10 +190,14 @@ GDN2_API const char *gdn2_status_str(int status);
  *     d_k = d_v = 128); larger problems return GDN2_ERR_NOALLOC_LIMIT and launch nothing.
  *   - The first call on a device looks up the array's device address on that device
  *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept per device and context: after a device reset
+ *     (cudaDeviceReset) the next call looks it up again in the new context.
  *   - All calls share the one array and it keeps the last call's contents (nothing in it
  *     needs to start at zero).  Calls that overlap on the GPU -- on different streams or
  *     from different host threads -- race on it: serialise them.
+ *   - The CUDA-core path it runs has no bounded waits and reports no device-side status:
+ *     there is no workspace, and gdn2_workspace_status does not apply.  The return value
+ *     reports argument checks and launch errors.
  */
 #define GDN2_NOALLOC_SCRATCH_BYTES (32u << 20)
 GDN2_API int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *alpha,

@@ -57,10 +57,24 @@ def f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+def elementwise_rel_err(got, ref):
+    """Elementwise relative error, floored at 1e-3 of the tensor's largest magnitude so that
+    entries near zero do not dominate: max_i |x_i - y_i| / (|y_i| + 1e-3 max|y|).  Reported
+    beside the bar's metric as information; the bar itself is the max-normalised error."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = np.max(np.abs(ref)) if ref.size else 0.0
+    if ref.size == 0 or scale == 0.0:
+        return float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    return float(np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * scale)))
+
+
 def assert_close(name, got, ref, tol):
     err = oracle.rel_err(got, ref)
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
-    assert err <= tol, f"{name}: rel err {err:.3e} > {tol:.1e}"
+    elem = elementwise_rel_err(got, ref)
+    print(f"{name}: max-normalised err {err:.3e} (bar {tol:.1e}); elementwise err {elem:.3e}")
+    assert err <= tol, f"{name}: rel err {err:.3e} > {tol:.1e} (elementwise {elem:.3e})"
     return err
 
 

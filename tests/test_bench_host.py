@@ -35,13 +35,18 @@ def test_peaks_loaded():
 
 def test_reference_arm_json(capsys, monkeypatch):
     monkeypatch.setenv("RANK", "0")
-    monkeypatch.setattr(bench, "oracle_sample_time", lambda pw, dw, budget_s, max_chains: (2.0, "stub", 3))
+    stub = {"measured_s": 0.5, "tokens": 1000.0, "full_step_s": 2.0, "desc": "stub", "cores": 3}
+    monkeypatch.setattr(bench, "oracle_sample_time", lambda pw, dw, budget_s, max_chains: stub)
     assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "1"]) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference"
     assert line["unit"] == "tokens/s" and line["metric"] == bench.METRIC
-    assert line["value"] == pytest.approx((8 * 4096 + 256) / 2.0)
+    # the sampled work per step is what ms_per_step reports; the rate is its tokens over its time
+    assert line["ms_per_step"] == pytest.approx(500.0)
+    assert line["value"] == pytest.approx(1000.0 / 0.5)
+    assert line["full_step_ms_extrapolated"] == pytest.approx(2000.0)
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] == 3
 
 
 def test_reference_arm_nonzero_rank_is_silent(capsys, monkeypatch):
@@ -54,8 +59,11 @@ def test_oracle_sample_time_small():
     import synth
     pw = synth.Workload("p", 1, 2, 128, 16, 16, "bf16", 1.0, seed=3)
     dw = synth.Workload("d", 4, 2, 1, 16, 16, "bf16", 1.0, s0_std=0.01, seed=4, decode=True)
-    sec, desc, cores = bench.oracle_sample_time(pw, dw, budget_s=0.5, max_chains=2)
-    assert sec > 0 and cores >= 1 and "oracle" in desc
+    r = bench.oracle_sample_time(pw, dw, budget_s=0.5, max_chains=2)
+    assert r["measured_s"] > 0 and r["cores"] >= 1 and "oracle" in r["desc"]
+    # 2 of 2 chains (T = 128 over H = 2) and 8 decode heads over H = 2
+    assert r["tokens"] == pytest.approx(2 * 128 / 2 + 8 / 2)
+    assert r["full_step_s"] >= r["measured_s"] * 0.99
 
 
 def _free_port():

@@ -195,3 +195,32 @@ def test_prefill_long_all_chains():
 
 def test_prefill_slow_decay_full_size_sampled():
     _sampled_check("prefill_slow_decay", [(0, 12), (2, 3), (6, 8)])
+
+
+@pytest.mark.parametrize("case", ["segmented", "simt_f32", "simt_bf16_d64"])
+def test_in_place_state_alias(case):
+    """S_T passed as the same buffer as S0 (the ABI allows it): the segmented path (few long
+    chains, B*H <= 64 and >= 32 chunks) and the CUDA-core path give the oracle's result."""
+    torch, g = cuda_or_skip()
+    if case == "segmented":
+        wl = synth.Workload("ip", 1, 2, 64 * 40 + 5, 128, 128, "bf16", 1.0, seed=84, s0_std=0.05,
+                            alpha_scale=0.02)
+    elif case == "simt_f32":
+        wl = synth.Workload("ip", 2, 3, 200, 64, 64, "f32", 0.0, seed=85, s0_std=0.05)
+    else:
+        wl = synth.Workload("ip", 2, 3, 130, 64, 128, "bf16", 1.0, seed=86, s0_std=0.05)
+    x = synth.make_inputs(wl)
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    S = torch.from_numpy(S0).cuda()
+    B, T, H, K = xd["q"].shape
+    V = xd["v"].shape[-1]
+    o = torch.full((B, T, H, V), float("nan"), dtype=xd["q"].dtype, device="cuda")
+    dt = g.GDN2_BF16 if wl.dtype == "bf16" else g.GDN2_F32
+    ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, dt))
+    g.gdn2_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["b"], xd["w"], S, o, S, workspace=ws)
+    torch.cuda.synchronize()
+    assert g.gdn2_workspace_status(ws) == 0
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
+    assert_close("o", f64(o), ref_o, TOL[wl.dtype])
+    assert_close("S_T (in place)", f64(S), ref_S, TOL[wl.dtype])
