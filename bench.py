@@ -26,6 +26,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "tokens/s GDN-2 chunk fwd (B8 H16 T4k d128) + decode; % tensor/HBM roofline"
+PATH_NAMES = {0: "simt", 1: "tcgen05 fused", 2: "tcgen05 two-stage (prep_kernel + walk_kernel)"}
 PREFILL = "prefill_1p3b"
 DECODE = "decode_b256"
 
@@ -441,9 +442,7 @@ def run_ours(args):
     pre_gbs = pb / (pre_ms * 1e-3) / 1e9
     dec_gbs = db / (dec_ms * 1e-3) / 1e9
     pflops = prefill_flops(B, T, H, K, V)
-    pre_kernel_key = "prefill_tc" if path == 1 else "prefill_simt"
-    pre_src = (["gated_delta_rule_96_b200/csrc/gdn2_chunk_tc.cu"] if path == 1
-               else ["gated_delta_rule_96_b200/csrc/gdn2_chunk_simt.cu"])
+    pre_kernel_key = {2: "prefill_two_stage", 1: "prefill_tc"}.get(path, "prefill_simt")
     tr_pre = recorded_traffic(pre_kernel_key)
     tr_dec = recorded_traffic("decode")
     roof_pre = {"bound": "hbm", "achieved": pre_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -495,7 +494,7 @@ def run_ours(args):
         except Exception as e:
             extras = {"unavailable": repr(e)[:200]}
 
-    launches_per_step = (1 if path == 1 else 2) + 1
+    launches_per_step = (1 if path == 1 else 2 * max(1, -(-((T + 63) // 64) // 64)) if path == 2 else 2) + 1
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -503,7 +502,7 @@ def run_ours(args):
         "config": bench_config(world),
         "roofline": roof_pre,
         "parts": {"prefill": {"ms": pre_ms_max, "tokens_per_s": B * T * world / (pre_ms_max * 1e-3),
-                              "path": "tcgen05" if path == 1 else "simt", "roofline": roof_pre},
+                              "path": PATH_NAMES.get(path, "simt"), "roofline": roof_pre},
                   "decode": {"ms": dec_ms_max, "tokens_per_s": dw.B * world / (dec_ms_max * 1e-3),
                              "roofline": roof_dec}},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -26,14 +26,26 @@ bool use_tc(int B, int H, int T, int K, int V, int C, int dtype) {
     return gdn2::tc_supported(B, H, T, K, V, C, dtype == GDN2_BF16 ? 1 : 0);
 }
 
+// Implementation for these sizes: 0 = CUDA-core two-kernel path; 1 = fused tcgen05 kernel (one CTA
+// per chain, the chain cut into segments in time when there are few long chains); 2 = two-stage
+// tcgen05 path (intra-chunk work parallel over every chunk-head, then the state chain), taken when
+// there are more chains than the fused kernel's segmentation serves.
+int select_path(int B, int H, int T, int K, int V, int C, int dtype) {
+    if (!use_tc(B, H, T, K, V, C, dtype)) return 0;
+    return (long long)B * H > 64 ? 2 : 1;
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t gdn2_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C, int dtype) {
     if (B < 0 || H < 0 || T < 0 || !dim_ok(d_k) || !dim_ok(d_v) || C != 64) return gdn2::kStatusBytes;
-    if (use_tc(B, H, T, d_k, d_v, C, dtype)) return gdn2::tc_workspace_bytes(B, H, T, d_k, d_v, C);
-    return gdn2::simt_workspace_bytes(B, H, T, d_k, d_v, C);
+    switch (select_path(B, H, T, d_k, d_v, C, dtype)) {
+        case 2: return gdn2::split_workspace_bytes(B, H, T);
+        case 1: return gdn2::tc_workspace_bytes(B, H, T, d_k, d_v, C);
+        default: return gdn2::simt_workspace_bytes(B, H, T, d_k, d_v, C);
+    }
 }
 
 size_t gdn2_chunk_fwd_edges_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C) {
@@ -42,7 +54,8 @@ size_t gdn2_chunk_fwd_edges_workspace_bytes(int B, int H, int T, int d_k, int d_
 }
 
 int gdn2_chunk_fwd_path(int B, int H, int T, int d_k, int d_v, int C, int dtype) {
-    return use_tc(B, H, T, d_k, d_v, C, dtype) ? 1 : 0;
+    if (B < 0 || H < 0 || T < 0) return 0;
+    return select_path(B, H, T, d_k, d_v, C, dtype);
 }
 
 int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
@@ -75,7 +88,10 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const float *alp
         return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
     }
     const int bf16 = dtype == GDN2_BF16 ? 1 : 0;
-    if (use_tc(B, H, T, d_k, d_v, C, dtype))
+    const int path = select_path(B, H, T, d_k, d_v, C, dtype);
+    if (path == 2)
+        rc = gdn2::launch_chunk_split(q, k, v, alpha, b, w, S0, o, S_T, B, H, T, workspace, st);
+    else if (path == 1)
         rc = gdn2::launch_chunk_tc(q, k, v, alpha, b, w, S0, o, S_T, B, H, T, d_k, d_v, C, workspace, st);
     else
         rc = gdn2::launch_chunk_simt(q, k, v, alpha, b, w, S0, o, S_T, B, H, T, d_k, d_v, C, bf16, workspace, st);

@@ -29,6 +29,13 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
                     const void *w, const float *S0, void *o, float *ST, int B, int H, int T, int K, int V,
                     int C, void *ws, cudaStream_t st, int edges = 0, const float *onorm = nullptr);
 
+// Two-stage tcgen05 prefill (bf16 tokens, d_k = d_v = 128, C = 64): the intra-chunk work in parallel
+// over every chunk-head, then the state chain; long sequences in windows of 64 chunks.
+size_t split_workspace_bytes(int B, int H, int T);
+int launch_chunk_split(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                       const void *w, const float *S0, void *o, float *ST, int B, int H, int T, void *ws,
+                       cudaStream_t st);
+
 // Backward pass (three sequential passes per chain; fp32 gradients; d_k, d_v in {64, 128}).
 size_t bwd_workspace_bytes(int B, int H, int T, int K, int V);
 int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,

@@ -170,6 +170,36 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
 }
 
+// Tiled tensor copies (TMA) through a CUtensorMap kernel parameter (passed by address).  No
+// multicast: every copy moves data between this GPU's global memory and this CTA's shared memory.
+// A 4-D box at coordinates {c0, c1, c2, c3} (c0 innermost; c0 * element size is a multiple of 16).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst_smem, const void *map, int c0, int c1, int c2, int c3,
+                                            uint32_t mbar) {
+    asm volatile("cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+                 "%4, %5}], [%6];" ::"r"(dst_smem),
+                 "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const void *map, int c0, int c1, int c2, int c3, uint32_t src_smem) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(map),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src_smem)
+                 : "memory");
+}
+// Brings a tensor map (a kernel parameter, by address) into the descriptor cache.
+__device__ __forceinline__ void prefetch_tmap(const void *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+// Untiled bulk store shared -> global (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src_smem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
+                 : "memory");
+}
+// Bulk-group bookkeeping of the issuing thread: close the group of stores issued so far; wait
+// until every group has finished reading its shared-memory source (.read) or has completed.
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Register budget of the calling warpgroup (all 128 threads execute it).
 template <uint32_t N>
 __device__ __forceinline__ void regs_inc() {

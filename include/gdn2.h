@@ -205,7 +205,11 @@ GDN2_API int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                     int H, int T, int d_k, int d_v, int C, int dtype, void *stream);
 
 /* Which prefill implementation gdn2_chunk_fwd selects for these sizes:
- * 0 = SIMT two-kernel path (fp32 FMA), 1 = fused tcgen05 tensor-core path. */
+ * 0 = SIMT two-kernel path (fp32 FMA; fp32 tokens, or d_k / d_v = 64);
+ * 1 = fused tcgen05 kernel, one CTA per (b, h) chain (bf16, d_k = d_v = 128, B*H <= 64; long
+ *     sequences are cut into segments in time and composed);
+ * 2 = two-stage tcgen05 path (bf16, d_k = d_v = 128, B*H > 64): the intra-chunk work runs in
+ *     parallel over every chunk of every chain, then one CTA per chain walks the state. */
 GDN2_API int gdn2_chunk_fwd_path(int B, int H, int T, int d_k, int d_v, int C, int dtype);
 
 #ifdef __cplusplus

@@ -55,8 +55,17 @@ def test_workspace_bytes():
 
 
 def test_workspace_bytes_tensor_core_path():
-    # many chains: the fused kernel needs only the status header
-    assert g.gdn2_chunk_fwd_workspace_bytes(8, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 256
+    # many chains: the two-stage path keeps one 75,776-byte record per chunk-head of a window of at
+    # most 64 chunks
+    rec = 75776
+    assert g.gdn2_chunk_fwd_workspace_bytes(8, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 256 + 8 * 16 * 64 * rec
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 65, 64 * 70 + 5, 128, 128, 64, g.GDN2_BF16) == 256 + 65 * 64 * rec
+    assert g.gdn2_chunk_fwd_workspace_bytes(2, 33, 65, 128, 128, 64, g.GDN2_BF16) == 256 + 66 * 2 * rec
+    assert g.gdn2_chunk_fwd_path(8, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 2
+    # up to 64 chains: the fused kernel; its few-chain form needs only the status header when short
+    assert g.gdn2_chunk_fwd_path(4, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 1
+    assert g.gdn2_chunk_fwd_workspace_bytes(4, 16, 1024, 128, 128, 64, g.GDN2_BF16) == 256
+    assert g.gdn2_chunk_fwd_path(8, 16, 4096, 128, 128, 64, g.GDN2_F32) == 0
     # few long chains run in parallel over segments: three fp32 states per (chain, segment)
     state = 4 * 128 * 128
     # B1 H16 T65536: 1,024 chunks, 8 segments of 128 chunks

@@ -51,10 +51,15 @@ def test_slow_decay_small():
     _full_check(wl, synth.make_state(wl))
 
 
-def test_extreme_decay_and_unit_decay():
+# (B, H): up to 64 chains run the fused kernel, more the two-stage path
+PATHS = pytest.mark.parametrize("BH", [(1, 2), (2, 33)], ids=["fused", "two_stage"])
+
+
+@PATHS
+def test_extreme_decay_and_unit_decay(BH):
     """alpha spanning 1e-30 .. 1 (every factor stays finite), exact alpha = 1 rows."""
     torch, g = cuda_or_skip()
-    wl = synth.Workload("x", 1, 2, 130, 128, 128, "bf16", 1.0, seed=79, s0_std=0.05)
+    wl = synth.Workload("x", BH[0], BH[1], 130, 128, 128, "bf16", 1.0, seed=79, s0_std=0.05)
     x = synth.make_inputs(wl)
     rng = np.random.default_rng(5)
     a = x["alpha"].copy()
@@ -70,15 +75,38 @@ def test_extreme_decay_and_unit_decay():
     assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
 
 
+@PATHS
+def test_tiny_first_decay_of_each_chunk(BH):
+    """The first alpha of every chunk is 1e-30 in half of the key channels, whose other tokens decay
+    by 1/2: each chunk's log-decay span (63 in log2) is far below the wide-span limit, but the
+    midpoint of its prefix lies near -131, so a decay factor formed as exp(-m) before the chunk's
+    first position would leave fp32's range.  Every factor the method needs, exp(g_r - m), is within
+    exp(+-span/2)."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("tf", BH[0], BH[1], 64 * 3 + 2, 128, 128, "bf16", 1.0, seed=88, s0_std=0.05)
+    x = synth.make_inputs(wl)
+    a = x["alpha"].copy()
+    a[..., ::2] = np.float32(0.5)
+    a[:, ::64, :, ::2] = np.float32(1e-30)
+    x["alpha"] = a
+    S0 = synth.make_state(wl)
+    xd = to_device(torch, x, wl.dtype)
+    o, ST = prefill(torch, g, xd, torch.from_numpy(S0).cuda())
+    ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
+    assert_close("o", f64(o), ref_o, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
+@PATHS
 @pytest.mark.parametrize("span", [120.0, 165.0, 172.0, 176.0])
-def test_chunk_spans_near_the_tensor_core_limit(span):
+def test_chunk_spans_near_the_tensor_core_limit(span, BH):
     """Every chunk decays by about `span` (log2) in half of the key channels, so the kernel's
     decay factors around the chunk midpoint reach 2^(span/2) and the frame factors of two
     consecutive chunks multiply to about 2^-span (below fp32's range for span > 149); 176 lies
     past the tensor-core limit (173) and takes the wide-span path.  The other channels decay
     slowly, so the carried state stays visible in o."""
     torch, g = cuda_or_skip()
-    wl = synth.Workload("x", 1, 2, 320, 128, 128, "bf16", 1.0, seed=81, s0_std=0.05)
+    wl = synth.Workload("x", BH[0], BH[1], 320, 128, 128, "bf16", 1.0, seed=81, s0_std=0.05)
     x = synth.make_inputs(wl)
     a = x["alpha"].copy()
     a[..., ::2] = np.float32(2.0 ** (-span / 64.0))    # per-token decay of the fast channels
@@ -197,7 +225,7 @@ def test_prefill_slow_decay_full_size_sampled():
     _sampled_check("prefill_slow_decay", [(0, 12), (2, 3), (6, 8)])
 
 
-@pytest.mark.parametrize("case", ["segmented", "simt_f32", "simt_bf16_d64"])
+@pytest.mark.parametrize("case", ["segmented", "two_stage", "simt_f32", "simt_bf16_d64"])
 def test_in_place_state_alias(case):
     """S_T passed as the same buffer as S0 (the ABI allows it): the segmented path (few long
     chains, B*H <= 64 and >= 32 chunks) and the CUDA-core path give the oracle's result."""
@@ -205,6 +233,8 @@ def test_in_place_state_alias(case):
     if case == "segmented":
         wl = synth.Workload("ip", 1, 2, 64 * 40 + 5, 128, 128, "bf16", 1.0, seed=84, s0_std=0.05,
                             alpha_scale=0.02)
+    elif case == "two_stage":
+        wl = synth.Workload("ip", 2, 33, 200, 128, 128, "bf16", 1.0, seed=87, s0_std=0.05)
     elif case == "simt_f32":
         wl = synth.Workload("ip", 2, 3, 200, 64, 64, "f32", 0.0, seed=85, s0_std=0.05)
     else:
@@ -224,3 +254,28 @@ def test_in_place_state_alias(case):
     ref_o, ref_S = oracle.recurrence(*(x[k] for k in ("q", "k", "v", "alpha", "b", "w")), S0)
     assert_close("o", f64(o), ref_o, TOL[wl.dtype])
     assert_close("S_T (in place)", f64(S), ref_S, TOL[wl.dtype])
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_two_stage_small(T):
+    """More than 64 chains: the intra-chunk stage runs over every chunk-head, then one block per
+    chain walks the state; ragged and single-token sequences included."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("ts", 2, 33, T, 128, 128, "bf16", 1.0, s0_std=0.05, seed=2000 + T)
+    assert g.gdn2_chunk_fwd_path(2, 33, T, 128, 128, 64, g.GDN2_BF16) == 2
+    _full_check(wl, synth.make_state(wl))
+
+
+@pytest.mark.parametrize("gates", ["kda", "gdn"])
+def test_two_stage_collapsed_gates(gates):
+    wl = synth.Workload("tc", 2, 33, 192, 128, 128, "bf16", 1.0, gates=gates, seed=2010)
+    _full_check(wl)
+
+
+def test_two_stage_windows():
+    """71 chunks of 65 chains: the record buffer holds 64 chunks, so the sequence runs as two windows
+    with the state carried between them; slow decay keeps the carried state visible."""
+    torch, g = cuda_or_skip()
+    wl = synth.Workload("tw", 1, 65, 64 * 70 + 5, 128, 128, "bf16", 1.0, s0_std=0.05, seed=2100, alpha_scale=0.02)
+    assert g.gdn2_chunk_fwd_path(1, 65, wl.T, 128, 128, 64, g.GDN2_BF16) == 2
+    _full_check(wl, synth.make_state(wl))
