@@ -328,6 +328,34 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- tensor-core phases
+
+def tensor_phase_probe(g, torch, dev, stream, peak_tflops, reps=(4000, 1500)):
+    """The prefill's tensor-core products of one chunk (G1, G2, G3, G4/G5 with the kernels' shapes and
+    shared-memory operand layouts), run alone on every SM: mode 0 back to back (the tensor pipe's rate
+    on these GEMM phases), mode 1 each group waiting for the one before (the prefill's dependency
+    order).  Event-timed; fractions of the measured bf16 peak."""
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    ws = g.new_workspace(256, dev)
+    out = {"kernel": "phase_kernel", "ctas": nsm, "flops_per_chunk": g.PHASE_PROBE_FLOPS_PER_CHUNK,
+           "peak": peak_tflops, "unit": "TFLOP/s"}
+    for mode, r in zip((0, 1), reps):
+        g.gdn2_gemm_phase_probe(mode, 50, nsm, ws, stream=stream)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.gdn2_gemm_phase_probe(mode, r, nsm, ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b)
+        tf = r * nsm * g.PHASE_PROBE_FLOPS_PER_CHUNK / (ms * 1e-3) / 1e12
+        key = "back_to_back" if mode == 0 else "dependent"
+        out[key] = {"chunks_per_cta": r, "ms": ms, "achieved": tf, "frac": tf / peak_tflops}
+    if g.gdn2_workspace_status(ws) != 0:
+        raise RuntimeError("phase probe reported an expired wait")
+    return out
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -340,6 +368,11 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     g.load_library()
     pw, dw = rank_workload(PREFILL, rank), rank_workload(DECODE, rank)
+    if args.prefill_shape:   # profiling aid: another prefill size (not a bench line)
+        Bp, Hp, Tp = (int(x) for x in args.prefill_shape.split(","))
+        fields = {f: getattr(pw, f) for f in pw.__dataclass_fields__}
+        fields.update(B=Bp, H=Hp, T=Tp)
+        pw = synth.Workload(**fields)
 
     def dev_tokens(x, dtype):
         out = {}
@@ -453,6 +486,15 @@ def run_ours(args):
                 "frac": dec_gbs / peaks["hbm_gbs"], "traffic": tr_dec, "peak_src": peaks["src"],
                 "kernel": "decode", "algorithmic_bytes_per_launch": db}
 
+    # ---- the tensor pipe on the prefill's GEMM phases (outside the timed region)
+    try:
+        tp = tensor_phase_probe(g, torch, dev, stream, peaks["bf16_tflops"])
+        roof_pre["tensor_phase_frac"] = tp["back_to_back"]["frac"]
+        roof_pre["tensor_phase_dependent_frac"] = tp["dependent"]["frac"]
+        roof_pre["tensor_phase"] = tp
+    except Exception as e:   # a measurement aid: never lose the step's line over it
+        roof_pre["tensor_phase"] = {"unavailable": repr(e)[:200]}
+
     # ---- end to end through the public API: pinned host inputs -> device -> results -> host
     host = {k: v.to("cpu").pin_memory() for k, v in P.items()}
     host_d = {k: v.to("cpu").pin_memory() for k, v in D.items()}
@@ -516,6 +558,8 @@ def run_ours(args):
         out["next_rows"] = extras
     if parts != {"prefill", "decode"}:
         out["config"]["parts_only"] = sorted(parts)   # profiling run: not a bench line
+    if args.prefill_shape:
+        out["config"]["prefill_shape"] = args.prefill_shape   # profiling run: not a bench line
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_sample_time(pw, dw)
         out["cpu_baseline"] = {"value": r["tokens"] / r["measured_s"], "unit": "tokens/s", "cores": r["cores"],
@@ -692,6 +736,8 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true", help="skip the backward / fused-edge timings")
     ap.add_argument("--steady-s", type=float, default=1.5,
                     help="length of the extra back-to-back region reported under 'steady' (0: skip)")
+    ap.add_argument("--prefill-shape", default="",
+                    help="profiling aid: B,H,T of the prefill instead of the bench workload (not a bench line)")
     ap.add_argument("--parts", default="prefill,decode",
                     help="profiling aid: run only some parts of the step (the default runs the whole step)")
     args = ap.parse_args(argv)

@@ -19,7 +19,8 @@ __all__ = [
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
-    "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_recurrence",
+    "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_recurrence", "gdn2_gemm_phase_probe",
+    "PHASE_PROBE_FLOPS_PER_CHUNK",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +30,7 @@ _lib = None
 GDN2_F32, GDN2_BF16 = 0, 1
 STATUS_HEADER_BYTES = 256
 NOALLOC_SCRATCH_BYTES = 32 << 20   # GDN2_NOALLOC_SCRATCH_BYTES in include/gdn2.h
+PHASE_PROBE_FLOPS_PER_CHUNK = 14680064   # GDN2_PHASE_PROBE_FLOPS_PER_CHUNK in include/gdn2.h
 
 
 class GDN2Error(RuntimeError):
@@ -72,6 +74,8 @@ def load_library():
     lib.gdn2_chunk_bwd_workspace_bytes.restype = sz
     lib.gdn2_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
     lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_gemm_phase_probe.argtypes = [i, i, i, vp, sz, vp]
+    lib.gdn2_gemm_phase_probe.restype = i
     lib.gdn2_status_str.argtypes = [i]
     lib.gdn2_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -288,6 +292,17 @@ def gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=None) -> None:
                                              _ptr(o), B, H, K, V, dt, _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_decode_step")
+
+
+def gdn2_gemm_phase_probe(mode, reps, nctas, workspace, stream=None) -> None:
+    """Measurement aid (include/gdn2.h): one chunk's tensor-core products, `reps` chunks per CTA on
+    `nctas` CTAs; mode 0 back to back, mode 1 each group waiting for the one before."""
+    _check_cuda(workspace)
+    with _on_device(workspace):
+        rc = load_library().gdn2_gemm_phase_probe(int(mode), int(reps), int(nctas), _ptr(workspace),
+                                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_gemm_phase_probe")
 
 
 def gdn2_workspace_status(workspace, clear=False, stream=None) -> int:

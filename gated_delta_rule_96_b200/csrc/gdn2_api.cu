@@ -164,6 +164,15 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const float *alp
                                   d_k, d_v, dtype == GDN2_BF16 ? 1 : 0, workspace, st);
 }
 
+int gdn2_gemm_phase_probe(int mode, int reps, int nctas, void *workspace, size_t workspace_bytes, void *stream) {
+    if ((mode != 0 && mode != 1) || reps < 1 || nctas < 1) return GDN2_ERR_SHAPE;
+    if (!workspace) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    if (workspace_bytes < gdn2::kStatusBytes) return GDN2_ERR_WORKSPACE;
+    return gdn2::launch_phase_probe(mode, reps, nctas, reinterpret_cast<unsigned int *>(workspace),
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
 int gdn2_workspace_status(void *workspace, int clear, int *out, void *stream) {
     if (!workspace || !out) return GDN2_ERR_NULL;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

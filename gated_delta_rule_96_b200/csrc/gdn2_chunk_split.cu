@@ -63,17 +63,33 @@ constexpr uint32_t R_COPY = R_VEC + 3 * 128 * 4;   // bytes moved per record
 constexpr uint32_t R_BYTES = 75776;                // record stride (1024-aligned)
 
 // ---------------------------------------------------------------------------- stage 1
-constexpr int P1_NT = 256;
+// One persistent CTA per SM over the window's chunk-heads, three roles working on consecutive
+// chunk-heads at once:
+//   warps 0-7   build group: alpha prefix, decay factors and the bf16 operands of chunk-head j+1,
+//               G1, then A (fp32, for the solve) and P (bf16, to the record) out of TMEM
+//   warps 8-11  solve group: T = (I + A)^-1, G2 and the W', Ũ rows of chunk-head j
+//   warp 12     producer: a two-stage ring of token tiles by TMA (alpha through one buffer)
+// The solve group stores each record by bulk copies (K̃ and Q̂ as soon as G1 has run, -W' and Ũ at the
+// end) and releases the stage once they have read it.
+constexpr int P1_NT = 416;
+constexpr uint32_t P1_STAGE = 81920;                 // per stage: EQ, KT, U, W tiles
 constexpr uint32_t P1_EQ = 0;                        // b -> Ê -> -W' (rows 0-63), q -> Q̂ (rows 64-127)
 constexpr uint32_t P1_KT = 32768;                    // k -> K̃
 constexpr uint32_t P1_U = 49152;                     // v -> U -> Ũ
-constexpr uint32_t P1_W = 65536;                     // w; then [T; P] (128 rows, K = 64)
-constexpr uint32_t P1_AS = 81920;                    // fp32 A / T^T [64][LDA]; first the prefix totals
-constexpr uint32_t P1_X = P1_AS + 64 * LDA * 4;      // solve scratch (4 KB)
-constexpr uint32_t P1_MISC = P1_X + 4096;
+constexpr uint32_t P1_W = 65536;                     // w; then [T; T] (128 rows, K = 64)
+constexpr uint32_t P1_A = 2 * P1_STAGE;              // alpha fp32 [64][128] (one buffer)
+constexpr uint32_t P1_AS = P1_A + 32768;             // solve group: fp32 A / T^T [64][LDA]
+constexpr uint32_t P1_X = P1_AS + 64 * LDA * 4;      // solve group scratch (4 KB)
+constexpr uint32_t P1_WT = P1_X + 4096;              // build group: [8][128] log2 totals, then g_0 [128]
+constexpr uint32_t P1_MISC = P1_WT + 4608;
 constexpr uint32_t P1_BYTES = P1_MISC + 256 + 1024;  // + alignment slack
-enum : uint32_t { M1_LOAD = 0, M1_G1 = 8, M1_G2 = 16, M1_TSLOT = 32, M1_ABORT = 36 };
-constexpr uint32_t P1_TM_D1 = 0, P1_TM_D2 = 0, P1_TM_D3 = 128, P1_TM_COLS = 256;
+// mbarriers: FULL and OUT per stage; alpha full / free; G1; A ready / A scratch free; G2
+enum : uint32_t {
+    M1_FULL = 0, M1_OUT = 16, M1_AFULL = 32, M1_AFREE = 40, M1_G1 = 48, M1_AREADY = 56, M1_ASFREE = 64,
+    M1_G2 = 72, M1_TSLOT = 96, M1_ABORT = 100
+};
+constexpr uint32_t P1_TM_D1 = 0, P1_TM_D2 = 128, P1_TM_D3 = 256, P1_TM_COLS = 512;
+constexpr uint32_t BAR_A = 1, BAR_B = 2;   // named barriers: build group (256), solve group (128)
 
 constexpr uint32_t ID_G1 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t ID_G2 = idesc_bf16(128, 128, 0, 1);
@@ -81,14 +97,24 @@ constexpr uint32_t ID_G3 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G4 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G5 = idesc_bf16(128, 128, 1, 1);
 
-struct TokMaps {   // [B, T, H, 128] bf16 token tensors as 4-D maps (d, H, T, B), box 64 x 1 x 64 x 1
-    CUtensorMap q, k, b, v, w;
+struct TokMaps {   // [B, T, H, 128] token tensors as 4-D maps (d, H, T, B): bf16 with a 64 x 1 x 64 x 1 box
+    CUtensorMap q, k, b, v, w, alpha;   // in the 128-byte swizzle; alpha fp32 with a 128 x 1 x 64 x 1 box
 };
 
-// Block-wide bounded wait: every thread gets the same verdict.
-__device__ __forceinline__ bool block_wait(uint32_t mb, uint32_t parity, volatile uint32_t *abort) {
+// Bounded wait of one thread (the producer); on expiry it sets the abort flag.
+__device__ __forceinline__ bool thread_wait1(uint32_t mb, uint32_t parity, volatile uint32_t *abort) {
+    if (!mbar_wait(mb, parity, WAIT_LIMIT) || *abort) {
+        *abort = 1u;
+        return false;
+    }
+    return true;
+}
+
+// Bounded wait of a warp group (named barrier `bar`, n threads): every thread gets the same verdict.
+__device__ __forceinline__ bool gwait(uint32_t mb, uint32_t parity, uint32_t bar, uint32_t n, volatile uint32_t *abort) {
     bool ok = mbar_wait(mb, parity, WAIT_LIMIT) && !*abort;
-    const bool fail = __syncthreads_or(!ok) != 0;
+    const bool fail = group_or(bar, n, !ok);
+    fence_after();
     if (fail) *abort = 1u;
     return !fail;
 }
@@ -142,315 +168,380 @@ __device__ __forceinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat
     wait_st();
 }
 
-__global__ void __launch_bounds__(P1_NT, 2)
+__global__ void __launch_bounds__(P1_NT, 1)
     prep_kernel(const __grid_constant__ TokMaps maps, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
-                const __nv_bfloat16 *b, const float *__restrict__ alpha, unsigned char *records, int H, int T,
-                int NC, int n0, int nw, int nch, unsigned int *status) {
+                const __nv_bfloat16 *b, const float *alpha, unsigned char *records, int H, int T, int n0, int nw,
+                int nch, unsigned int *status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t misc = smem_u32(sm + P1_MISC);
     volatile uint32_t *abort = reinterpret_cast<volatile uint32_t *>(sm + P1_MISC + M1_ABORT);
-    const uint32_t aEQ = smem_u32(sm + P1_EQ), aKT = smem_u32(sm + P1_KT), aU = smem_u32(sm + P1_U),
-                   aW = smem_u32(sm + P1_W);
-    float *AS = reinterpret_cast<float *>(sm + P1_AS);
-    float *WT = AS;              // [8][128] per-warp log2 totals, then g_0 [128]
-    float *v_g0 = WT + 8 * 128;
 
     if (warp == 0) tmem_alloc(misc + M1_TSLOT, P1_TM_COLS);
     if (tid == 0) {
-        mbar_init(misc + M1_LOAD, 1);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(misc + M1_FULL + 8 * st, 1);
+            mbar_init(misc + M1_OUT + 8 * st, 1);
+        }
+        mbar_init(misc + M1_AFULL, 1);
+        mbar_init(misc + M1_AFREE, 1);
         mbar_init(misc + M1_G1, 1);
+        mbar_init(misc + M1_AREADY, 1);
+        mbar_init(misc + M1_ASFREE, 1);
         mbar_init(misc + M1_G2, 1);
         *abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b);
-        prefetch_tmap(&maps.v); prefetch_tmap(&maps.w);
     }
     fence_before();
     __syncthreads();
     fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + P1_MISC + M1_TSLOT);
+    // chunk-heads of the window in (batch, chunk, head) order: neighbouring CTAs read adjacent heads
+    auto coords = [&](int ch, int &h, int &bb, int &n) {
+        h = ch % H;
+        n = n0 + (ch / H) % nw;
+        bb = ch / (H * nw);
+    };
+    const int njobs = (int)blockIdx.x < nch ? (nch - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto rec_of = [&](int j) { return records + (size_t)(blockIdx.x + j * gridDim.x) * R_BYTES; };
 
-    const int c4 = lane * 4, p0 = warp * 8;   // build mapping: 8 positions x 4 channels per thread
-    int it = 0;
-    for (int ch = blockIdx.x; ch < nch; ch += gridDim.x, ++it) {
-        // chunk-heads of the window in (batch, chunk, head) order: neighbouring CTAs read adjacent heads
-        const int h = ch % H, nl = (ch / H) % nw, bb = ch / (H * nw), n = n0 + nl;
-        const int t0 = n * C, L = min(C, T - t0);
-        unsigned char *rec = records + (size_t)ch * R_BYTES;
-        const uint32_t par = (uint32_t)(it & 1);
-
-        // ------------------------------------------------------------------ token tiles by TMA
-        if (tid == 0) {
-            bulk_wait_read_all();   // the previous chunk-head's record stores have read their sources
-            mbar_arrive_expect_tx(misc + M1_LOAD, 10u * 8192u);
+    if (warp == 12) {
+        // ------------------------------------------------------------------ producer (one thread)
+        if (lane == 0) {
+            prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b);
+            prefetch_tmap(&maps.v); prefetch_tmap(&maps.w); prefetch_tmap(&maps.alpha);
+            int last_tiles[2] = {-1, -1}, last_alpha = -1;
+            for (int j = 0; j < njobs; ++j) {
+                const int stg = j & 1;
+                int h, bb, n;
+                coords(blockIdx.x + j * gridDim.x, h, bb, n);
+                const int t0 = n * C;
+                // alpha into its single buffer once the previous job's prefix has read it
+                if (j >= 1 && !thread_wait1(misc + M1_AFREE, (uint32_t)((j - 1) & 1), abort)) break;
+                mbar_arrive_expect_tx(misc + M1_AFULL, 32768u);
+                tma_load_4d(smem_u32(sm + P1_A), &maps.alpha, 0, h, t0, bb, misc + M1_AFULL);
+                last_alpha = j;
+                // the token tiles once the stage's previous job is finished and its record stores have read it
+                if (j >= 2 && !thread_wait1(misc + M1_OUT + 8 * stg, (uint32_t)(((j - 2) >> 1) & 1), abort)) break;
+                const uint32_t st = smem_u32(sm + stg * P1_STAGE), fb = misc + M1_FULL + 8 * stg;
+                mbar_arrive_expect_tx(fb, 10u * 8192u);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                tma_load_4d(aEQ + hf * 16384, &maps.b, 64 * hf, h, t0, bb, misc + M1_LOAD);
-                tma_load_4d(aEQ + hf * 16384 + 8192, &maps.q, 64 * hf, h, t0, bb, misc + M1_LOAD);
-                tma_load_4d(aKT + hf * 8192, &maps.k, 64 * hf, h, t0, bb, misc + M1_LOAD);
-                tma_load_4d(aU + hf * 8192, &maps.v, 64 * hf, h, t0, bb, misc + M1_LOAD);
-                tma_load_4d(aW + hf * 8192, &maps.w, 64 * hf, h, t0, bb, misc + M1_LOAD);
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_4d(st + P1_EQ + hf * 16384, &maps.b, 64 * hf, h, t0, bb, fb);
+                    tma_load_4d(st + P1_EQ + hf * 16384 + 8192, &maps.q, 64 * hf, h, t0, bb, fb);
+                    tma_load_4d(st + P1_KT + hf * 8192, &maps.k, 64 * hf, h, t0, bb, fb);
+                    tma_load_4d(st + P1_U + hf * 8192, &maps.v, 64 * hf, h, t0, bb, fb);
+                    tma_load_4d(st + P1_W + hf * 8192, &maps.w, 64 * hf, h, t0, bb, fb);
+                }
+                last_tiles[stg] = j;
             }
+            // no tile load may be left in flight when the block exits (after an abort)
+            for (int stg = 0; stg < 2; ++stg)
+                if (last_tiles[stg] >= 0) mbar_wait(misc + M1_FULL + 8 * stg, (uint32_t)((last_tiles[stg] >> 1) & 1), WAIT_LIMIT);
+            if (last_alpha >= 0) mbar_wait(misc + M1_AFULL, (uint32_t)(last_alpha & 1), WAIT_LIMIT);
         }
-        // ------------------------------------------------------------------ alpha and the log-decay prefix
-        const size_t row0 = ((size_t)bb * T + t0) * H + h;
-        float al[8][4];
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(alpha + (row0 + (size_t)min(p0 + p, L - 1) * H) * KD + c4));
-            al[p][0] = a4.x; al[p][1] = a4.y; al[p][2] = a4.z; al[p][3] = a4.w;
-        }
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)   // past the end: alpha = 1; subnormal alpha: smallest normal
-                al[p][j] = p0 + p >= L ? 1.f : fmaxf(al[p][j], 1.17549435e-38f);
-        // log2 of the product of the thread's 8 alphas per channel: the exponent fields plus log2 of
-        // the product of the mantissas (in [1, 256))
-        float lw[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int ex = 0;
-            float mp = 1.f;
+    } else if (warp < 8) {
+        // ------------------------------------------------------------------ build group
+        float *WT = reinterpret_cast<float *>(sm + P1_WT);
+        float *v_g0 = WT + 8 * 128;
+        const float *AL = reinterpret_cast<const float *>(sm + P1_A);
+        const int c4 = lane * 4, p0 = warp * 8;   // 8 positions x 4 channels per thread
+        for (int j = 0; j < njobs; ++j) {
+            const int stg = j & 1;
+            int h, bb, n;
+            coords(blockIdx.x + j * gridDim.x, h, bb, n);
+            const int t0 = n * C, L = min(C, T - t0);
+            unsigned char *S = sm + stg * P1_STAGE;
+            const uint32_t aEQ = smem_u32(S + P1_EQ), aKT = smem_u32(S + P1_KT);
+            const uint32_t d1 = tmem + P1_TM_D1;
+
+            // ---------------------------------------------------------------- alpha and the log-decay prefix
+            if (!gwait(misc + M1_AFULL, (uint32_t)(j & 1), BAR_A, 256, abort)) break;
+            float al[8][4];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const uint32_t u = __float_as_uint(al[p][j]);
-                ex += (int)(u >> 23) - 127;
-                mp *= __uint_as_float((u & 0x7FFFFFu) | 0x3F800000u);
+                const float4 a4 = *reinterpret_cast<const float4 *>(AL + (p0 + p) * KD + c4);
+                // past the end: alpha = 1 (the copy filled zeros); subnormal alpha: smallest normal
+                al[p][0] = p0 + p >= L ? 1.f : fmaxf(a4.x, 1.17549435e-38f);
+                al[p][1] = p0 + p >= L ? 1.f : fmaxf(a4.y, 1.17549435e-38f);
+                al[p][2] = p0 + p >= L ? 1.f : fmaxf(a4.z, 1.17549435e-38f);
+                al[p][3] = p0 + p >= L ? 1.f : fmaxf(a4.w, 1.17549435e-38f);
             }
-            lw[j] = (float)ex + fast_log2(mp);
-        }
-        *reinterpret_cast<float4 *>(WT + warp * 128 + c4) = make_float4(lw[0], lw[1], lw[2], lw[3]);
-        if (warp == 0)
-            *reinterpret_cast<float4 *>(v_g0 + c4) =
-                make_float4(fast_log2(al[0][0]), fast_log2(al[0][1]), fast_log2(al[0][2]), fast_log2(al[0][3]));
-        __syncthreads();
-        float pre[4] = {0.f, 0.f, 0.f, 0.f}, gC[4] = {0.f, 0.f, 0.f, 0.f};
+            // log2 of the product of the thread's 8 alphas per channel: the exponent fields plus log2 of
+            // the product of the mantissas (in [1, 256))
+            float lw[4];
 #pragma unroll
-        for (int w2 = 0; w2 < 8; ++w2) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(WT + w2 * 128 + c4);
-            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+            for (int jj = 0; jj < 4; ++jj) {
+                int ex = 0;
+                float mp = 1.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                gC[j] += tv[j];
-                if (w2 < warp) pre[j] += tv[j];
+                for (int p = 0; p < 8; ++p) {
+                    const uint32_t u = __float_as_uint(al[p][jj]);
+                    ex += (int)(u >> 23) - 127;
+                    mp *= __uint_as_float((u & 0x7FFFFFu) | 0x3F800000u);
+                }
+                lw[jj] = (float)ex + fast_log2(mp);
             }
-        }
-        const float4 g04 = *reinterpret_cast<const float4 *>(v_g0 + c4);
-        const float g0[4] = {g04.x, g04.y, g04.z, g04.w};
-        int wide_l = 0;
+            *reinterpret_cast<float4 *>(WT + warp * 128 + c4) = make_float4(lw[0], lw[1], lw[2], lw[3]);
+            if (warp == 0)
+                *reinterpret_cast<float4 *>(v_g0 + c4) =
+                    make_float4(fast_log2(al[0][0]), fast_log2(al[0][1]), fast_log2(al[0][2]), fast_log2(al[0][3]));
+            group_sync(BAR_A, 256);
+            if (tid == 0) mbar_arrive(misc + M1_AFREE);   // the alpha buffer has been read
+            float pre[4] = {0.f, 0.f, 0.f, 0.f}, gC[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) wide_l |= (g0[j] - gC[j] > SPAN_MAX_LOG2);
-        const bool wide = __syncthreads_or(wide_l) != 0;   // also: WT and v_g0 reads done
-        float m2[4];
+            for (int w2 = 0; w2 < 8; ++w2) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(WT + w2 * 128 + c4);
+                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) m2[j] = wide ? 0.f : 0.5f * (g0[j] + gC[j]);
-        if (warp == 0) {
-            // sS: scale of the bf16 state operand (exp(m)); sZ: scale of the TMEM state that G5
-            // accumulates into; sPost: the factor that turns the accumulated Z into the next state.
-            // Tensor-core chunk: sS = sZ = exp(m), sPost = exp(g_C - m).  Wide-span chunk: sS = 1,
-            // sZ = exp(g_C), sPost = 1 (K̃ is then exp(g_C - g) ⊙ k).
-            float sS[4], sZ[4], sP[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                sS[j] = wide ? 1.f : fast_exp2(m2[j]);
-                sZ[j] = wide ? fast_exp2(gC[j]) : sS[j];
-                sP[j] = wide ? 1.f : fast_exp2(gC[j] - m2[j]);
+                for (int jj = 0; jj < 4; ++jj) {
+                    gC[jj] += tv[jj];
+                    if (w2 < warp) pre[jj] += tv[jj];
+                }
             }
-            float *vec = reinterpret_cast<float *>(rec + R_VEC);
-            *reinterpret_cast<float4 *>(vec + c4) = make_float4(sS[0], sS[1], sS[2], sS[3]);
-            *reinterpret_cast<float4 *>(vec + 128 + c4) = make_float4(sZ[0], sZ[1], sZ[2], sZ[3]);
-            *reinterpret_cast<float4 *>(vec + 256 + c4) = make_float4(sP[0], sP[1], sP[2], sP[3]);
-        }
+            const float4 g04 = *reinterpret_cast<const float4 *>(v_g0 + c4);
+            const float g0[4] = {g04.x, g04.y, g04.z, g04.w};
+            int wide_l = 0;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) wide_l |= (g0[jj] - gC[jj] > SPAN_MAX_LOG2);
+            const bool wide = group_or(BAR_A, 256, wide_l != 0);   // also: WT and v_g0 reads done
+            float m2[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) m2[jj] = wide ? 0.f : 0.5f * (g0[jj] + gC[jj]);
+            if (warp == 0) {
+                // sS: scale of the bf16 state operand (exp(m)); sZ: scale of the TMEM state that G5
+                // accumulates into; sPost: the factor that turns the accumulated Z into the next state.
+                // Tensor-core chunk: sS = sZ = exp(m), sPost = exp(g_C - m).  Wide-span chunk: sS = 1,
+                // sZ = exp(g_C), sPost = 1 (K̃ is then exp(g_C - g) ⊙ k).
+                float sS[4], sZ[4], sP[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    sS[jj] = wide ? 1.f : fast_exp2(m2[jj]);
+                    sZ[jj] = wide ? fast_exp2(gC[jj]) : sS[jj];
+                    sP[jj] = wide ? 1.f : fast_exp2(gC[jj] - m2[jj]);
+                }
+                float *vec = reinterpret_cast<float *>(rec_of(j) + R_VEC);
+                *reinterpret_cast<float4 *>(vec + c4) = make_float4(sS[0], sS[1], sS[2], sS[3]);
+                *reinterpret_cast<float4 *>(vec + 128 + c4) = make_float4(sZ[0], sZ[1], sZ[2], sZ[3]);
+                *reinterpret_cast<float4 *>(vec + 256 + c4) = make_float4(sP[0], sP[1], sP[2], sP[3]);
+            }
 
-        // ------------------------------------------------------------------ build (in place)
-        if (!block_wait(misc + M1_LOAD, par, abort)) break;
-        {
-            uint2 rq[8], rk[8], rb[8];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int r = p0 + p;
-                rb[p] = *reinterpret_cast<const uint2 *>(sm + P1_EQ + sw_off(r, c4, 128));
-                rq[p] = *reinterpret_cast<const uint2 *>(sm + P1_EQ + sw_off(64 + r, c4, 128));
-                rk[p] = *reinterpret_cast<const uint2 *>(sm + P1_KT + sw_off(r, c4, 64));
-                const uint2 rv = *reinterpret_cast<const uint2 *>(sm + P1_U + sw_off(r, c4, 64));
-                const uint2 rw = *reinterpret_cast<const uint2 *>(sm + P1_W + sw_off(r, c4, 64));
-                *reinterpret_cast<uint2 *>(sm + P1_U + sw_off(r, c4, 64)) = make_uint2(bmul2(rw.x, rv.x), bmul2(rw.y, rv.y));
-            }
-            if (!wide) {
-                // exp(g - m) from one exponential at the thread's first position and running
-                // products of alpha after it; exp(m - g) backwards from one exponential at its last
-                // position.  Both start inside the chunk, where every factor lies within
-                // exp(+-span/2): a start before the first position (exp(-m) itself) can leave fp32's
-                // range when the chunk's first alpha is tiny.  Packed bf16 arithmetic: each factor
-                // and each product is rounded to bf16 once.
-                float f1[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) f1[j] = fast_exp2(pre[j] + fast_log2(al[0][j]) - m2[j]);
+            // ---------------------------------------------------------------- build (in place)
+            if (!gwait(misc + M1_FULL + 8 * stg, (uint32_t)((j >> 1) & 1), BAR_A, 256, abort)) break;
+            {
+                uint2 rq[8], rk[8], rb[8];
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
                     const int r = p0 + p;
-                    if (p > 0)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) f1[j] *= al[p][j];
-                    const uint32_t F01 = pack_bf16(f1[0], f1[1]), F23 = pack_bf16(f1[2], f1[3]);
-                    *reinterpret_cast<uint2 *>(sm + P1_EQ + sw_off(r, c4, 128)) =
-                        make_uint2(bmul2(bmul2(rb[p].x, rk[p].x), F01), bmul2(bmul2(rb[p].y, rk[p].y), F23));
-                    *reinterpret_cast<uint2 *>(sm + P1_EQ + sw_off(64 + r, c4, 128)) =
-                        make_uint2(bmul2(rq[p].x, F01), bmul2(rq[p].y, F23));
+                    rb[p] = *reinterpret_cast<const uint2 *>(S + P1_EQ + sw_off(r, c4, 128));
+                    rq[p] = *reinterpret_cast<const uint2 *>(S + P1_EQ + sw_off(64 + r, c4, 128));
+                    rk[p] = *reinterpret_cast<const uint2 *>(S + P1_KT + sw_off(r, c4, 64));
+                    const uint2 rv = *reinterpret_cast<const uint2 *>(S + P1_U + sw_off(r, c4, 64));
+                    const uint2 rw = *reinterpret_cast<const uint2 *>(S + P1_W + sw_off(r, c4, 64));
+                    *reinterpret_cast<uint2 *>(S + P1_U + sw_off(r, c4, 64)) = make_uint2(bmul2(rw.x, rv.x), bmul2(rw.y, rv.y));
                 }
-                float f2[4];
+                if (!wide) {
+                    // exp(g - m) from one exponential at the thread's first position and running
+                    // products of alpha after it; exp(m - g) backwards from one exponential at its last
+                    // position.  Both start inside the chunk, where every factor lies within
+                    // exp(+-span/2): a start before the first position (exp(-m) itself) can leave fp32's
+                    // range when the chunk's first alpha is tiny.  Packed bf16 arithmetic: each factor
+                    // and each product is rounded to bf16 once.
+                    float f1[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) f2[j] = fast_exp2(m2[j] - (pre[j] + lw[j]));
+                    for (int jj = 0; jj < 4; ++jj) f1[jj] = fast_exp2(pre[jj] + fast_log2(al[0][jj]) - m2[jj]);
 #pragma unroll
-                for (int p = 7; p >= 0; --p) {
-                    const int r = p0 + p;
-                    *reinterpret_cast<uint2 *>(sm + P1_KT + sw_off(r, c4, 64)) =
-                        make_uint2(bmul2(rk[p].x, pack_bf16(f2[0], f2[1])), bmul2(rk[p].y, pack_bf16(f2[2], f2[3])));
+                    for (int p = 0; p < 8; ++p) {
+                        const int r = p0 + p;
+                        if (p > 0)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) f2[j] *= al[p][j];
-                }
-            } else {
-                float run[4] = {pre[0], pre[1], pre[2], pre[3]};
-#pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    const int r = p0 + p;
-                    const float2 q01 = unpack2(rq[p].x), q23 = unpack2(rq[p].y);
-                    const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
-                    const float2 b01 = unpack2(rb[p].x), b23 = unpack2(rb[p].y);
-                    const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
-                    const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
-                    float E[4], Qh[4], Kt[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        run[j] += fast_log2(al[p][j]);
-                        const float gam = exp2f(run[j]);
-                        E[j] = bv[j] * kk[j] * gam;
-                        Qh[j] = qq[j] * gam;
-                        Kt[j] = kk[j] * exp2f(gC[j] - run[j]);
+                            for (int jj = 0; jj < 4; ++jj) f1[jj] *= al[p][jj];
+                        const uint32_t F01 = pack_bf16(f1[0], f1[1]), F23 = pack_bf16(f1[2], f1[3]);
+                        *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(r, c4, 128)) =
+                            make_uint2(bmul2(bmul2(rb[p].x, rk[p].x), F01), bmul2(bmul2(rb[p].y, rk[p].y), F23));
+                        *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(64 + r, c4, 128)) =
+                            make_uint2(bmul2(rq[p].x, F01), bmul2(rq[p].y, F23));
                     }
-                    *reinterpret_cast<uint2 *>(sm + P1_EQ + sw_off(r, c4, 128)) =
-                        make_uint2(pack_bf16(E[0], E[1]), pack_bf16(E[2], E[3]));
-                    *reinterpret_cast<uint2 *>(sm + P1_EQ + sw_off(64 + r, c4, 128)) =
-                        make_uint2(pack_bf16(Qh[0], Qh[1]), pack_bf16(Qh[2], Qh[3]));
-                    *reinterpret_cast<uint2 *>(sm + P1_KT + sw_off(r, c4, 64)) =
-                        make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
-                }
-                if (tid < 128) wide_span_ap(tmem + P1_TM_D1, q, k, b, alpha, row0, (size_t)H, tid, L);
-            }
-        }
-        fence_async_smem();
-        fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            fence_after();
-            if (!wide) {
+                    float f2[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    mma_ss(tmem + P1_TM_D1, desc_kmajor(aEQ, 128, j), desc_kmajor(aKT, 64, j), ID_G1, j > 0);
-                mma_commit(misc + M1_G1);
-            } else {
-                mbar_arrive(misc + M1_G1);   // A and P were written into D1 directly
-            }
-            bulk_s2g(rec + R_KT, aKT, 16384);   // K̃ is final
-        }
-        // the T tile's blocks above the diagonal are zero (w, which shared the tile, is consumed)
-        for (int i = tid; i < 512; i += P1_NT) reinterpret_cast<uint4 *>(sm + P1_W)[i] = make_uint4(0u, 0u, 0u, 0u);
-
-        // ------------------------------------------------------------------ A (fp32) and P (bf16) out of TMEM
-        if (!block_wait(misc + M1_G1, par, abort)) break;
-        fence_after();
-        {
-            const int rowl = 32 * (warp & 3) + lane, col0 = 32 * (warp >> 2);
-            uint32_t ra[32];
-            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + P1_TM_D1 + col0, ra);
-            wait_ld();
-            if (rowl < 64) {   // A: strictly lower
+                    for (int jj = 0; jj < 4; ++jj) f2[jj] = fast_exp2(m2[jj] - (pre[jj] + lw[jj]));
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    float4 x;
-                    x.x = col0 + i < rowl ? __uint_as_float(ra[i]) : 0.f;
-                    x.y = col0 + i + 1 < rowl ? __uint_as_float(ra[i + 1]) : 0.f;
-                    x.z = col0 + i + 2 < rowl ? __uint_as_float(ra[i + 2]) : 0.f;
-                    x.w = col0 + i + 3 < rowl ? __uint_as_float(ra[i + 3]) : 0.f;
-                    *reinterpret_cast<float4 *>(AS + rowl * LDA + col0 + i) = x;
-                }
-            } else {           // P: lower with the diagonal, rows 64-127 of the [T; P] tile
-                const int r = rowl - 64;
+                    for (int p = 7; p >= 0; --p) {
+                        const int r = p0 + p;
+                        *reinterpret_cast<uint2 *>(S + P1_KT + sw_off(r, c4, 64)) =
+                            make_uint2(bmul2(rk[p].x, pack_bf16(f2[0], f2[1])), bmul2(rk[p].y, pack_bf16(f2[2], f2[3])));
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int cc = col0 + 8 * u + 2 * i;
-                        pk[i] = pack_bf16(cc <= r ? __uint_as_float(ra[8 * u + 2 * i]) : 0.f,
-                                          cc + 1 <= r ? __uint_as_float(ra[8 * u + 2 * i + 1]) : 0.f);
+                        for (int jj = 0; jj < 4; ++jj) f2[jj] *= al[p][jj];
                     }
-                    *reinterpret_cast<uint4 *>(sm + P1_W + sw_off(64 + r, col0 + 8 * u, 128)) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                } else {
+                    float run[4] = {pre[0], pre[1], pre[2], pre[3]};
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const int r = p0 + p;
+                        const float2 q01 = unpack2(rq[p].x), q23 = unpack2(rq[p].y);
+                        const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
+                        const float2 b01 = unpack2(rb[p].x), b23 = unpack2(rb[p].y);
+                        const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
+                        const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
+                        float E[4], Qh[4], Kt[4];
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            run[jj] += fast_log2(al[p][jj]);
+                            const float gam = exp2f(run[jj]);
+                            E[jj] = bv[jj] * kk[jj] * gam;
+                            Qh[jj] = qq[jj] * gam;
+                            Kt[jj] = kk[jj] * exp2f(gC[jj] - run[jj]);
+                        }
+                        *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(r, c4, 128)) =
+                            make_uint2(pack_bf16(E[0], E[1]), pack_bf16(E[2], E[3]));
+                        *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(64 + r, c4, 128)) =
+                            make_uint2(pack_bf16(Qh[0], Qh[1]), pack_bf16(Qh[2], Qh[3]));
+                        *reinterpret_cast<uint2 *>(S + P1_KT + sw_off(r, c4, 64)) =
+                            make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
+                    }
+                    // A and P straight into D1 (this group read the previous chunk-head's out of it)
+                    if (tid < 128) wide_span_ap(d1, q, k, b, alpha, ((size_t)bb * T + t0) * H + h, (size_t)H, tid, L);
                 }
             }
-        }
-        fence_async_smem();
-        fence_before();
-        __syncthreads();
-        // ------------------------------------------------------------------ T = (I + A)^-1 (warps 4-7)
-        if (tid == 0) bulk_s2g(rec + R_P, aW + 8192, 8192);   // P is final
-        if (warp >= 4) {
-            solve_unit_lower(AS, reinterpret_cast<float *>(sm + P1_X), sm + P1_W, tid - 128, 1);
             fence_async_smem();
-        }
-        __syncthreads();
-        // ------------------------------------------------------------------ G2: W' = T Ê, Ũ = T U
-        if (tid == 0) {
-            fence_after();
+            fence_before();
+            group_sync(BAR_A, 256);
+            if (tid == 0) {
+                if (!wide) {
+                    fence_after();
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_ss(tmem + P1_TM_D2, desc_kmajor(aW, 128, j), desc_mnmajor(aEQ, 128, j), ID_G2, j > 0);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_ss(tmem + P1_TM_D3, desc_kmajor(aW, 128, j), desc_mnmajor(aU, 64, j), ID_G2, j > 0);
-            mma_commit(misc + M1_G2);
-        }
-        if (!block_wait(misc + M1_G2, par, abort)) break;
-        fence_after();
-        if ((warp & 3) < 2) {   // TMEM lanes 0-63: rows of W' (warps 0, 1) and of Ũ (warps 4, 5)
-            const int i = 32 * (warp & 3) + lane;
-            const bool isW = warp < 4;
-            const uint32_t src = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (isW ? P1_TM_D2 : P1_TM_D3);
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-                uint32_t r32[32];
-                tmem_ld32(src + 32 * u2, r32);
+                    for (int jj = 0; jj < 8; ++jj)
+                        mma_ss(d1, desc_kmajor(aEQ, 128, jj), desc_kmajor(aKT, 64, jj), ID_G1, jj > 0);
+                    mma_commit(misc + M1_G1);
+                } else {
+                    mbar_arrive(misc + M1_G1);   // A and P were written into D1 directly
+                }
+            }
+            // the T tile (w, which shared it, is consumed): zero rows 0-63, whose blocks above the diagonal
+            // the solve leaves untouched
+            for (int i = tid; i < 512; i += 256) reinterpret_cast<uint4 *>(S + P1_W)[i] = make_uint4(0u, 0u, 0u, 0u);
+            fence_async_smem();
+            // ---------------------------------------------------------------- A (fp32, for the solve) and P (bf16, to the record)
+            if (!gwait(misc + M1_G1, (uint32_t)(j & 1), BAR_A, 256, abort)) break;
+            if (j >= 1 && !gwait(misc + M1_ASFREE, (uint32_t)((j - 1) & 1), BAR_A, 256, abort)) break;
+            {
+                const int rowl = 32 * (warp & 3) + lane, col0 = 32 * (warp >> 2);
+                uint32_t x[32];
+                tmem_ld32(d1 + ((uint32_t)(32 * (warp & 3)) << 16) + col0, x);
                 wait_ld();
+                if (rowl < 64) {   // A: strictly lower
+                    float *AS = reinterpret_cast<float *>(sm + P1_AS);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        float4 v;
+                        v.x = col0 + i < rowl ? __uint_as_float(x[i]) : 0.f;
+                        v.y = col0 + i + 1 < rowl ? __uint_as_float(x[i + 1]) : 0.f;
+                        v.z = col0 + i + 2 < rowl ? __uint_as_float(x[i + 2]) : 0.f;
+                        v.w = col0 + i + 3 < rowl ? __uint_as_float(x[i + 3]) : 0.f;
+                        *reinterpret_cast<float4 *>(AS + rowl * LDA + col0 + i) = v;
+                    }
+                } else {           // P: lower with the diagonal, straight into the record's swizzled image
+                    const int r = rowl - 64;
+                    unsigned char *pdst = rec_of(j) + R_P;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int cc = col0 + 8 * u + 2 * i;
+                            pk[i] = pack_bf16(cc <= r ? __uint_as_float(x[8 * u + 2 * i]) : 0.f,
+                                              cc + 1 <= r ? __uint_as_float(x[8 * u + 2 * i + 1]) : 0.f);
+                        }
+                        *reinterpret_cast<uint4 *>(pdst + sw_off(r, col0 + 8 * u, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            fence_before();
+            group_sync(BAR_A, 256);
+            if (tid == 0) mbar_arrive(misc + M1_AREADY);   // A is in the scratch, D1 may be overwritten
+        }
+    } else {
+        // ------------------------------------------------------------------ solve group (warps 8-11)
+        const int tb = tid - 256, wb = warp - 8;   // wb = TMEM lane quarter
+        float *AS = reinterpret_cast<float *>(sm + P1_AS);
+        for (int j = 0; j < njobs; ++j) {
+            const int stg = j & 1;
+            unsigned char *S = sm + stg * P1_STAGE;
+            const uint32_t aEQ = smem_u32(S + P1_EQ), aU = smem_u32(S + P1_U), aW = smem_u32(S + P1_W);
+            if (!gwait(misc + M1_AREADY, (uint32_t)(j & 1), BAR_B, 128, abort)) break;
+            unsigned char *rec = rec_of(j);
+            if (tb == 0) {   // K̃ and Q̂ are final: out by bulk copies while the chunk is solved
+                bulk_s2g(rec + R_KT, smem_u32(S + P1_KT), 16384);
+                bulk_s2g(rec + R_A3 + 8192, aEQ + 8192, 8192);       // Q̂: rows 64-127 of both column
+                bulk_s2g(rec + R_A3 + 24576, aEQ + 24576, 8192);     // halves of [-W'; Q̂]
+            }
+            // ---------------------------------------------------------------- T = (I + A)^-1, duplicated as [T; T]
+            solve_unit_lower(AS, reinterpret_cast<float *>(sm + P1_X), S + P1_W, tb, BAR_B);
+            group_sync(BAR_B, 128);
+            if (tb == 0) mbar_arrive(misc + M1_ASFREE);   // the A scratch may take the next chunk-head's A
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {   // rows 64-127 = rows 0-63: W' and Ũ land in all 128 TMEM lanes
+                const int idx = tb + 128 * i;
+                reinterpret_cast<uint4 *>(S + P1_W + 8192)[idx] = reinterpret_cast<const uint4 *>(S + P1_W)[idx];
+            }
+            fence_async_smem();
+            group_sync(BAR_B, 128);
+            // ---------------------------------------------------------------- G2: [W'; W'] = [T; T] Ê, [Ũ; Ũ] = [T; T] U
+            if (tb == 0) {
+                fence_after();
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    mma_ss(tmem + P1_TM_D2, desc_kmajor(aW, 128, jj), desc_mnmajor(aEQ, 128, jj), ID_G2, jj > 0);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    mma_ss(tmem + P1_TM_D3, desc_kmajor(aW, 128, jj), desc_mnmajor(aU, 64, jj), ID_G2, jj > 0);
+                mma_commit(misc + M1_G2);
+            }
+            if (!gwait(misc + M1_G2, (uint32_t)(j & 1), BAR_B, 128, abort)) break;
+            {   // lanes 0-63 (warps 8, 9): -W' rows into the [-W'; Q̂] tile; lanes 64-127 (warps 10, 11): the
+                // same rows of Ũ into the U tile; bf16
+                const int i = 32 * (wb & 1) + lane;
+                const bool isW = wb < 2;
+                const uint32_t src = tmem + ((uint32_t)(32 * wb) << 16) + (isW ? P1_TM_D2 : P1_TM_D3);
+                unsigned char *dst = S + (isW ? P1_EQ : P1_U);
                 const float sg = isW ? -1.f : 1.f;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int cc = 32 * u2 + 8 * u;
-                    const uint32_t *x = r32 + 8 * u;
-                    const uint4 pk = make_uint4(pack_bf16(sg * __uint_as_float(x[0]), sg * __uint_as_float(x[1])),
-                                                pack_bf16(sg * __uint_as_float(x[2]), sg * __uint_as_float(x[3])),
-                                                pack_bf16(sg * __uint_as_float(x[4]), sg * __uint_as_float(x[5])),
-                                                pack_bf16(sg * __uint_as_float(x[6]), sg * __uint_as_float(x[7])));
-                    if (isW)
-                        *reinterpret_cast<uint4 *>(sm + P1_EQ + sw_off(i, cc, 128)) = pk;
-                    else
-                        *reinterpret_cast<uint4 *>(sm + P1_U + sw_off(i, cc, 64)) = pk;
+                for (int u2 = 0; u2 < 4; u2 += 2) {
+                    uint32_t x0[32], x1[32];
+                    tmem_ld32(src + 32 * u2, x0);
+                    tmem_ld32(src + 32 * u2 + 32, x1);
+                    wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int cc = 32 * u2 + 8 * u;
+                        const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
+                        const uint4 pk = make_uint4(pack_bf16(sg * __uint_as_float(x[0]), sg * __uint_as_float(x[1])),
+                                                    pack_bf16(sg * __uint_as_float(x[2]), sg * __uint_as_float(x[3])),
+                                                    pack_bf16(sg * __uint_as_float(x[4]), sg * __uint_as_float(x[5])),
+                                                    pack_bf16(sg * __uint_as_float(x[6]), sg * __uint_as_float(x[7])));
+                        *reinterpret_cast<uint4 *>(dst + sw_off(i, cc, isW ? 128 : 64)) = pk;
+                    }
                 }
             }
+            fence_async_smem();
+            fence_before();
+            group_sync(BAR_B, 128);
+            if (tb == 0) {   // -W' (rows 0-63 of both column halves) and Ũ out; the stage is free once every
+                             // store of the record has read it
+                bulk_s2g(rec + R_A3, aEQ, 8192);
+                bulk_s2g(rec + R_A3 + 16384, aEQ + 16384, 8192);
+                bulk_s2g(rec + R_U, aU, 16384);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive(misc + M1_OUT + 8 * stg);
+            }
         }
-        fence_async_smem();
-        fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_s2g(rec + R_A3, aEQ, 32768);
-            bulk_s2g(rec + R_U, aU, 16384);
+        if (tb == 0) {   // the record stores complete before the block exits
             bulk_commit();
+            bulk_wait_all();
         }
     }
-    if (tid == 0) bulk_wait_all();   // the record stores complete before the block exits
     fence_before();
     __syncthreads();
     fence_after();
@@ -459,17 +550,20 @@ __global__ void __launch_bounds__(P1_NT, 2)
 }
 
 // ---------------------------------------------------------------------------- stage 2
-constexpr int W2_NT = 256;
+// Warps 0-7 walk the chain: TMEM lane quarter w % 4, value-column half w / 4.  All eight rescale the
+// state; warps 0, 1, 4, 5 (lanes 0-63) form Delta; warps 2, 3, 6, 7 (lanes 64-127) write the o rows
+// of the previous chunk while Delta is formed.  Warp 8 issues the record copies.
+constexpr int W2_NT = 288;
 constexpr uint32_t W2_S = 0;                          // Z̃ bf16 [c x v] (MN-major B of G3)
 constexpr uint32_t W2_DL = 32768;                     // Delta bf16 [i x v]
 constexpr uint32_t W2_SLOT = 49152;                   // 2 record slots
 constexpr uint32_t W2_OST = W2_SLOT + 2 * R_BYTES;    // o rows staged for the TMA store (16 KB)
 constexpr uint32_t W2_MISC = W2_OST + 16384;
 constexpr uint32_t W2_BYTES = W2_MISC + 256 + 1024;
-// mbarriers: FULL and G45 per slot, D3FREE per accumulator buffer, G3
-enum : uint32_t { M2_FULL = 0, M2_G45 = 16, M2_D3FREE = 32, M2_G3 = 48, M2_TSLOT = 64, M2_ABORT = 68 };
+// mbarriers: FULL and G45 per slot, G3
+enum : uint32_t { M2_FULL = 0, M2_G45 = 16, M2_G3 = 32, M2_TSLOT = 48, M2_ABORT = 52 };
 constexpr uint32_t W2_TM_Z = 0, W2_TM_D3 = 128, W2_TM_COLS = 512;   // D3 buffers at 128 and 256
-constexpr uint32_t BAR_STATE = 1, BAR_O = 2;
+constexpr uint32_t BAR_ALL = 1, BAR_DELTA = 2, BAR_O = 3;            // named barriers (128 or 256 threads)
 
 __device__ __forceinline__ bool group_wait2(uint32_t mb, uint32_t parity, uint32_t bar, uint32_t n,
                                             volatile uint32_t *abort) {
@@ -488,6 +582,37 @@ __device__ __forceinline__ bool thread_wait(uint32_t mb, uint32_t parity, volati
     return true;
 }
 
+// o rows of one chunk (TMEM lanes 64-127 of its D3 buffer, value columns cb .. cb + 63) -> bf16 staging
+// tile -> TMA store; rows past the end of the sequence are clipped by the copy.  ot: 0..127 over
+// warps 2, 3, 6, 7.
+__device__ __forceinline__ void store_o(const CUtensorMap *map_o, unsigned char *sm, uint32_t d3, int ot, int r,
+                                        int cb, int h, int t0, int bb) {
+    if (ot == 0) bulk_wait_read_all();   // the previous chunk's o store has read the staging tile
+    group_sync(BAR_O, 128);
+    uint32_t x0[32], x1[32];
+    const uint32_t src = d3 + ((uint32_t)(64 + (r & ~31)) << 16) + cb;
+    tmem_ld32(src, x0);
+    tmem_ld32(src + 32, x1);
+    wait_ld();
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
+        const uint4 pk = make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                                    pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                                    pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                                    pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+        *reinterpret_cast<uint4 *>(sm + W2_OST + sw_off(r, cb + 8 * u, 64)) = pk;
+    }
+    fence_before();
+    fence_async_smem();
+    group_sync(BAR_O, 128);
+    if (ot == 0) {
+        tma_store_4d(map_o, 0, h, t0, bb, smem_u32(sm + W2_OST));
+        tma_store_4d(map_o, 64, h, t0, bb, smem_u32(sm + W2_OST + 8192));
+        bulk_commit();
+    }
+}
+
 __global__ void __launch_bounds__(W2_NT, 1)
     walk_kernel(const __grid_constant__ CUtensorMap map_o, const unsigned char *records, const float *S0, float *ST,
                 int H, int T, int n0, int nw, unsigned int *status) {
@@ -503,7 +628,6 @@ __global__ void __launch_bounds__(W2_NT, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(misc + M2_FULL + 8 * s, 1);
             mbar_init(misc + M2_G45 + 8 * s, 1);
-            mbar_init(misc + M2_D3FREE + 8 * s, 64);
         }
         mbar_init(misc + M2_G3, 1);
         *abort = 0u;
@@ -518,14 +642,16 @@ __global__ void __launch_bounds__(W2_NT, 1)
     auto d3 = [&](int n) { return tmem + W2_TM_D3 + 128u * (uint32_t)(n & 1); };
     auto rec_of = [&](int nl) { return records + ((size_t)(bb * nw + nl) * H + h) * R_BYTES; };
 
-    if (warp < 4) {
-        // ------------------------------------------------------------------ state group: rows c of Z
-        const int crow = tid;
-        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    if (warp < 8) {
+        const int q4 = warp & 3, cb = 64 * (warp >> 2);   // TMEM lane quarter, value-column half
+        const int crow = 32 * q4 + lane;                  // row c of Z (and row of D3)
+        const uint32_t lq = (uint32_t)(32 * q4) << 16;
+        const bool is_delta = q4 < 2;
+        const int ot = 32 * (q4 - 2) + lane + 64 * (warp >> 2);   // o warps: 0..127
         {   // Z <- S0 (or 0); the first rescale multiplies by chunk 0's exp(m)
-            const float *src = S0 ? S0 + ((size_t)chain * KD + crow) * VD : nullptr;
+            const float *src = S0 ? S0 + ((size_t)chain * KD + crow) * VD + cb : nullptr;
 #pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
+            for (int u2 = 0; u2 < 2; ++u2) {
                 uint32_t r32[32];
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
@@ -533,148 +659,135 @@ __global__ void __launch_bounds__(W2_NT, 1)
                     r32[i] = __float_as_uint(x.x); r32[i + 1] = __float_as_uint(x.y);
                     r32[i + 2] = __float_as_uint(x.z); r32[i + 3] = __float_as_uint(x.w);
                 }
-                tmem_st32(tmem + lrow + W2_TM_Z + 32 * u2, r32);
+                tmem_st32(tmem + lq + W2_TM_Z + cb + 32 * u2, r32);
             }
             wait_st();
         }
         float egm_prev = 1.f;
         bool ok = true;
-        for (int nl = 0; nl < nw && ok; ++nl) {
-            const uint32_t slot = slot_addr(nl);
-            const float *vec = reinterpret_cast<const float *>(sm + slot + R_VEC);
-            if (!group_wait2(misc + M2_FULL + 8 * (nl & 1), (uint32_t)((nl >> 1) & 1), BAR_STATE, 128, abort)) { ok = false; break; }
-            if (nl > 0 && !group_wait2(misc + M2_G45 + 8 * ((nl - 1) & 1), (uint32_t)(((nl - 1) >> 1) & 1), BAR_STATE, 128, abort)) { ok = false; break; }
-            // S_n = sPost_{n-1} Z, then Z <- sZ_n S_n and the bf16 operand sS_n S_n; the factors are
-            // applied one after the other (their product alone can lie below fp32's range)
-            const float post = egm_prev, ssc = vec[crow], zsc = vec[128 + crow];
-            egm_prev = vec[256 + crow];
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-                uint32_t r32[32];
-                tmem_ld32(tmem + lrow + W2_TM_Z + 32 * u2, r32);
-                wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(post * __uint_as_float(r32[i]));
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float *x = reinterpret_cast<const float *>(r32) + 8 * u;
-                    const uint4 pk = make_uint4(pack_bf16(ssc * x[0], ssc * x[1]), pack_bf16(ssc * x[2], ssc * x[3]),
-                                                pack_bf16(ssc * x[4], ssc * x[5]), pack_bf16(ssc * x[6], ssc * x[7]));
-                    *reinterpret_cast<uint4 *>(sm + W2_S + sw_off(crow, 32 * u2 + 8 * u, 128)) = pk;
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(zsc * __uint_as_float(r32[i]));
-                tmem_st32(tmem + lrow + W2_TM_Z + 32 * u2, r32);
-            }
-            wait_st();
-            fence_async_smem();
-            fence_before();
-            group_sync(BAR_STATE, 128);
-            if (tid == 0) {   // G3: [-W'Z̃; Q̂Z̃] into D3 of this chunk, once its o rows of chunk n-2 are out
-                fence_after();
-                if (nl < 2 || thread_wait(misc + M2_D3FREE + 8 * (nl & 1), (uint32_t)(((nl - 2) >> 1) & 1), abort)) {
-                    const uint32_t aA3 = smem_u32(sm + slot + R_A3), aS = smem_u32(sm + W2_S);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        mma_ss(d3(nl), desc_kmajor(aA3, 128, j), desc_mnmajor(aS, 128, j), ID_G3, j > 0);
-                    mma_commit(misc + M2_G3);
-                }
-            }
-            if (!group_wait2(misc + M2_G3, (uint32_t)(nl & 1), BAR_STATE, 128, abort)) { ok = false; break; }
-            if (warp < 2) {   // Delta = Ũ - W'Z̃ (rows i < 64) -> bf16 tile
-                const unsigned char *Ut = sm + slot + R_U;
-#pragma unroll
-                for (int u2 = 0; u2 < 4; ++u2) {
-                    uint32_t r32[32];
-                    tmem_ld32(d3(nl) + lrow + 32 * u2, r32);
-                    wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int vv = 32 * u2 + 8 * u;
-                        const uint4 ut = *reinterpret_cast<const uint4 *>(Ut + sw_off(crow, vv, 64));
-                        const float2 a = unpack2(ut.x), b2 = unpack2(ut.y), c2 = unpack2(ut.z), d2 = unpack2(ut.w);
-                        const float *x = reinterpret_cast<const float *>(r32) + 8 * u;
-                        const uint4 pk = make_uint4(pack_bf16(a.x + x[0], a.y + x[1]), pack_bf16(b2.x + x[2], b2.y + x[3]),
-                                                    pack_bf16(c2.x + x[4], c2.y + x[5]), pack_bf16(d2.x + x[6], d2.y + x[7]));
-                        *reinterpret_cast<uint4 *>(sm + W2_DL + sw_off(crow, vv, 64)) = pk;
-                    }
-                }
-            }
-            fence_async_smem();
-            fence_before();
-            group_sync(BAR_STATE, 128);
-            if (tid == 0) {   // G4: O += P Delta (rows 0-63 of the A tile are Ũ's bytes: their products
-                              // land in the Delta rows of D3, already read); G5: Z += K̃^T Delta
-                fence_after();
-                const uint32_t aPA = smem_u32(sm + slot + R_P - 8192), aKT = smem_u32(sm + slot + R_KT),
-                               aDL = smem_u32(sm + W2_DL);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) mma_ss(d3(nl), desc_kmajor(aPA, 128, j), desc_mnmajor(aDL, 64, j), ID_G4, 1);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_ss(tmem + W2_TM_Z, desc_mnmajor(aKT, 64, j), desc_mnmajor(aDL, 64, j), ID_G5, 1);
-                mma_commit(misc + M2_G45 + 8 * (nl & 1));
-            }
-        }
-        // S_T = Diag(sPost) Z of the last chunk, once its G4/G5 are complete
-        if (ok && group_wait2(misc + M2_G45 + 8 * ((nw - 1) & 1), (uint32_t)(((nw - 1) >> 1) & 1), BAR_STATE, 128, abort)) {
-            float *dst = ST + ((size_t)chain * KD + crow) * VD;
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-                uint32_t r32[32];
-                tmem_ld32(tmem + lrow + W2_TM_Z + 32 * u2, r32);
-                wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4 *>(dst + 32 * u2 + i) =
-                        make_float4(egm_prev * __uint_as_float(r32[i]), egm_prev * __uint_as_float(r32[i + 1]),
-                                    egm_prev * __uint_as_float(r32[i + 2]), egm_prev * __uint_as_float(r32[i + 3]));
-            }
-        }
-    } else if (warp == 4) {
-        // ------------------------------------------------------------------ producer: one bulk copy per record
-        if (lane == 0) {
-            for (int nl = 0; nl < nw; ++nl) {
-                if (nl >= 2 && !thread_wait(misc + M2_G45 + 8 * (nl & 1), (uint32_t)(((nl - 2) >> 1) & 1), abort)) break;
-                mbar_arrive_expect_tx(misc + M2_FULL + 8 * (nl & 1), R_COPY);
-                bulk_g2s(smem_u32(sm + slot_addr(nl)), rec_of(nl), R_COPY, misc + M2_FULL + 8 * (nl & 1));
-            }
-        }
-    } else if (warp >= 6) {
-        // ------------------------------------------------------------------ o group: TMEM lanes 64-127 of D3
-        const int ot = tid - 192;   // O row of the chunk
-        const uint32_t lrow = (uint32_t)(64 + 32 * (warp - 6)) << 16;
         for (int nl = 0; nl < nw; ++nl) {
-            const int t0 = (n0 + nl) * C;
-            if (!group_wait2(misc + M2_G45 + 8 * (nl & 1), (uint32_t)((nl >> 1) & 1), BAR_O, 64, abort)) break;
-            if (ot == 0) bulk_wait_read_all();   // the previous chunk's o store has read the staging tile
-            group_sync(BAR_O, 64);
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-                uint32_t r32[32];
-                tmem_ld32(d3(nl) + lrow + 32 * u2, r32);
+            const uint32_t slot = slot_addr(nl);
+            // ---------------------------------------------------------------- record n in, chunk n-1 done
+            {
+                bool w_ok = mbar_wait(misc + M2_FULL + 8 * (nl & 1), (uint32_t)((nl >> 1) & 1), WAIT_LIMIT);
+                if (nl > 0)
+                    w_ok = w_ok && mbar_wait(misc + M2_G45 + 8 * ((nl - 1) & 1), (uint32_t)(((nl - 1) >> 1) & 1), WAIT_LIMIT);
+                w_ok = w_ok && !*abort;
+                const bool fail = group_or(BAR_ALL, 256, !w_ok);
+                fence_after();
+                if (fail) { *abort = 1u; ok = false; break; }
+            }
+            // ---------------------------------------------------------------- S_n = sPost_{n-1} Z; Z <- sZ_n S_n; Z̃ = bf16(sS_n S_n)
+            // (the factors are applied one after the other: their product alone can lie below fp32's range)
+            {
+                const float *vec = reinterpret_cast<const float *>(sm + slot + R_VEC);
+                const float post = egm_prev, ssc = vec[crow], zsc = vec[128 + crow];
+                egm_prev = vec[256 + crow];
+                uint32_t x0[32], x1[32];
+                tmem_ld32(tmem + lq + W2_TM_Z + cb, x0);
+                tmem_ld32(tmem + lq + W2_TM_Z + cb + 32, x1);
                 wait_ld();
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t *x = r32 + 8 * u;
-                    const uint4 pk = make_uint4(pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
-                                                pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
-                                                pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
-                                                pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
-                    *reinterpret_cast<uint4 *>(sm + W2_OST + sw_off(ot, 32 * u2 + 8 * u, 64)) = pk;
+                for (int i = 0; i < 32; ++i) {
+                    x0[i] = __float_as_uint(post * __uint_as_float(x0[i]));
+                    x1[i] = __float_as_uint(post * __uint_as_float(x1[i]));
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
+                    const uint4 pk = make_uint4(pack_bf16(ssc * __uint_as_float(x[0]), ssc * __uint_as_float(x[1])),
+                                                pack_bf16(ssc * __uint_as_float(x[2]), ssc * __uint_as_float(x[3])),
+                                                pack_bf16(ssc * __uint_as_float(x[4]), ssc * __uint_as_float(x[5])),
+                                                pack_bf16(ssc * __uint_as_float(x[6]), ssc * __uint_as_float(x[7])));
+                    *reinterpret_cast<uint4 *>(sm + W2_S + sw_off(crow, cb + 8 * u, 128)) = pk;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    x0[i] = __float_as_uint(zsc * __uint_as_float(x0[i]));
+                    x1[i] = __float_as_uint(zsc * __uint_as_float(x1[i]));
+                }
+                tmem_st32(tmem + lq + W2_TM_Z + cb, x0);
+                tmem_st32(tmem + lq + W2_TM_Z + cb + 32, x1);
+                wait_st();
+            }
+            fence_async_smem();
+            fence_before();
+            group_sync(BAR_ALL, 256);
+            if (tid == 0) {   // G3: [-W'Z̃; Q̂Z̃] into this chunk's D3 buffer (its o rows of chunk n-2 are out)
+                fence_after();
+                const uint32_t aA3 = smem_u32(sm + slot + R_A3), aS = smem_u32(sm + W2_S);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    mma_ss(d3(nl), desc_kmajor(aA3, 128, j), desc_mnmajor(aS, 128, j), ID_G3, j > 0);
+                mma_commit(misc + M2_G3);
+            }
+            if (!is_delta) {
+                // ------------------------------------------------------------ o rows of chunk n-1
+                if (nl > 0) store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + nl - 1) * C, bb);
+            } else {
+                // ------------------------------------------------------------ Delta = Ũ - W'Z̃ -> bf16 tile; G4/G5
+                if (!group_wait2(misc + M2_G3, (uint32_t)(nl & 1), BAR_DELTA, 128, abort)) continue;
+                const unsigned char *Ut = sm + slot + R_U;
+                uint32_t x0[32], x1[32];
+                tmem_ld32(d3(nl) + lq + cb, x0);
+                tmem_ld32(d3(nl) + lq + cb + 32, x1);
+                wait_ld();
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int vv = cb + 8 * u;
+                    const uint4 ut = *reinterpret_cast<const uint4 *>(Ut + sw_off(crow, vv, 64));
+                    const float2 a = unpack2(ut.x), b2 = unpack2(ut.y), c2 = unpack2(ut.z), d2 = unpack2(ut.w);
+                    const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
+                    const uint4 pk = make_uint4(
+                        pack_bf16(a.x + __uint_as_float(x[0]), a.y + __uint_as_float(x[1])),
+                        pack_bf16(b2.x + __uint_as_float(x[2]), b2.y + __uint_as_float(x[3])),
+                        pack_bf16(c2.x + __uint_as_float(x[4]), c2.y + __uint_as_float(x[5])),
+                        pack_bf16(d2.x + __uint_as_float(x[6]), d2.y + __uint_as_float(x[7])));
+                    *reinterpret_cast<uint4 *>(sm + W2_DL + sw_off(crow, vv, 64)) = pk;
+                }
+                fence_async_smem();
+                fence_before();
+                group_sync(BAR_DELTA, 128);
+                if (tid == 0) {   // G4: O += P Delta (rows 0-63 of the A tile are Ũ's bytes: their products
+                                  // land in the Delta rows of D3, already read); G5: Z += K̃^T Delta
+                    fence_after();
+                    const uint32_t aPA = smem_u32(sm + slot + R_P - 8192), aKT = smem_u32(sm + slot + R_KT),
+                                   aDL = smem_u32(sm + W2_DL);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) mma_ss(d3(nl), desc_kmajor(aPA, 128, j), desc_mnmajor(aDL, 64, j), ID_G4, 1);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mma_ss(tmem + W2_TM_Z, desc_mnmajor(aKT, 64, j), desc_mnmajor(aDL, 64, j), ID_G5, 1);
+                    mma_commit(misc + M2_G45 + 8 * (nl & 1));
                 }
             }
-            fence_before();
-            mbar_arrive(misc + M2_D3FREE + 8 * (nl & 1));
-            fence_async_smem();
-            group_sync(BAR_O, 64);
-            if (ot == 0) {   // rows past the end of the sequence are clipped by the copy
-                tma_store_4d(&map_o, 0, h, t0, bb, smem_u32(sm + W2_OST));
-                tma_store_4d(&map_o, 64, h, t0, bb, smem_u32(sm + W2_OST + 8192));
-                bulk_commit();
+        }
+        // the last chunk: its o rows, then S_T = Diag(sPost) Z, once its G4/G5 are complete
+        if (ok && group_wait2(misc + M2_G45 + 8 * ((nw - 1) & 1), (uint32_t)(((nw - 1) >> 1) & 1), BAR_ALL, 256, abort)) {
+            if (!is_delta) store_o(&map_o, sm, d3(nw - 1), ot, crow - 64, cb, h, (n0 + nw - 1) * C, bb);
+            float *dst = ST + ((size_t)chain * KD + crow) * VD + cb;
+            uint32_t x0[32], x1[32];
+            tmem_ld32(tmem + lq + W2_TM_Z + cb, x0);
+            tmem_ld32(tmem + lq + W2_TM_Z + cb + 32, x1);
+            wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                *reinterpret_cast<float4 *>(dst + i) =
+                    make_float4(egm_prev * __uint_as_float(x0[i]), egm_prev * __uint_as_float(x0[i + 1]),
+                                egm_prev * __uint_as_float(x0[i + 2]), egm_prev * __uint_as_float(x0[i + 3]));
+                *reinterpret_cast<float4 *>(dst + 32 + i) =
+                    make_float4(egm_prev * __uint_as_float(x1[i]), egm_prev * __uint_as_float(x1[i + 1]),
+                                egm_prev * __uint_as_float(x1[i + 2]), egm_prev * __uint_as_float(x1[i + 3]));
             }
         }
-        if (ot == 0) bulk_wait_all();
+        if (!is_delta && ot == 0) bulk_wait_all();   // the o stores complete before the block exits
+    } else if (lane == 0) {
+        // ------------------------------------------------------------------ producer: one bulk copy per record
+        for (int nl = 0; nl < nw; ++nl) {
+            if (nl >= 2 && !thread_wait(misc + M2_G45 + 8 * (nl & 1), (uint32_t)(((nl - 2) >> 1) & 1), abort)) break;
+            mbar_arrive_expect_tx(misc + M2_FULL + 8 * (nl & 1), R_COPY);
+            bulk_g2s(smem_u32(sm + slot_addr(nl)), rec_of(nl), R_COPY, misc + M2_FULL + 8 * (nl & 1));
+        }
     }
     fence_before();
     __syncthreads();
@@ -702,16 +815,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A [B, T, H, 128] bf16 token tensor as the 4-D map (d, H, T, B) with a 64 x 1 x 64 x 1 box in the
-// 128-byte swizzle: one box is the 64 x 64 half-tile of the operand layout.  Rows past T read as zero.
-bool token_map(CUtensorMap *m, const void *base, int B, int T, int H) {
+// A [B, T, H, 128] token tensor as the 4-D map (d, H, T, B).  bf16: a 64 x 1 x 64 x 1 box in the 128-byte
+// swizzle, one box being the 64 x 64 half-tile of the operand layout; fp32 (alpha): a 128 x 1 x 64 x 1
+// box, rows of 512 bytes.  Rows past T read as zero.
+bool token_map(CUtensorMap *m, const void *base, int B, int T, int H, bool fp32 = false) {
     const EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const cuuint64_t es_bytes = fp32 ? 4 : 2;
     const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {256, 256ull * H, 256ull * H * T};
-    const cuuint32_t box[4] = {64, 1, 64, 1}, es[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const cuuint64_t strides[3] = {128 * es_bytes, 128 * es_bytes * H, 128 * es_bytes * H * T};
+    const cuuint32_t box[4] = {fp32 ? 128u : 64u, 1, 64, 1}, es[4] = {1, 1, 1, 1};
+    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
+              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              fp32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -736,7 +852,8 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
     split::TokMaps maps;
     CUtensorMap map_o;
     if (!token_map(&maps.q, q, B, T, H) || !token_map(&maps.k, k, B, T, H) || !token_map(&maps.b, b, B, T, H) ||
-        !token_map(&maps.v, v, B, T, H) || !token_map(&maps.w, w, B, T, H) || !token_map(&map_o, o, B, T, H))
+        !token_map(&maps.v, v, B, T, H) || !token_map(&maps.w, w, B, T, H) ||
+        !token_map(&maps.alpha, alpha, B, T, H, true) || !token_map(&map_o, o, B, T, H))
         return -6;
     const int smem1 = (int)split::P1_BYTES, smem2 = (int)split::W2_BYTES;
     if (cudaFuncSetAttribute(split::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess ||
@@ -749,9 +866,9 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
     const int NC = (T + split::C - 1) / split::C;
     for (int n0 = 0; n0 < NC; n0 += kWindowChunks) {
         const int nw = std::min(kWindowChunks, NC - n0), nch = B * H * nw;
-        split::prep_kernel<<<std::min(nch, 2 * nsm), split::P1_NT, smem1, st>>>(
+        split::prep_kernel<<<std::min(nch, nsm), split::P1_NT, smem1, st>>>(
             maps, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)b, alpha, records, H, T,
-            NC, n0, nw, nch, status);
+            n0, nw, nch, status);
         split::walk_kernel<<<B * H, split::W2_NT, smem2, st>>>(map_o, records, n0 == 0 ? S0 : ST, ST, H, T, n0, nw,
                                                                status);
     }

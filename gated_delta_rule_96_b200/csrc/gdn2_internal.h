@@ -36,6 +36,10 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
                        const void *w, const float *S0, void *o, float *ST, int B, int H, int T, void *ws,
                        cudaStream_t st);
 
+// Measurement kernel of the prefill's tensor-core phases (mode 0: back to back; 1: each group waits
+// for the previous one), `reps` chunks per CTA on `nctas` CTAs.
+int launch_phase_probe(int mode, int reps, int nctas, unsigned int *status, cudaStream_t st);
+
 // Backward pass (three sequential passes per chain; fp32 gradients; d_k, d_v in {64, 128}).
 size_t bwd_workspace_bytes(int B, int H, int T, int K, int V);
 int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,

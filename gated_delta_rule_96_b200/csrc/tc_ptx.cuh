@@ -185,6 +185,12 @@ __device__ __forceinline__ void tma_store_4d(const void *map, int c0, int c1, in
                  "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src_smem)
                  : "memory");
 }
+// L2 prefetch of a 4-D box through a tensor map (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_4d(const void *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(map), "r"(c0),
+                 "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
 // Brings a tensor map (a kernel parameter, by address) into the descriptor cache.
 __device__ __forceinline__ void prefetch_tmap(const void *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

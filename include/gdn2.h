@@ -163,6 +163,20 @@ GDN2_API int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const f
                             int T, int d_k, int d_v, int dtype, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/*
+ * Measurement aid (not part of the recurrence): runs the tensor-core products of one chunk of the
+ * chunkwise prefill -- G1 [A; P] = [Ê; Q̂] K̃^T (M128 N64 K128), G2 (2 x M128 N128 K64), G3 (M128 N128
+ * K128), G4 and G5 (2 x M128 N128 K64), with the prefill kernels' shapes and shared-memory operand
+ * layouts -- `reps` chunks in a row on each of `nctas` CTAs (one per SM), on operands that stay in
+ * shared memory; 14,680,064 flops per chunk as issued.  mode 0 issues every product back to back
+ * (the tensor pipe's rate on these shapes); mode 1 lets each group wait for the completion of the
+ * one before it, as the prefill's data flow does.  Time it with events on `stream`.  The workspace
+ * holds only the 256-byte status header (zeroed once); a bounded wait that expires sets it.
+ */
+#define GDN2_PHASE_PROBE_FLOPS_PER_CHUNK 14680064.0
+GDN2_API int gdn2_gemm_phase_probe(int mode, int reps, int nctas, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
 /* Reads the device status word of a workspace (synchronises `stream` first).
  * *out receives 0 when every kernel that used this workspace finished normally, or a
  * nonzero code naming the first internal error.  With clear != 0 the word is reset.

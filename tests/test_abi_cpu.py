@@ -27,7 +27,7 @@ def test_header_declares_entry_points():
     for name in ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_fwd_workspace_bytes", "gdn2_status_str",
                  "gdn2_workspace_status", "gdn2_chunk_fwd_path", "gdn2_chunk_fwd_edges",
                  "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
-                 "gdn2_chunk_fwd_noalloc"):
+                 "gdn2_chunk_fwd_noalloc", "gdn2_gemm_phase_probe"):
         assert name in syms
 
 
@@ -253,3 +253,13 @@ def test_library_is_standalone():
     assert needed, out
     for lib_name in needed:
         assert not re.search(r"torch|c10|python|cudart", lib_name), lib_name
+
+
+def test_phase_probe_validation(lib):
+    ws = ctypes.c_void_p(0x10000)   # never dereferenced: every case fails validation first
+    assert lib.gdn2_gemm_phase_probe(2, 1, 1, ws, 256, None) == -2
+    assert lib.gdn2_gemm_phase_probe(0, 0, 1, ws, 256, None) == -2
+    assert lib.gdn2_gemm_phase_probe(0, 1, 0, ws, 256, None) == -2
+    assert lib.gdn2_gemm_phase_probe(0, 1, 1, None, 256, None) == -5
+    assert lib.gdn2_gemm_phase_probe(0, 1, 1, ws, 255, None) == -5
+    assert lib.gdn2_gemm_phase_probe(1, 1, 1, ctypes.c_void_p(0x10004), 256, None) == -7
