@@ -27,12 +27,13 @@ bool use_tc(int B, int H, int T, int K, int V, int C, int dtype) {
 }
 
 // Implementation for these sizes: 0 = CUDA-core two-kernel path; 1 = fused tcgen05 kernel (one CTA
-// per chain, the chain cut into segments in time when there are few long chains); 2 = two-stage
-// tcgen05 path (intra-chunk work parallel over every chunk-head, then the state chain), taken when
-// there are more chains than the fused kernel's segmentation serves.
+// per chain), for up to 64 chains of fewer than 32 chunks; 2 = two-stage tcgen05 path (intra-chunk
+// work parallel over every chunk-head, then the state chain, cut into segments in time when there
+// are few long chains), for everything else.
 int select_path(int B, int H, int T, int K, int V, int C, int dtype) {
     if (!use_tc(B, H, T, K, V, C, dtype)) return 0;
-    return (long long)B * H > 64 ? 2 : 1;
+    const long long chains = (long long)B * H, NC = (T + 63) / 64;
+    return chains > 64 || NC >= 32 ? 2 : 1;
 }
 
 }  // namespace

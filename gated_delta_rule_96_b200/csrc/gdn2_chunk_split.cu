@@ -613,13 +613,27 @@ __device__ __forceinline__ void store_o(const CUtensorMap *map_o, unsigned char 
     }
 }
 
+// Launch flags of the segmented walk (few long chains): block blockIdx.x walks segment
+// blockIdx.x % nseg (chunks [seg * seg_len, (seg + 1) * seg_len) of the window) of chain
+// blockIdx.x / nseg; S0 and S_T are then indexed by block.
+enum : uint32_t {
+    WALK_ZERO_WRITES = 1,   // Ũ = 0: the walk propagates the state only (the segment's homogeneous map)
+    WALK_SKIP_O = 2,        // o is not stored
+    WALK_IDENTITY_S0 = 4,   // the segment starts from S = I (d_k = d_v)
+    WALK_ST_LAST = 8,       // only the chain's last segment stores S_T, at S_T[chain]
+};
+
 __global__ void __launch_bounds__(W2_NT, 1)
     walk_kernel(const __grid_constant__ CUtensorMap map_o, const unsigned char *records, const float *S0, float *ST,
-                int H, int T, int n0, int nw, unsigned int *status) {
+                int H, int T, int n0, int nw, int nseg, int seg_len, uint32_t flags, unsigned int *status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int chain = blockIdx.x, bb = chain / H, h = chain % H;
+    const int chain = blockIdx.x / nseg, seg = blockIdx.x % nseg, bb = chain / H, h = chain % H;
+    const int c0 = seg * seg_len, nc = min(nw, c0 + seg_len) - c0;   // this block's chunks of the window
+    const bool zero_writes = (flags & WALK_ZERO_WRITES) != 0, store_out = (flags & WALK_SKIP_O) == 0;
+    float *st_dst = (flags & WALK_ST_LAST) ? (seg == nseg - 1 ? ST + (size_t)chain * KD * VD : nullptr)
+                                           : ST + (size_t)blockIdx.x * KD * VD;
     const uint32_t misc = smem_u32(sm + W2_MISC);
     volatile uint32_t *abort = reinterpret_cast<volatile uint32_t *>(sm + W2_MISC + M2_ABORT);
 
@@ -640,7 +654,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + W2_MISC + M2_TSLOT);
     auto slot_addr = [&](int n) { return W2_SLOT + (uint32_t)(n & 1) * R_BYTES; };
     auto d3 = [&](int n) { return tmem + W2_TM_D3 + 128u * (uint32_t)(n & 1); };
-    auto rec_of = [&](int nl) { return records + ((size_t)(bb * nw + nl) * H + h) * R_BYTES; };
+    auto rec_of = [&](int nl) { return records + ((size_t)(bb * nw + c0 + nl) * H + h) * R_BYTES; };
 
     if (warp < 8) {
         const int q4 = warp & 3, cb = 64 * (warp >> 2);   // TMEM lane quarter, value-column half
@@ -648,8 +662,9 @@ __global__ void __launch_bounds__(W2_NT, 1)
         const uint32_t lq = (uint32_t)(32 * q4) << 16;
         const bool is_delta = q4 < 2;
         const int ot = 32 * (q4 - 2) + lane + 64 * (warp >> 2);   // o warps: 0..127
-        {   // Z <- S0 (or 0); the first rescale multiplies by chunk 0's exp(m)
-            const float *src = S0 ? S0 + ((size_t)chain * KD + crow) * VD + cb : nullptr;
+        {   // Z <- S0 (or 0, or I); the first rescale multiplies by chunk 0's exp(m)
+            const float *src = S0 ? S0 + ((size_t)blockIdx.x * KD + crow) * VD + cb : nullptr;
+            const bool ident = (flags & WALK_IDENTITY_S0) != 0;
 #pragma unroll
             for (int u2 = 0; u2 < 2; ++u2) {
                 uint32_t r32[32];
@@ -659,13 +674,16 @@ __global__ void __launch_bounds__(W2_NT, 1)
                     r32[i] = __float_as_uint(x.x); r32[i + 1] = __float_as_uint(x.y);
                     r32[i + 2] = __float_as_uint(x.z); r32[i + 3] = __float_as_uint(x.w);
                 }
+                if (ident)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(cb + 32 * u2 + i == crow ? 1.f : 0.f);
                 tmem_st32(tmem + lq + W2_TM_Z + cb + 32 * u2, r32);
             }
             wait_st();
         }
         float egm_prev = 1.f;
         bool ok = true;
-        for (int nl = 0; nl < nw; ++nl) {
+        for (int nl = 0; nl < nc; ++nl) {
             const uint32_t slot = slot_addr(nl);
             // ---------------------------------------------------------------- record n in, chunk n-1 done
             {
@@ -723,7 +741,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
             }
             if (!is_delta) {
                 // ------------------------------------------------------------ o rows of chunk n-1
-                if (nl > 0) store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + nl - 1) * C, bb);
+                if (nl > 0 && store_out) store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + c0 + nl - 1) * C, bb);
             } else {
                 // ------------------------------------------------------------ Delta = Ũ - W'Z̃ -> bf16 tile; G4/G5
                 if (!group_wait2(misc + M2_G3, (uint32_t)(nl & 1), BAR_DELTA, 128, abort)) continue;
@@ -735,7 +753,8 @@ __global__ void __launch_bounds__(W2_NT, 1)
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int vv = cb + 8 * u;
-                    const uint4 ut = *reinterpret_cast<const uint4 *>(Ut + sw_off(crow, vv, 64));
+                    const uint4 ut = zero_writes ? make_uint4(0u, 0u, 0u, 0u)
+                                                 : *reinterpret_cast<const uint4 *>(Ut + sw_off(crow, vv, 64));
                     const float2 a = unpack2(ut.x), b2 = unpack2(ut.y), c2 = unpack2(ut.z), d2 = unpack2(ut.w);
                     const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
                     const uint4 pk = make_uint4(
@@ -763,9 +782,11 @@ __global__ void __launch_bounds__(W2_NT, 1)
             }
         }
         // the last chunk: its o rows, then S_T = Diag(sPost) Z, once its G4/G5 are complete
-        if (ok && group_wait2(misc + M2_G45 + 8 * ((nw - 1) & 1), (uint32_t)(((nw - 1) >> 1) & 1), BAR_ALL, 256, abort)) {
-            if (!is_delta) store_o(&map_o, sm, d3(nw - 1), ot, crow - 64, cb, h, (n0 + nw - 1) * C, bb);
-            float *dst = ST + ((size_t)chain * KD + crow) * VD + cb;
+        ok = ok && nc > 0 &&
+             group_wait2(misc + M2_G45 + 8 * ((nc - 1) & 1), (uint32_t)(((nc - 1) >> 1) & 1), BAR_ALL, 256, abort);
+        if (ok && !is_delta && store_out) store_o(&map_o, sm, d3(nc - 1), ot, crow - 64, cb, h, (n0 + c0 + nc - 1) * C, bb);
+        if (ok && st_dst) {
+            float *dst = st_dst + (size_t)crow * VD + cb;
             uint32_t x0[32], x1[32];
             tmem_ld32(tmem + lq + W2_TM_Z + cb, x0);
             tmem_ld32(tmem + lq + W2_TM_Z + cb + 32, x1);
@@ -783,7 +804,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
         if (!is_delta && ot == 0) bulk_wait_all();   // the o stores complete before the block exits
     } else if (lane == 0) {
         // ------------------------------------------------------------------ producer: one bulk copy per record
-        for (int nl = 0; nl < nw; ++nl) {
+        for (int nl = 0; nl < nc; ++nl) {
             if (nl >= 2 && !thread_wait(misc + M2_G45 + 8 * (nl & 1), (uint32_t)(((nl - 2) >> 1) & 1), abort)) break;
             mbar_arrive_expect_tx(misc + M2_FULL + 8 * (nl & 1), R_COPY);
             bulk_g2s(smem_u32(sm + slot_addr(nl)), rec_of(nl), R_COPY, misc + M2_FULL + 8 * (nl & 1));
@@ -838,13 +859,32 @@ int sm_count() {
     return n;
 }
 
-constexpr int kWindowChunks = 64;   // chunks per window: bounds the record buffer
+// Plan of a two-stage call.  The record buffer holds one window of chunks of every chain (at most
+// 16,384 chunk-heads, 1.24 GB, and at least 64 chunks).  With few chains (B*H <= 64) each chain's
+// window is cut into nseg segments walked in parallel: each segment's state map S_out = M S_in + N is
+// found by two walks over its records (N from S_in = 0, M from S_in = I with the writes switched
+// off), the maps are composed along the chain in fp32, and a final walk runs every segment from its
+// true start state.
+struct SplitPlan {
+    int nw;     // chunks per window
+    int nseg;   // segments per chain in a full window (1: plain walk)
+};
+SplitPlan split_plan(int B, int H, int T) {
+    const int chains = B * H, NC = (T + split::C - 1) / split::C;
+    int nw = chains > 0 ? std::max(64, 16384 / chains) : 64;
+    nw = std::min(nw, std::max(NC, 1));
+    int nseg = 1;
+    if (chains <= 64 && nw >= 32) nseg = std::max(1, std::min(128 / std::max(chains, 1), nw / 8));
+    return {nw, nseg};
+}
+constexpr size_t kStateBytes = sizeof(float) * 128 * 128;
 
 }  // namespace
 
 size_t split_workspace_bytes(int B, int H, int T) {
-    const int NC = (T + split::C - 1) / split::C, nw = std::min(NC, kWindowChunks);
-    return kStatusBytes + (size_t)B * H * nw * split::R_BYTES;
+    const SplitPlan p = split_plan(B, H, T);
+    const size_t seg = p.nseg > 1 ? 3 * kStateBytes * (size_t)B * H * p.nseg : 0;
+    return kStatusBytes + (size_t)B * H * p.nw * split::R_BYTES + seg;
 }
 
 int launch_chunk_split(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
@@ -861,16 +901,36 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
         return -6;
     const int nsm = sm_count();
     if (nsm <= 0) return -6;
+    const SplitPlan plan = split_plan(B, H, T);
+    const int chains = B * H, NC = (T + split::C - 1) / split::C;
     unsigned int *status = reinterpret_cast<unsigned int *>(ws);
     unsigned char *records = static_cast<unsigned char *>(ws) + kStatusBytes;
-    const int NC = (T + split::C - 1) / split::C;
-    for (int n0 = 0; n0 < NC; n0 += kWindowChunks) {
-        const int nw = std::min(kWindowChunks, NC - n0), nch = B * H * nw;
+    float *Nm = reinterpret_cast<float *>(records + (size_t)chains * plan.nw * split::R_BYTES);
+    float *Mm = Nm + (size_t)chains * plan.nseg * 128 * 128, *Sg = Mm + (size_t)chains * plan.nseg * 128 * 128;
+    for (int n0 = 0; n0 < NC; n0 += plan.nw) {
+        const int nw = std::min(plan.nw, NC - n0), nch = chains * nw;
+        const float *s_in = n0 == 0 ? S0 : ST;
         split::prep_kernel<<<std::min(nch, nsm), split::P1_NT, smem1, st>>>(
             maps, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)b, alpha, records, H, T,
             n0, nw, nch, status);
-        split::walk_kernel<<<B * H, split::W2_NT, smem2, st>>>(map_o, records, n0 == 0 ? S0 : ST, ST, H, T, n0, nw,
-                                                               status);
+        int nseg = plan.nseg > 1 && nw >= 16 ? std::min(plan.nseg, nw / 8) : 1;
+        if (nseg <= 1) {
+            split::walk_kernel<<<chains, split::W2_NT, smem2, st>>>(map_o, records, s_in, ST, H, T, n0, nw, 1, nw, 0u,
+                                                                    status);
+            continue;
+        }
+        const int seg_len = (nw + nseg - 1) / nseg;
+        nseg = (nw + seg_len - 1) / seg_len;   // every segment non-empty
+        const uint32_t skip = split::WALK_SKIP_O;
+        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, nullptr, Nm, H, T, n0, nw, nseg,
+                                                                       seg_len, skip, status);
+        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(
+            map_o, records, nullptr, Mm, H, T, n0, nw, nseg, seg_len,
+            skip | split::WALK_ZERO_WRITES | split::WALK_IDENTITY_S0, status);
+        const int rc = launch_segment_scan(Mm, Nm, s_in, Sg, chains, nseg, st);
+        if (rc != 0) return rc;
+        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, Sg, ST, H, T, n0, nw, nseg,
+                                                                       seg_len, split::WALK_ST_LAST, status);
     }
     return launch_status();
 }

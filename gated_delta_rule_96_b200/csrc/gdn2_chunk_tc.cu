@@ -1111,6 +1111,12 @@ size_t tc_workspace_bytes(int B, int H, int T, int, int, int, int edges) {
     return kStatusBytes + seg + ring;
 }
 
+int launch_segment_scan(const float *M, const float *N, const float *S0, float *Sg, int chains, int nseg,
+                        cudaStream_t st) {
+    tcfwd::segment_scan_kernel<<<dim3(chains, tcfwd::VD / 16), 256, 0, st>>>(M, N, S0, Sg, nseg);
+    return launch_status();
+}
+
 int launch_chunk_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
                     const float *S0, void *o, float *ST, int B, int H, int T, int K, int V, int C, void *ws,
                     cudaStream_t st, int edges, const float *onorm) {

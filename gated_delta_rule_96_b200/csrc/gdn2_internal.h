@@ -30,7 +30,8 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
                     int C, void *ws, cudaStream_t st, int edges = 0, const float *onorm = nullptr);
 
 // Two-stage tcgen05 prefill (bf16 tokens, d_k = d_v = 128, C = 64): the intra-chunk work in parallel
-// over every chunk-head, then the state chain; long sequences in windows of 64 chunks.
+// over every chunk-head, then the state chain; long sequences in windows, few long chains cut into
+// segments in time.
 size_t split_workspace_bytes(int B, int H, int T);
 int launch_chunk_split(const void *q, const void *k, const void *v, const float *alpha, const void *b,
                        const void *w, const float *S0, void *o, float *ST, int B, int H, int T, void *ws,
@@ -39,6 +40,11 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
 // Measurement kernel of the prefill's tensor-core phases (mode 0: back to back; 1: each group waits
 // for the previous one), `reps` chunks per CTA on `nctas` CTAs.
 int launch_phase_probe(int mode, int reps, int nctas, unsigned int *status, cudaStream_t st);
+
+// S_g = M_(g-1) S_(g-1) + N_(g-1) along nseg segments of each chain (fp32; M, N, Sg [chains][nseg][128][128],
+// S0 [chains][128][128] or null for zero).
+int launch_segment_scan(const float *M, const float *N, const float *S0, float *Sg, int chains, int nseg,
+                        cudaStream_t st);
 
 // Backward pass (three sequential passes per chain; fp32 gradients; d_k, d_v in {64, 128}).
 size_t bwd_workspace_bytes(int B, int H, int T, int K, int V);

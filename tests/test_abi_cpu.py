@@ -59,20 +59,26 @@ def test_workspace_bytes_tensor_core_path():
     # most 64 chunks
     rec = 75776
     assert g.gdn2_chunk_fwd_workspace_bytes(8, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 256 + 8 * 16 * 64 * rec
-    assert g.gdn2_chunk_fwd_workspace_bytes(1, 65, 64 * 70 + 5, 128, 128, 64, g.GDN2_BF16) == 256 + 65 * 64 * rec
+    # a window holds at most 16,384 chunk-heads but at least 64 chunks: 65 chains take 252 chunks at once
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 65, 64 * 70 + 5, 128, 128, 64, g.GDN2_BF16) == 256 + 65 * 71 * rec
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 65, 64 * 260, 128, 128, 64, g.GDN2_BF16) == 256 + 65 * 252 * rec
     assert g.gdn2_chunk_fwd_workspace_bytes(2, 33, 65, 128, 128, 64, g.GDN2_BF16) == 256 + 66 * 2 * rec
     assert g.gdn2_chunk_fwd_path(8, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 2
-    # up to 64 chains: the fused kernel; its few-chain form needs only the status header when short
-    assert g.gdn2_chunk_fwd_path(4, 16, 4096, 128, 128, 64, g.GDN2_BF16) == 1
+    assert g.gdn2_chunk_fwd_path(4, 16, 1024, 128, 128, 64, g.GDN2_BF16) == 1
     assert g.gdn2_chunk_fwd_workspace_bytes(4, 16, 1024, 128, 128, 64, g.GDN2_BF16) == 256
     assert g.gdn2_chunk_fwd_path(8, 16, 4096, 128, 128, 64, g.GDN2_F32) == 0
-    # few long chains run in parallel over segments: three fp32 states per (chain, segment)
+    # few long chains: the two-stage path over a window of up to 16,384 chunk-heads, each chain cut into
+    # segments walked in parallel (three fp32 states per chain and segment)
     state = 4 * 128 * 128
-    # B1 H16 T65536: 1,024 chunks, 8 segments of 128 chunks
-    assert g.gdn2_chunk_fwd_workspace_bytes(1, 16, 65536, 128, 128, 64, g.GDN2_BF16) == 256 + 3 * 16 * 8 * state
+    # B1 H16 T65536: 1,024 chunks in one window, 8 segments of 128 chunks
+    assert g.gdn2_chunk_fwd_path(1, 16, 65536, 128, 128, 64, g.GDN2_BF16) == 2
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 16, 65536, 128, 128, 64, g.GDN2_BF16) == \
+        256 + 16 * 1024 * rec + 3 * 16 * 8 * state
     # B1 H2, 41 chunks: at most 64 segments by chains, at least 8 chunks each -> 5 segments of 9 chunks
-    assert g.gdn2_chunk_fwd_workspace_bytes(1, 2, 64 * 40 + 37, 128, 128, 64, g.GDN2_BF16) == 256 + 3 * 2 * 5 * state
-    # short sequences are not split
+    assert g.gdn2_chunk_fwd_workspace_bytes(1, 2, 64 * 40 + 37, 128, 128, 64, g.GDN2_BF16) == \
+        256 + 2 * 41 * rec + 3 * 2 * 5 * state
+    # up to 64 chains of fewer than 32 chunks: the fused kernel, status header only
+    assert g.gdn2_chunk_fwd_path(1, 2, 64 * 31, 128, 128, 64, g.GDN2_BF16) == 1
     assert g.gdn2_chunk_fwd_workspace_bytes(1, 2, 64 * 31, 128, 128, 64, g.GDN2_BF16) == 256
 
 

@@ -22,7 +22,8 @@ int main(void) {
     size_t ws = gdn2_chunk_fwd_workspace_bytes(8, 16, 4096, 128, 128, 64, GDN2_BF16);
     if (ws < 256) { printf("workspace %zu\n", ws); ++fails; }
     if (gdn2_chunk_fwd_path(8, 16, 4096, 128, 128, 64, GDN2_BF16) != 2) ++fails;
-    if (gdn2_chunk_fwd_path(1, 16, 65536, 128, 128, 64, GDN2_BF16) != 1) ++fails;
+    if (gdn2_chunk_fwd_path(1, 16, 65536, 128, 128, 64, GDN2_BF16) != 2) ++fails;
+    if (gdn2_chunk_fwd_path(1, 16, 1024, 128, 128, 64, GDN2_BF16) != 1) ++fails;
     if (gdn2_chunk_fwd_path(1, 2, 256, 64, 64, 64, GDN2_F32) != 0) ++fails;
     if (gdn2_chunk_fwd(fake, fake, fake, (const float *)fake, fake, fake, NULL, fake, (float *)fake, 1, 1, 8, 96,
                        128, 64, GDN2_BF16, fake, ws, NULL) != GDN2_ERR_UNSUPPORTED) ++fails;
