@@ -653,6 +653,54 @@ def long_prefill_row(g, torch, dev, stream, timed, with_cpu):
     return row
 
 
+def fp32_row_workloads():
+    import synth
+    return (("tiny_f32", synth.WORKLOADS["tiny_f32"]),
+            ("prefill_1p3b_f32", synth.Workload("prefill_1p3b_f32", 8, 16, 4096, 128, 128, "f32", 1.0, seed=0x9D2 + 1)))
+
+
+def fp32_prefill_rows(g, torch, dev, stream, timed, with_cpu):
+    """The CUDA-core prefill (fp32 tokens, or d = 64): the tiny fp32 workload the 1e-4 bar applies to
+    (B1 H2 T256 d64) and the 1.3B-scale layer with fp32 tokens (B8 H16 T4096 d128), each against the
+    HBM roofline of its algorithmic bytes (fp32 q, k, v, b, w, alpha read once, o and S_T written once)."""
+    import numpy as np
+    import threadpoolctl
+
+    import oracle
+    import synth
+    peaks = load_peaks()
+    rows = {}
+    for name, wl in fp32_row_workloads():
+        x = synth.make_inputs(wl)
+        X = {k: torch.from_numpy(a).to(dev) for k, a in x.items()}
+        B, T, H, K = X["q"].shape
+        V = X["v"].shape[-1]
+        o = torch.empty((B, T, H, V), device=dev)
+        S_T = torch.empty((B, H, K, V), device=dev)
+        ws = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_F32), dev)
+        ms = timed(lambda: g.gdn2_chunk_fwd(X["q"], X["k"], X["v"], X["alpha"], X["b"], X["w"], None, o, S_T,
+                                            workspace=ws, stream=stream), warm=3, reps=20 if T * B * H < 1e5 else 5)
+        nbytes = prefill_bytes(B, T, H, K, V, tok_bytes=4)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        row = {"workload": f"{name} (B{B} H{H} T{T} d_k=d_v={K}, fp32 tokens)", "ms": ms,
+               "tokens_per_s": B * T / (ms * 1e-3), "launches": 2, "path": "simt",
+               "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+                            "traffic": None, "peak_src": peaks["src"]}}
+        del X, o, S_T, ws
+        if with_cpu:
+            xs = synth.as_f64(synth.make_inputs(wl, chains=[(0, 0)]))
+            with threadpoolctl.threadpool_limits(1):
+                t0 = time.perf_counter()
+                oracle.chain_recurrence(*(xs[k] for k in ("q", "k", "v", "alpha", "b", "w")), None, threads=1)
+                sec = time.perf_counter() - t0
+            row["cpu_baseline"] = {"value": B * T / (sec * B * H), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                   "sample": f"one chain (b=0, h=0, T={T}) of the {B * H}, one thread, scaled by the "
+                                             "chain count"}
+        rows[name] = row
+    return rows
+
+
 def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=True):
     """Timings of the rows beyond the step (not part of `value`): the backward pass of the
     prefill workload and the prefill with the layer edges fused, both on that workload's sizes."""
@@ -707,7 +755,23 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=
                                                    S_T, workspace=ws, stream=stream))
     if g.gdn2_workspace_status(ws) != 0:
         raise RuntimeError("edge prefill kernel reported an internal error")
-    edges = {"ms": edge_ms, "tokens_per_s": B * T / (edge_ms * 1e-3), "launches": 1, "rmsnorm": True,
+    # the unfused layer on the same inputs: the map kernel, the plain prefill, RMSNorm
+    M = {"q": torch.empty_like(R["q"]), "k": torch.empty_like(R["k"]), "b": torch.empty_like(R["b"]),
+         "w": torch.empty_like(R["w"]), "alpha": torch.empty_like(R["a"])}
+    ws2 = g.new_workspace(g.gdn2_chunk_fwd_workspace_bytes(B, H, T, K, V, 64, g.GDN2_BF16), dev)
+
+    def unfused():
+        g.gdn2_layer_edge_maps(R["q"], R["k"], R["a"], R["b"], R["w"], M["q"], M["k"], M["alpha"], M["b"], M["w"],
+                               stream=stream)
+        g.gdn2_chunk_fwd(M["q"], M["k"], R["v"], M["alpha"], M["b"], M["w"], None, o, S_T, workspace=ws2,
+                         stream=stream)
+        g.gdn2_rms_norm(o, weight, stream=stream)
+
+    unfused_ms = timed(unfused)
+    del M, ws2
+    edges = {"ms": edge_ms, "tokens_per_s": B * T / (edge_ms * 1e-3), "launches": 2, "rmsnorm": True,
+             "unfused_ms": unfused_ms,
+             "unfused": "gdn2_layer_edge_maps + gdn2_chunk_fwd + gdn2_rms_norm on the same inputs",
              "plain_prefill_ms": plain_prefill_ms,
              "inputs": "raw q, k ~ N(0, 9), decay logit ~ N(1, 1) (alpha = exp(-softplus(a)): the plain "
                        "workload's alpha distribution), gate logits ~ N(0, 1)"}
@@ -723,6 +787,10 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=
         out["segmented_prefill"] = long_prefill_row(g, torch, dev, stream, timed, with_cpu)
     except Exception as e:   # likewise: this row must not cost the step's line
         out["segmented_prefill"] = {"unavailable": repr(e)[:200]}
+    try:
+        out["fp32_prefill"] = fp32_prefill_rows(g, torch, dev, stream, timed, with_cpu)
+    except Exception as e:
+        out["fp32_prefill"] = {"unavailable": repr(e)[:200]}
     return out
 
 

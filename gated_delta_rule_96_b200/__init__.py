@@ -20,7 +20,7 @@ __all__ = [
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
     "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_recurrence", "gdn2_gemm_phase_probe",
-    "PHASE_PROBE_FLOPS_PER_CHUNK",
+    "PHASE_PROBE_FLOPS_PER_CHUNK", "gdn2_layer_edge_maps", "gdn2_rms_norm",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -74,6 +74,10 @@ def load_library():
     lib.gdn2_chunk_bwd_workspace_bytes.restype = sz
     lib.gdn2_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
     lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_layer_edge_maps.argtypes = [vp] * 10 + [i] * 5 + [vp]
+    lib.gdn2_layer_edge_maps.restype = i
+    lib.gdn2_rms_norm.argtypes = [vp, vp, ctypes.c_longlong, i, vp]
+    lib.gdn2_rms_norm.restype = i
     lib.gdn2_gemm_phase_probe.argtypes = [i, i, i, vp, sz, vp]
     lib.gdn2_gemm_phase_probe.restype = i
     lib.gdn2_status_str.argtypes = [i]
@@ -292,6 +296,43 @@ def gdn2_decode_step(q, k, v, alpha, b, w, S, o, stream=None) -> None:
                                              _ptr(o), B, H, K, V, dt, _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_decode_step")
+
+
+def gdn2_layer_edge_maps(q_raw, k_raw, a_logit, b_logit, w_logit, q, k, alpha, b, w, stream=None) -> None:
+    """The layer's edge maps as one kernel (include/gdn2.h): raw q, k, decay and gate logits -> the
+    normalised q, k, alpha = exp(-softplus(a)), b = sigmoid, w = sigmoid.  bf16 tokens, fp32 logits of alpha."""
+    import torch
+    _check_cuda(q_raw, k_raw, a_logit, b_logit, w_logit, q, k, alpha, b, w)
+    B, T, H, K = q_raw.shape
+    V = w_logit.shape[-1]
+    for name, t in (("a_logit", a_logit), ("alpha", alpha)):
+        if t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    for name, t in (("q_raw", q_raw), ("k_raw", k_raw), ("b_logit", b_logit), ("w_logit", w_logit), ("q", q),
+                    ("k", k), ("b", b), ("w", w)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    tk, tv = (B, T, H, K), (B, T, H, V)
+    _check_shapes((("k_raw", k_raw, tk), ("a_logit", a_logit, tk), ("b_logit", b_logit, tk), ("w_logit", w_logit, tv),
+                   ("q", q, tk), ("k", k, tk), ("alpha", alpha, tk), ("b", b, tk), ("w", w, tv)))
+    with _on_device(q_raw):
+        rc = load_library().gdn2_layer_edge_maps(*(_ptr(t) for t in (q_raw, k_raw, a_logit, b_logit, w_logit, q, k,
+                                                                     alpha, b, w)), B, T, H, K, V, _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_layer_edge_maps")
+
+
+def gdn2_rms_norm(o, weight, stream=None) -> None:
+    """RMSNorm of o in place over its last axis (include/gdn2.h): bf16 o, fp32 weight [d_v]."""
+    import torch
+    _check_cuda(o, weight)
+    V = o.shape[-1]
+    if o.dtype != torch.bfloat16 or weight.dtype != torch.float32 or tuple(weight.shape) != (V,):
+        raise TypeError("o must be bfloat16 and weight float32 of shape [d_v]")
+    with _on_device(o):
+        rc = load_library().gdn2_rms_norm(_ptr(o), _ptr(weight), o.numel() // V, V, _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_rms_norm")
 
 
 def gdn2_gemm_phase_probe(mode, reps, nctas, workspace, stream=None) -> None:

@@ -51,6 +51,7 @@ size_t gdn2_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int
 
 size_t gdn2_chunk_fwd_edges_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C) {
     if (B < 0 || H < 0 || T < 0 || !use_tc(B, H, T, d_k, d_v, C, GDN2_BF16)) return gdn2::kStatusBytes;
+    if (select_path(B, H, T, d_k, d_v, C, GDN2_BF16) == 2) return gdn2::split_workspace_bytes(B, H, T);
     return gdn2::tc_workspace_bytes(B, H, T, d_k, d_v, C, 1);
 }
 
@@ -115,6 +116,9 @@ int gdn2_chunk_fwd_edges(const void *q_raw, const void *k_raw, const void *v, co
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     if (workspace_bytes < gdn2_chunk_fwd_edges_workspace_bytes(B, H, T, d_k, d_v, C)) return GDN2_ERR_WORKSPACE;
     if (B == 0 || H == 0) return GDN2_OK;
+    if (select_path(B, H, T, d_k, d_v, C, dtype) == 2)
+        return gdn2::launch_chunk_split(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o, S_T, B, H, T, workspace,
+                                        reinterpret_cast<cudaStream_t>(stream), 1, o_weight);
     return gdn2::launch_chunk_tc(q_raw, k_raw, v, a_logit, b_logit, w_logit, S0, o, S_T, B, H, T, d_k, d_v, C,
                                  workspace, reinterpret_cast<cudaStream_t>(stream), 1, o_weight);
 }
@@ -163,6 +167,31 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const float *alp
     if (B == 0 || H == 0) return GDN2_OK;
     return gdn2::launch_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, B, H, T,
                                   d_k, d_v, dtype == GDN2_BF16 ? 1 : 0, workspace, st);
+}
+
+int gdn2_layer_edge_maps(const void *q_raw, const void *k_raw, const float *a_logit, const void *b_logit,
+                         const void *w_logit, void *q, void *k, float *alpha, void *b, void *w, int B, int T, int H,
+                         int d_k, int d_v, void *stream) {
+    if (B < 0 || T < 0 || H < 0) return GDN2_ERR_SHAPE;
+    if (!dim_ok(d_k) || !dim_ok(d_v)) return GDN2_ERR_UNSUPPORTED;
+    const long long rows = (long long)B * T * H;
+    if (rows == 0) return GDN2_OK;
+    const void *ptrs[10] = {q_raw, k_raw, a_logit, b_logit, w_logit, q, k, alpha, b, w};
+    for (const void *p : ptrs) {
+        if (!p) return GDN2_ERR_NULL;
+        if (!aligned16(p)) return GDN2_ERR_ALIGN;
+    }
+    return gdn2::launch_edge_maps(q_raw, k_raw, a_logit, b_logit, w_logit, q, k, alpha, b, w, rows, d_k, d_v,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gdn2_rms_norm(void *o, const float *weight, long long rows, int d_v, void *stream) {
+    if (rows < 0) return GDN2_ERR_SHAPE;
+    if (!dim_ok(d_v)) return GDN2_ERR_UNSUPPORTED;
+    if (rows == 0) return GDN2_OK;
+    if (!o || !weight) return GDN2_ERR_NULL;
+    if (!aligned16(o) || !aligned16(weight)) return GDN2_ERR_ALIGN;
+    return gdn2::launch_rms_norm(o, weight, rows, d_v, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int gdn2_gemm_phase_probe(int mode, int reps, int nctas, void *workspace, size_t workspace_bytes, void *stream) {

@@ -122,8 +122,11 @@ __device__ __forceinline__ bool gwait(uint32_t mb, uint32_t parity, uint32_t bar
 // Wide-span chunk: A_ri = sum_c e_rc k_ic exp2(g_rc - g_ic) (i < r) and P_ri likewise with q
 // (i <= r), one row per thread (threads 0-63 rows of A, 64-127 rows of P: the TMEM lanes G1 would
 // have written).  The exponent is summed from log2 alpha while i walks down from r, so it never
-// leaves [-inf, 0]; rows are read again from global memory.
-__device__ __forceinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+// leaves [-inf, 0]; rows are read again from global memory.  Layer-edge variant: q, k raw (their
+// inverse norms applied here), b and alpha from their logits.
+// (A rare correctness path: kept out of line so that it does not weigh on the build's registers.)
+template <bool EDGES>
+__device__ __noinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                              const __nv_bfloat16 *b, const float *alpha, size_t row0, size_t stride,
                                              int tid, int L) {
     const int r = tid & 63;
@@ -132,17 +135,32 @@ __device__ __forceinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat
     const int rc = min(r, L - 1);
     const size_t rowr = row0 + (size_t)rc * stride;
     auto row = [&](int t) { return row0 + (size_t)t * stride; };
-    auto log2a = [&](int t, int cc) { return fast_log2(fmaxf(alpha[row(t) * KD + cc], 1.17549435e-38f)); };
+    auto log2a = [&](int t, int cc) {
+        const float a = alpha[row(t) * KD + cc];
+        return fast_log2(fmaxf(EDGES ? alpha_of_logit(a) : a, 1.17549435e-38f));
+    };
+    auto inv_norm = [&](const __nv_bfloat16 *x, size_t rw) {   // 1 / max(|x_row|, eps)
+        float ss = 0.f;
+        for (int cc = 0; cc < KD; ++cc) {
+            const float v = __bfloat162float(x[rw * KD + cc]);
+            ss += v * v;
+        }
+        return rsqrtf(fmaxf(ss, EDGE_NORM_EPS * EDGE_NORM_EPS));
+    };
+    const float sr = EDGES ? inv_norm(isP ? q : k, rowr) : 1.f;
 #pragma unroll 1
     for (int i0 = 0; i0 < 64; i0 += 16) {
-        float acc[16];
+        float acc[16], sk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 16; ++i) {
+            acc[i] = 0.f;
+            sk[i] = EDGES ? inv_norm(k, row(min(i0 + i, L - 1))) : 1.f;
+        }
         if (r < L && i0 <= r) {
 #pragma unroll 1
             for (int cc = 0; cc < KD; ++cc) {
-                const float x = isP ? __bfloat162float(q[rowr * KD + cc])
-                                    : __bfloat162float(b[rowr * KD + cc]) * __bfloat162float(k[rowr * KD + cc]);
+                const float bg = EDGES ? sigmoid_f(__bfloat162float(b[rowr * KD + cc])) : __bfloat162float(b[rowr * KD + cc]);
+                const float x = sr * (isP ? __bfloat162float(q[rowr * KD + cc]) : bg * __bfloat162float(k[rowr * KD + cc]));
                 const int itop = min(i0 + 15, r);
                 float d = 0.f;
 #pragma unroll 1
@@ -150,7 +168,7 @@ __device__ __forceinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat
 #pragma unroll
                 for (int i = 15; i >= 0; --i) {
                     if (i0 + i <= itop) {
-                        acc[i] += x * __bfloat162float(k[row(i0 + i) * KD + cc]) * exp2f(d);
+                        acc[i] += x * sk[i] * __bfloat162float(k[row(i0 + i) * KD + cc]) * exp2f(d);
                         d += log2a(i0 + i, cc);
                     }
                 }
@@ -168,6 +186,11 @@ __device__ __forceinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat
     wait_st();
 }
 
+// Layer-edge variant (EDGES): the tensors are the layer's raw inputs -- q and k are divided by their
+// L2 norms over the 128 channels, b and w pass a sigmoid, alpha = exp(-softplus(a)) comes from the decay
+// logit -- folded into the build: the inverse norms join the decay factors before their one bf16
+// rounding, so q and k are never rounded after normalisation.
+template <bool EDGES>
 __global__ void __launch_bounds__(P1_NT, 1)
     prep_kernel(const __grid_constant__ TokMaps maps, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                 const __nv_bfloat16 *b, const float *alpha, unsigned char *records, int H, int T, int n0, int nw,
@@ -261,7 +284,9 @@ __global__ void __launch_bounds__(P1_NT, 1)
             float al[8][4];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(AL + (p0 + p) * KD + c4);
+                float4 a4 = *reinterpret_cast<const float4 *>(AL + (p0 + p) * KD + c4);
+                if (EDGES) a4 = make_float4(alpha_of_logit(a4.x), alpha_of_logit(a4.y), alpha_of_logit(a4.z),
+                                            alpha_of_logit(a4.w));
                 // past the end: alpha = 1 (the copy filled zeros); subnormal alpha: smallest normal
                 al[p][0] = p0 + p >= L ? 1.f : fmaxf(a4.x, 1.17549435e-38f);
                 al[p][1] = p0 + p >= L ? 1.f : fmaxf(a4.y, 1.17549435e-38f);
@@ -338,9 +363,34 @@ __global__ void __launch_bounds__(P1_NT, 1)
                     rq[p] = *reinterpret_cast<const uint2 *>(S + P1_EQ + sw_off(64 + r, c4, 128));
                     rk[p] = *reinterpret_cast<const uint2 *>(S + P1_KT + sw_off(r, c4, 64));
                     const uint2 rv = *reinterpret_cast<const uint2 *>(S + P1_U + sw_off(r, c4, 64));
-                    const uint2 rw = *reinterpret_cast<const uint2 *>(S + P1_W + sw_off(r, c4, 64));
+                    uint2 rw = *reinterpret_cast<const uint2 *>(S + P1_W + sw_off(r, c4, 64));
+                    if (EDGES) {
+                        rw = make_uint2(bsigmoid2(rw.x), bsigmoid2(rw.y));
+                        rb[p] = make_uint2(bsigmoid2(rb[p].x), bsigmoid2(rb[p].y));
+                    }
                     *reinterpret_cast<uint2 *>(S + P1_U + sw_off(r, c4, 64)) = make_uint2(bmul2(rw.x, rv.x), bmul2(rw.y, rv.y));
                 }
+                // layer edges: inverse L2 norms of the warp's 8 q and k rows (a warp holds each row, 4
+                // channels a lane), kept in the prefix scratch (read out by now) rather than in registers
+                float *inv = WT + 16 * warp;   // [0, 8): q rows, [8, 16): k rows
+                if (EDGES) {
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const float2 qa = unpack2(rq[p].x), qb = unpack2(rq[p].y), ka = unpack2(rk[p].x), kb = unpack2(rk[p].y);
+                        float sq = qa.x * qa.x + qa.y * qa.y + qb.x * qb.x + qb.y * qb.y;
+                        float sk = ka.x * ka.x + ka.y * ka.y + kb.x * kb.x + kb.y * kb.y;
+#pragma unroll
+                        for (int msk = 16; msk > 0; msk >>= 1) {
+                            sq += __shfl_xor_sync(0xffffffffu, sq, msk);
+                            sk += __shfl_xor_sync(0xffffffffu, sk, msk);
+                        }
+                        if (lane == p) inv[p] = rsqrtf(fmaxf(sq, EDGE_NORM_EPS * EDGE_NORM_EPS));
+                        if (lane == 8 + p) inv[8 + p] = rsqrtf(fmaxf(sk, EDGE_NORM_EPS * EDGE_NORM_EPS));
+                    }
+                    __syncwarp();
+                }
+                auto iq = [&](int p) { return EDGES ? inv[p] : 1.f; };
+                auto ik = [&](int p) { return EDGES ? inv[8 + p] : 1.f; };
                 if (!wide) {
                     // exp(g - m) from one exponential at the thread's first position and running
                     // products of alpha after it; exp(m - g) backwards from one exponential at its last
@@ -357,9 +407,12 @@ __global__ void __launch_bounds__(P1_NT, 1)
                         if (p > 0)
 #pragma unroll
                             for (int jj = 0; jj < 4; ++jj) f1[jj] *= al[p][jj];
-                        const uint32_t F01 = pack_bf16(f1[0], f1[1]), F23 = pack_bf16(f1[2], f1[3]);
+                        // layer edges: the inverse norms join the decay factors before their one rounding
+                        const float sk = ik(p), sq = iq(p);
+                        const uint32_t E01 = pack_bf16(f1[0] * sk, f1[1] * sk), E23 = pack_bf16(f1[2] * sk, f1[3] * sk);
+                        const uint32_t F01 = pack_bf16(f1[0] * sq, f1[1] * sq), F23 = pack_bf16(f1[2] * sq, f1[3] * sq);
                         *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(r, c4, 128)) =
-                            make_uint2(bmul2(bmul2(rb[p].x, rk[p].x), F01), bmul2(bmul2(rb[p].y, rk[p].y), F23));
+                            make_uint2(bmul2(bmul2(rb[p].x, rk[p].x), E01), bmul2(bmul2(rb[p].y, rk[p].y), E23));
                         *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(64 + r, c4, 128)) =
                             make_uint2(bmul2(rq[p].x, F01), bmul2(rq[p].y, F23));
                     }
@@ -370,7 +423,8 @@ __global__ void __launch_bounds__(P1_NT, 1)
                     for (int p = 7; p >= 0; --p) {
                         const int r = p0 + p;
                         *reinterpret_cast<uint2 *>(S + P1_KT + sw_off(r, c4, 64)) =
-                            make_uint2(bmul2(rk[p].x, pack_bf16(f2[0], f2[1])), bmul2(rk[p].y, pack_bf16(f2[2], f2[3])));
+                            make_uint2(bmul2(rk[p].x, pack_bf16(f2[0] * ik(p), f2[1] * ik(p))),
+                                       bmul2(rk[p].y, pack_bf16(f2[2] * ik(p), f2[3] * ik(p))));
 #pragma unroll
                         for (int jj = 0; jj < 4; ++jj) f2[jj] *= al[p][jj];
                     }
@@ -382,7 +436,9 @@ __global__ void __launch_bounds__(P1_NT, 1)
                         const float2 q01 = unpack2(rq[p].x), q23 = unpack2(rq[p].y);
                         const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
                         const float2 b01 = unpack2(rb[p].x), b23 = unpack2(rb[p].y);
-                        const float qq[4] = {q01.x, q01.y, q23.x, q23.y}, kk[4] = {k01.x, k01.y, k23.x, k23.y};
+                        const float sq = iq(p), sk = ik(p);
+                        const float qq[4] = {q01.x * sq, q01.y * sq, q23.x * sq, q23.y * sq};
+                        const float kk[4] = {k01.x * sk, k01.y * sk, k23.x * sk, k23.y * sk};
                         const float bv[4] = {b01.x, b01.y, b23.x, b23.y};
                         float E[4], Qh[4], Kt[4];
 #pragma unroll
@@ -401,7 +457,7 @@ __global__ void __launch_bounds__(P1_NT, 1)
                             make_uint2(pack_bf16(Kt[0], Kt[1]), pack_bf16(Kt[2], Kt[3]));
                     }
                     // A and P straight into D1 (this group read the previous chunk-head's out of it)
-                    if (tid < 128) wide_span_ap(d1, q, k, b, alpha, ((size_t)bb * T + t0) * H + h, (size_t)H, tid, L);
+                    if (tid < 128) wide_span_ap<EDGES>(d1, q, k, b, alpha, ((size_t)bb * T + t0) * H + h, (size_t)H, tid, L);
                 }
             }
             fence_async_smem();
@@ -559,7 +615,8 @@ constexpr uint32_t W2_DL = 32768;                     // Delta bf16 [i x v]
 constexpr uint32_t W2_SLOT = 49152;                   // 2 record slots
 constexpr uint32_t W2_OST = W2_SLOT + 2 * R_BYTES;    // o rows staged for the TMA store (16 KB)
 constexpr uint32_t W2_MISC = W2_OST + 16384;
-constexpr uint32_t W2_BYTES = W2_MISC + 256 + 1024;
+constexpr uint32_t W2_RMS = W2_MISC + 256;            // RMSNorm partial sums [64 rows][2 halves]
+constexpr uint32_t W2_BYTES = W2_MISC + 768 + 1024;
 // mbarriers: FULL and G45 per slot, G3
 enum : uint32_t { M2_FULL = 0, M2_G45 = 16, M2_G3 = 32, M2_TSLOT = 48, M2_ABORT = 52 };
 constexpr uint32_t W2_TM_Z = 0, W2_TM_D3 = 128, W2_TM_COLS = 512;   // D3 buffers at 128 and 256
@@ -584,9 +641,10 @@ __device__ __forceinline__ bool thread_wait(uint32_t mb, uint32_t parity, volati
 
 // o rows of one chunk (TMEM lanes 64-127 of its D3 buffer, value columns cb .. cb + 63) -> bf16 staging
 // tile -> TMA store; rows past the end of the sequence are clipped by the copy.  ot: 0..127 over
-// warps 2, 3, 6, 7.
+// warps 2, 3, 6, 7.  With a weight (layer edges), each row passes RMSNorm first: the two column halves
+// of a row sit in warps w and w + 4 and add their sums of squares through shared memory.
 __device__ __forceinline__ void store_o(const CUtensorMap *map_o, unsigned char *sm, uint32_t d3, int ot, int r,
-                                        int cb, int h, int t0, int bb) {
+                                        int cb, int h, int t0, int bb, const float *onorm) {
     if (ot == 0) bulk_wait_read_all();   // the previous chunk's o store has read the staging tile
     group_sync(BAR_O, 128);
     uint32_t x0[32], x1[32];
@@ -594,6 +652,21 @@ __device__ __forceinline__ void store_o(const CUtensorMap *map_o, unsigned char 
     tmem_ld32(src, x0);
     tmem_ld32(src + 32, x1);
     wait_ld();
+    if (onorm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            ss += __uint_as_float(x0[i]) * __uint_as_float(x0[i]) + __uint_as_float(x1[i]) * __uint_as_float(x1[i]);
+        float *part = reinterpret_cast<float *>(sm + W2_RMS);
+        part[2 * r + (cb >> 6)] = ss;
+        group_sync(BAR_O, 128);
+        const float scale = rsqrtf((part[2 * r] + part[2 * r + 1]) * (1.f / VD) + EDGE_RMS_EPS);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            x0[i] = __float_as_uint(__uint_as_float(x0[i]) * scale * __ldg(onorm + cb + i));
+            x1[i] = __float_as_uint(__uint_as_float(x1[i]) * scale * __ldg(onorm + cb + 32 + i));
+        }
+    }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
@@ -625,7 +698,8 @@ enum : uint32_t {
 
 __global__ void __launch_bounds__(W2_NT, 1)
     walk_kernel(const __grid_constant__ CUtensorMap map_o, const unsigned char *records, const float *S0, float *ST,
-                int H, int T, int n0, int nw, int nseg, int seg_len, uint32_t flags, unsigned int *status) {
+                int H, int T, int n0, int nw, int nseg, int seg_len, uint32_t flags, const float *onorm,
+                unsigned int *status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -741,7 +815,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
             }
             if (!is_delta) {
                 // ------------------------------------------------------------ o rows of chunk n-1
-                if (nl > 0 && store_out) store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + c0 + nl - 1) * C, bb);
+                if (nl > 0 && store_out) store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + c0 + nl - 1) * C, bb, onorm);
             } else {
                 // ------------------------------------------------------------ Delta = Ũ - W'Z̃ -> bf16 tile; G4/G5
                 if (!group_wait2(misc + M2_G3, (uint32_t)(nl & 1), BAR_DELTA, 128, abort)) continue;
@@ -784,7 +858,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
         // the last chunk: its o rows, then S_T = Diag(sPost) Z, once its G4/G5 are complete
         ok = ok && nc > 0 &&
              group_wait2(misc + M2_G45 + 8 * ((nc - 1) & 1), (uint32_t)(((nc - 1) >> 1) & 1), BAR_ALL, 256, abort);
-        if (ok && !is_delta && store_out) store_o(&map_o, sm, d3(nc - 1), ot, crow - 64, cb, h, (n0 + c0 + nc - 1) * C, bb);
+        if (ok && !is_delta && store_out) store_o(&map_o, sm, d3(nc - 1), ot, crow - 64, cb, h, (n0 + c0 + nc - 1) * C, bb, onorm);
         if (ok && st_dst) {
             float *dst = st_dst + (size_t)crow * VD + cb;
             uint32_t x0[32], x1[32];
@@ -888,7 +962,8 @@ size_t split_workspace_bytes(int B, int H, int T) {
 }
 
 int launch_chunk_split(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
-                       const float *S0, void *o, float *ST, int B, int H, int T, void *ws, cudaStream_t st) {
+                       const float *S0, void *o, float *ST, int B, int H, int T, void *ws, cudaStream_t st, int edges,
+                       const float *onorm) {
     split::TokMaps maps;
     CUtensorMap map_o;
     if (!token_map(&maps.q, q, B, T, H) || !token_map(&maps.k, k, B, T, H) || !token_map(&maps.b, b, B, T, H) ||
@@ -896,7 +971,9 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
         !token_map(&maps.alpha, alpha, B, T, H, true) || !token_map(&map_o, o, B, T, H))
         return -6;
     const int smem1 = (int)split::P1_BYTES, smem2 = (int)split::W2_BYTES;
-    if (cudaFuncSetAttribute(split::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess ||
+    auto prep = edges ? split::prep_kernel<true> : split::prep_kernel<false>;
+    if (!edges) onorm = nullptr;
+    if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess ||
         cudaFuncSetAttribute(split::walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
         return -6;
     const int nsm = sm_count();
@@ -910,27 +987,27 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
     for (int n0 = 0; n0 < NC; n0 += plan.nw) {
         const int nw = std::min(plan.nw, NC - n0), nch = chains * nw;
         const float *s_in = n0 == 0 ? S0 : ST;
-        split::prep_kernel<<<std::min(nch, nsm), split::P1_NT, smem1, st>>>(
+        prep<<<std::min(nch, nsm), split::P1_NT, smem1, st>>>(
             maps, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)b, alpha, records, H, T,
             n0, nw, nch, status);
         int nseg = plan.nseg > 1 && nw >= 16 ? std::min(plan.nseg, nw / 8) : 1;
         if (nseg <= 1) {
             split::walk_kernel<<<chains, split::W2_NT, smem2, st>>>(map_o, records, s_in, ST, H, T, n0, nw, 1, nw, 0u,
-                                                                    status);
+                                                                    onorm, status);
             continue;
         }
         const int seg_len = (nw + nseg - 1) / nseg;
         nseg = (nw + seg_len - 1) / seg_len;   // every segment non-empty
         const uint32_t skip = split::WALK_SKIP_O;
         split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, nullptr, Nm, H, T, n0, nw, nseg,
-                                                                       seg_len, skip, status);
+                                                                       seg_len, skip, onorm, status);
         split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(
             map_o, records, nullptr, Mm, H, T, n0, nw, nseg, seg_len,
-            skip | split::WALK_ZERO_WRITES | split::WALK_IDENTITY_S0, status);
+            skip | split::WALK_ZERO_WRITES | split::WALK_IDENTITY_S0, onorm, status);
         const int rc = launch_segment_scan(Mm, Nm, s_in, Sg, chains, nseg, st);
         if (rc != 0) return rc;
         split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, Sg, ST, H, T, n0, nw, nseg,
-                                                                       seg_len, split::WALK_ST_LAST, status);
+                                                                       seg_len, split::WALK_ST_LAST, onorm, status);
     }
     return launch_status();
 }

@@ -128,19 +128,6 @@ constexpr uint32_t ID_G3 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G4 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G5 = idesc_bf16(128, 128, 1, 1);
 
-// Layer edges fused into the prefill (the layer around the recurrence: q and k L2-normalised per
-// token and head, b and w sigmoid gates, the decay from a logit, the output through RMSNorm).
-constexpr float EDGE_NORM_EPS = 1e-6f;   // q / max(|q|, eps), likewise k
-constexpr float EDGE_RMS_EPS = 1e-6f;    // o / sqrt(mean(o^2) + eps) * weight
-__device__ __forceinline__ float fast_rcp(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// sigmoid(x) = 1 / (1 + 2^(-x log2 e)); the exponential saturates to +inf (result 0) or 0 (result 1)
-__device__ __forceinline__ float sigmoid_f(float x) { return fast_rcp(1.f + fast_exp2(-1.4426950408889634f * x)); }
-// alpha = exp(-softplus(a)) = 1 / (1 + e^a) = sigmoid(-a) (0 past fp32's range: the caller floors it)
-__device__ __forceinline__ float alpha_of_logit(float a) { return fast_rcp(1.f + fast_exp2(1.4426950408889634f * a)); }
 // load of data that other warps of the block wrote earlier in this kernel (the layer-edge
 // ring): a plain global load, not the read-only path
 __device__ __forceinline__ float4 ld_f4(const float *p) {
@@ -148,10 +135,7 @@ __device__ __forceinline__ float4 ld_f4(const float *p) {
     asm volatile("ld.global.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ uint32_t bsigmoid2(uint32_t a) {
-    const float2 f = unpack2(a);
-    return pack_bf16(sigmoid_f(f.x), sigmoid_f(f.y));
-}
+
 struct Ctx {
     unsigned char *sm;
     uint32_t tmem, misc;

@@ -33,9 +33,11 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
 // over every chunk-head, then the state chain; long sequences in windows, few long chains cut into
 // segments in time.
 size_t split_workspace_bytes(int B, int H, int T);
+// edges != 0: q, k, b, w, alpha are the layer's raw inputs (see gdn2_chunk_fwd_edges); onorm, if not
+// null, is the RMSNorm weight applied to o.
 int launch_chunk_split(const void *q, const void *k, const void *v, const float *alpha, const void *b,
                        const void *w, const float *S0, void *o, float *ST, int B, int H, int T, void *ws,
-                       cudaStream_t st);
+                       cudaStream_t st, int edges = 0, const float *onorm = nullptr);
 
 // Measurement kernel of the prefill's tensor-core phases (mode 0: back to back; 1: each group waits
 // for the previous one), `reps` chunks per CTA on `nctas` CTAs.
@@ -45,6 +47,12 @@ int launch_phase_probe(int mode, int reps, int nctas, unsigned int *status, cuda
 // S0 [chains][128][128] or null for zero).
 int launch_segment_scan(const float *M, const float *N, const float *S0, float *Sg, int chains, int nseg,
                         cudaStream_t st);
+
+// The layer's edge maps on their own (bf16 tokens, d in {64, 128}; rows = B*T*H).
+int launch_edge_maps(const void *q_raw, const void *k_raw, const float *a_logit, const void *b_logit,
+                     const void *w_logit, void *q, void *k, float *alpha, void *b, void *w, long long rows, int K, int V,
+                     cudaStream_t st);
+int launch_rms_norm(void *o, const float *weight, long long rows, int V, cudaStream_t st);
 
 // Backward pass (three sequential passes per chain; fp32 gradients; d_k, d_v in {64, 128}).
 size_t bwd_workspace_bytes(int B, int H, int T, int K, int V);

@@ -124,6 +124,24 @@ __device__ __forceinline__ void tile_store_t(float *AS, int r0, int c0, const fl
     AS[(c0 + 2 * tq + 1) * LDA + r0 + gq + 8] = sc * d[3];
 }
 
+// Layer edges fused into the prefill (the layer around the recurrence: q and k L2-normalised per
+// token and head, b and w sigmoid gates, the decay from a logit, the output through RMSNorm).
+constexpr float EDGE_NORM_EPS = 1e-6f;   // q / max(|q|, eps), likewise k
+constexpr float EDGE_RMS_EPS = 1e-6f;    // o / sqrt(mean(o^2) + eps) * weight
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// sigmoid(x) = 1 / (1 + 2^(-x log2 e)); the exponential saturates to +inf (result 0) or 0 (result 1)
+__device__ __forceinline__ float sigmoid_f(float x) { return fast_rcp(1.f + fast_exp2(-1.4426950408889634f * x)); }
+// alpha = exp(-softplus(a)) = 1 / (1 + e^a) = sigmoid(-a) (0 past fp32's range: the caller floors it)
+__device__ __forceinline__ float alpha_of_logit(float a) { return fast_rcp(1.f + fast_exp2(1.4426950408889634f * a)); }
+__device__ __forceinline__ uint32_t bsigmoid2(uint32_t a) {
+    const float2 f = unpack2(a);
+    return pack_bf16(sigmoid_f(f.x), sigmoid_f(f.y));
+}
+
 // T = (I + A)^-1 for the strictly lower-triangular 64 x 64 matrix A held in AS (fp32, row stride
 // LDA, zeros on and above the diagonal).  On return T^T is on and above AS's diagonal (A stays
 // below it) and T, in bf16, is in the swizzled 64 x 64 tile Tt, whose blocks above the diagonal

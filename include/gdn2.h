@@ -115,6 +115,24 @@ GDN2_API int gdn2_chunk_fwd_edges(const void *q_raw, const void *k_raw, const vo
                                   void *stream);
 
 /*
+ * The layer's edge maps on their own, as one elementwise kernel: the maps gdn2_chunk_fwd_edges
+ * applies inside the prefill (same page and paragraph), for callers that keep the recurrence's
+ * inputs mapped, and to measure the fused prefill against the unfused layer.  Per (b, t, h):
+ *   q = q_raw / max(|q_raw|_2, 1e-6),  k = k_raw / max(|k_raw|_2, 1e-6)
+ *   b = sigmoid(b_logit),  w = sigmoid(w_logit),  alpha = exp(-softplus(a_logit))
+ * Inputs as gdn2_chunk_fwd_edges (bf16, a_logit fp32); outputs q, k, b [B, T, H, d_k] bf16,
+ * w [B, T, H, d_v] bf16, alpha [B, T, H, d_k] fp32 -- the inputs of gdn2_chunk_fwd.  d_k, d_v in
+ * {64, 128}; outputs must not alias inputs.
+ */
+GDN2_API int gdn2_layer_edge_maps(const void *q_raw, const void *k_raw, const float *a_logit, const void *b_logit,
+                                  const void *w_logit, void *q, void *k, float *alpha, void *b, void *w, int B, int T,
+                                  int H, int d_k, int d_v, void *stream);
+
+/* RMSNorm of the layer output in place: o <- o / sqrt(mean_v(o^2) + 1e-6) * weight, per row of d_v.
+ * o [rows, d_v] bf16, weight [d_v] fp32; d_v in {64, 128}. */
+GDN2_API int gdn2_rms_norm(void *o, const float *weight, long long rows, int d_v, void *stream);
+
+/*
  * One decode token per sequence, state updated in place (constant memory per token,
  * page "NVIDIA улучшила память LLM ...", section "Контекст").
  *

@@ -27,7 +27,7 @@ def test_header_declares_entry_points():
     for name in ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_fwd_workspace_bytes", "gdn2_status_str",
                  "gdn2_workspace_status", "gdn2_chunk_fwd_path", "gdn2_chunk_fwd_edges",
                  "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
-                 "gdn2_chunk_fwd_noalloc", "gdn2_gemm_phase_probe"):
+                 "gdn2_chunk_fwd_noalloc", "gdn2_gemm_phase_probe", "gdn2_layer_edge_maps", "gdn2_rms_norm"):
         assert name in syms
 
 
@@ -172,12 +172,14 @@ def test_chunk_bwd_validation(lib):
 
 
 def test_edges_workspace_bytes():
+    # on the two-stage path the edge-fused prefill needs exactly the plain prefill's workspace
+    for shape in ((8, 16, 4096), (1, 16, 65536), (1, 65, 64 * 70 + 5)):
+        assert g.gdn2_chunk_fwd_edges_workspace_bytes(*shape, 128, 128) == \
+            g.gdn2_chunk_fwd_workspace_bytes(*shape, 128, 128, 64, g.GDN2_BF16)
+    # on the fused kernel (up to 64 chains of fewer than 32 chunks): one decay ring per block
     ring = 4 * 64 * 128 * 4   # four slots of a chunk's decay rows (fp32)
     assert ring == 128 * 1024
-    assert g.gdn2_chunk_fwd_edges_workspace_bytes(8, 16, 4096, 128, 128) == 256 + 128 * ring
-    # segmented: the segment maps plus one ring per (chain, segment) block
-    state = 4 * 128 * 128
-    assert g.gdn2_chunk_fwd_edges_workspace_bytes(1, 16, 65536, 128, 128) == 256 + 3 * 16 * 8 * state + 16 * 8 * ring
+    assert g.gdn2_chunk_fwd_edges_workspace_bytes(4, 16, 1024, 128, 128) == 256 + 64 * ring
     # unsupported shapes need only the status header (the call itself is refused)
     assert g.gdn2_chunk_fwd_edges_workspace_bytes(1, 1, 64, 64, 64) == 256
 
@@ -269,3 +271,17 @@ def test_phase_probe_validation(lib):
     assert lib.gdn2_gemm_phase_probe(0, 1, 1, None, 256, None) == -5
     assert lib.gdn2_gemm_phase_probe(0, 1, 1, ws, 255, None) == -5
     assert lib.gdn2_gemm_phase_probe(1, 1, 1, ctypes.c_void_p(0x10004), 256, None) == -7
+
+
+def test_edge_maps_and_rms_norm_validation(lib):
+    f = ctypes.c_void_p(0x10000)   # never dereferenced: every case fails validation first
+    assert lib.gdn2_layer_edge_maps(*(f,) * 10, -1, 1, 1, 128, 128, None) == -2
+    assert lib.gdn2_layer_edge_maps(*(f,) * 10, 1, 1, 1, 96, 128, None) == -4
+    assert lib.gdn2_layer_edge_maps(*(f,) * 9, None, 1, 1, 1, 128, 128, None) == -1
+    assert lib.gdn2_layer_edge_maps(*(f,) * 9, ctypes.c_void_p(0x10008), 1, 1, 1, 128, 128, None) == -7
+    assert lib.gdn2_layer_edge_maps(*(f,) * 10, 0, 1, 1, 128, 128, None) == 0
+    assert lib.gdn2_rms_norm(f, f, -1, 128, None) == -2
+    assert lib.gdn2_rms_norm(f, f, 1, 32, None) == -4
+    assert lib.gdn2_rms_norm(None, f, 1, 128, None) == -1
+    assert lib.gdn2_rms_norm(f, ctypes.c_void_p(0x10004), 1, 128, None) == -7
+    assert lib.gdn2_rms_norm(f, f, 0, 128, None) == 0

@@ -155,11 +155,19 @@ def test_next_rows_run_on_cpu_through_the_binding(rec, monkeypatch):
 
     monkeypatch.setitem(synth.WORKLOADS, "prefill_long",
                         synth.Workload("prefill_long", 1, 2, 200, 128, 128, "bf16", 1.0, s0_std=0.01, seed=7))
+    monkeypatch.setattr(bench, "fp32_row_workloads", lambda: (
+        ("tiny_f32", synth.WORKLOADS["tiny_f32"]),
+        ("prefill_1p3b_f32", synth.Workload("f", 2, 3, 70, 128, 128, "f32", 1.0, seed=9))))
     wl = synth.Workload("nr", 1, 2, 96, 128, 128, "bf16", 1.0, seed=5)
     out = bench.run_next_rows(g, FakeTorch(), "cpu", None, wl, 0.5, {"sm_max_mhz": 1965.0})
     names = [c[0] for c in rec.calls]
     assert names.count("gdn2_chunk_bwd") == 7 and names.count("gdn2_chunk_fwd_edges") == 7
-    assert names.count("gdn2_chunk_fwd") == 7
+    # segmented row 7; unfused edge layer 7; fp32 rows: tiny 3 + 20, the other 3 + 20 (small here)
+    assert names.count("gdn2_chunk_fwd") == 7 + 7 + 23 + 23
+    assert names.count("gdn2_layer_edge_maps") == 7 and names.count("gdn2_rms_norm") == 7
+    f32 = out["fp32_prefill"]
+    assert f32["tiny_f32"]["roofline"]["algorithmic_bytes_per_launch"] == bench.prefill_bytes(1, 256, 2, 64, 64, 4)
+    assert f32["tiny_f32"]["cpu_baseline"]["value"] > 0
     bw, ed, sp = out["backward"], out["edges_prefill"], out["segmented_prefill"]
     ms = 1.0 / 5
     assert bw["ms"] == ms and bw["tokens_per_s"] == pytest.approx(96 / (ms * 1e-3))

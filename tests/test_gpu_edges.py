@@ -105,3 +105,68 @@ def test_edges_rejects_unsupported_shapes():
     with pytest.raises(g.GDN2Error):
         g.gdn2_chunk_fwd_edges(small["q"], small["k"], small["v"], small["a"], small["b"], small["w"], None, None,
                                o, ST)
+
+
+@pytest.mark.parametrize("norm", [False, True])
+@pytest.mark.parametrize("T", [1, 65, 200])
+def test_edges_two_stage_small(norm, T):
+    """More than 64 chains: the maps fused into the two-stage path (prep: norms, sigmoids and the
+    decay from its logit; walk: RMSNorm of the o rows)."""
+    torch, g = cuda_or_skip()
+    assert g.gdn2_chunk_fwd_path(2, 33, T, 128, 128, 64, g.GDN2_BF16) == 2
+    x = raw_inputs(2, T, 33, seed=95)
+    S0 = np.random.default_rng(12).normal(scale=0.05, size=(2, 33, 128, 128)).astype(np.float32)
+    weight = np.random.default_rng(13).normal(size=128).astype(np.float32) if norm else None
+    o, ST = run(torch, g, to_dev(torch, x), torch.from_numpy(S0).cuda(),
+                None if weight is None else torch.from_numpy(weight).cuda())
+    ref_o, ref_S = reference(x, S0)
+    if weight is None:
+        assert_close("o", f64(o), ref_o, TOL["bf16"])
+    else:
+        assert_normed_close("o", f64(o), ref_o, weight, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
+
+
+def test_layer_edge_maps_and_rms_norm():
+    """The stand-alone map kernels against the oracle's maps: q, k, b, w are bf16 roundings of the
+    fp64 maps (half an ulp, 2^-9 relative, plus the fp32 arithmetic), alpha fp32; RMSNorm likewise."""
+    torch, g = cuda_or_skip()
+    for B, T, H in ((2, 70, 3), (1, 5, 40)):
+        x = raw_inputs(B, T, H, seed=96)
+        xd = to_dev(torch, x)
+        q, k, b = (torch.empty_like(xd["q"]) for _ in range(3))
+        w = torch.empty_like(xd["w"])
+        alpha = torch.empty_like(xd["a"])
+        g.gdn2_layer_edge_maps(xd["q"], xd["k"], xd["a"], xd["b"], xd["w"], q, k, alpha, b, w)
+        torch.cuda.synchronize()
+        ref = oracle.layer_edges(*(xd[n].double().cpu().numpy() for n in ("q", "k", "a", "b", "w")))
+        for name, got, r in zip(("q", "k", "alpha", "b", "w"), (q, k, alpha, b, w), ref):
+            bar = 1e-5 if name == "alpha" else 2.0 ** -8
+            err = np.max(np.abs(f64(got) - r) / np.maximum(np.abs(r), 1e-30))
+            assert err <= bar, f"{name}: elementwise rel err {err:.2e} > {bar:.1e}"
+        o = torch.randn((B, T, H, 128), device="cuda").to(torch.bfloat16)
+        weight = torch.randn(128, device="cuda")
+        ref_n = oracle.rms_norm(f64(o), weight.double().cpu().numpy())
+        g.gdn2_rms_norm(o, weight)
+        torch.cuda.synchronize()
+        assert_close("rms_norm", f64(o), ref_n, 2.0 ** -7)
+
+
+def test_edges_unfused_layer_matches():
+    """The unfused layer -- the map kernel, the plain prefill, RMSNorm -- gives the oracle's result on
+    the two-stage shapes, like the fused entry point."""
+    torch, g = cuda_or_skip()
+    x = raw_inputs(2, 130, 33, seed=97)
+    xd = to_dev(torch, x)
+    q, k, b = (torch.empty_like(xd["q"]) for _ in range(3))
+    w = torch.empty_like(xd["w"])
+    alpha = torch.empty_like(xd["a"])
+    weight_np = np.random.default_rng(14).normal(size=128).astype(np.float32)
+    weight = torch.from_numpy(weight_np).cuda()
+    g.gdn2_layer_edge_maps(xd["q"], xd["k"], xd["a"], xd["b"], xd["w"], q, k, alpha, b, w)
+    o, ST = g.chunk_fwd(q, k, xd["v"], alpha, b, w)
+    g.gdn2_rms_norm(o, weight)
+    torch.cuda.synchronize()
+    ref_o, ref_S = reference(x, None)
+    assert_normed_close("o", f64(o), ref_o, weight_np, TOL["bf16"])
+    assert_close("S_T", f64(ST), ref_S, TOL["bf16"])
