@@ -618,7 +618,8 @@ constexpr uint32_t W2_MISC = W2_OST + 16384;
 constexpr uint32_t W2_RMS = W2_MISC + 256;            // RMSNorm partial sums [64 rows][2 halves]
 constexpr uint32_t W2_BYTES = W2_MISC + 768 + 1024;
 // mbarriers: FULL and G45 per slot, G3
-enum : uint32_t { M2_FULL = 0, M2_G45 = 16, M2_G3 = 32, M2_TSLOT = 48, M2_ABORT = 52 };
+// G5 per slot completes before G4: the next chunk's rescale waits for G5 only, the o rows for G4/G5
+enum : uint32_t { M2_FULL = 0, M2_G45 = 16, M2_G3 = 32, M2_ZST = 40, M2_G5 = 48, M2_TSLOT = 64, M2_ABORT = 68 };
 constexpr uint32_t W2_TM_Z = 0, W2_TM_D3 = 128, W2_TM_COLS = 512;   // D3 buffers at 128 and 256
 constexpr uint32_t BAR_ALL = 1, BAR_DELTA = 2, BAR_O = 3;            // named barriers (128 or 256 threads)
 
@@ -716,8 +717,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(misc + M2_FULL + 8 * s, 1);
             mbar_init(misc + M2_G45 + 8 * s, 1);
+            mbar_init(misc + M2_G5 + 8 * s, 1);
         }
         mbar_init(misc + M2_G3, 1);
+        mbar_init(misc + M2_ZST, 128);
         *abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         prefetch_tmap(&map_o);
@@ -763,7 +766,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
             {
                 bool w_ok = mbar_wait(misc + M2_FULL + 8 * (nl & 1), (uint32_t)((nl >> 1) & 1), WAIT_LIMIT);
                 if (nl > 0)
-                    w_ok = w_ok && mbar_wait(misc + M2_G45 + 8 * ((nl - 1) & 1), (uint32_t)(((nl - 1) >> 1) & 1), WAIT_LIMIT);
+                    w_ok = w_ok && mbar_wait(misc + M2_G5 + 8 * ((nl - 1) & 1), (uint32_t)(((nl - 1) >> 1) & 1), WAIT_LIMIT);
                 w_ok = w_ok && !*abort;
                 const bool fail = group_or(BAR_ALL, 256, !w_ok);
                 fence_after();
@@ -793,6 +796,19 @@ __global__ void __launch_bounds__(W2_NT, 1)
                                                 pack_bf16(ssc * __uint_as_float(x[6]), ssc * __uint_as_float(x[7])));
                     *reinterpret_cast<uint4 *>(sm + W2_S + sw_off(crow, cb + 8 * u, 128)) = pk;
                 }
+                // G3 needs only the bf16 copy: issue it first, then write Z back (G5, its next reader, is
+                // issued once every thread's store is complete)
+                fence_async_smem();
+                fence_before();
+                group_sync(BAR_ALL, 256);
+                if (tid == 0) {   // G3: [-W'Z̃; Q̂Z̃] into this chunk's D3 buffer (its o rows of chunk n-2 are out)
+                    fence_after();
+                    const uint32_t aA3 = smem_u32(sm + slot + R_A3), aS = smem_u32(sm + W2_S);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        mma_ss(d3(nl), desc_kmajor(aA3, 128, j), desc_mnmajor(aS, 128, j), ID_G3, j > 0);
+                    mma_commit(misc + M2_G3);
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     x0[i] = __float_as_uint(zsc * __uint_as_float(x0[i]));
@@ -801,25 +817,25 @@ __global__ void __launch_bounds__(W2_NT, 1)
                 tmem_st32(tmem + lq + W2_TM_Z + cb, x0);
                 tmem_st32(tmem + lq + W2_TM_Z + cb + 32, x1);
                 wait_st();
-            }
-            fence_async_smem();
-            fence_before();
-            group_sync(BAR_ALL, 256);
-            if (tid == 0) {   // G3: [-W'Z̃; Q̂Z̃] into this chunk's D3 buffer (its o rows of chunk n-2 are out)
-                fence_after();
-                const uint32_t aA3 = smem_u32(sm + slot + R_A3), aS = smem_u32(sm + W2_S);
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    mma_ss(d3(nl), desc_kmajor(aA3, 128, j), desc_mnmajor(aS, 128, j), ID_G3, j > 0);
-                mma_commit(misc + M2_G3);
+                fence_before();
+                if (!is_delta) mbar_arrive(misc + M2_ZST);   // the o warps' rows of Z are written back
             }
             if (!is_delta) {
                 // ------------------------------------------------------------ o rows of chunk n-1
-                if (nl > 0 && store_out) store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + c0 + nl - 1) * C, bb, onorm);
+                if (nl > 0 && store_out) {   // once G4 of chunk n-1 is complete
+                    if (!group_wait2(misc + M2_G45 + 8 * ((nl - 1) & 1), (uint32_t)(((nl - 1) >> 1) & 1), BAR_O, 128, abort))
+                        continue;
+                    store_o(&map_o, sm, d3(nl - 1), ot, crow - 64, cb, h, (n0 + c0 + nl - 1) * C, bb, onorm);
+                }
             } else {
                 // ------------------------------------------------------------ Delta = Ũ - W'Z̃ -> bf16 tile; G4/G5
-                if (!group_wait2(misc + M2_G3, (uint32_t)(nl & 1), BAR_DELTA, 128, abort)) continue;
                 const unsigned char *Ut = sm + slot + R_U;
+                uint4 ut8[8];   // Ũ of this thread's row, read while G3 runs
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    ut8[u] = zero_writes ? make_uint4(0u, 0u, 0u, 0u)
+                                         : *reinterpret_cast<const uint4 *>(Ut + sw_off(crow, cb + 8 * u, 64));
+                if (!group_wait2(misc + M2_G3, (uint32_t)(nl & 1), BAR_DELTA, 128, abort)) continue;
                 uint32_t x0[32], x1[32];
                 tmem_ld32(d3(nl) + lq + cb, x0);
                 tmem_ld32(d3(nl) + lq + cb + 32, x1);
@@ -827,8 +843,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int vv = cb + 8 * u;
-                    const uint4 ut = zero_writes ? make_uint4(0u, 0u, 0u, 0u)
-                                                 : *reinterpret_cast<const uint4 *>(Ut + sw_off(crow, vv, 64));
+                    const uint4 ut = ut8[u];
                     const float2 a = unpack2(ut.x), b2 = unpack2(ut.y), c2 = unpack2(ut.z), d2 = unpack2(ut.w);
                     const uint32_t *x = (u < 4 ? x0 : x1) + 8 * (u & 3);
                     const uint4 pk = make_uint4(
@@ -842,16 +857,21 @@ __global__ void __launch_bounds__(W2_NT, 1)
                 fence_before();
                 group_sync(BAR_DELTA, 128);
                 if (tid == 0) {   // G4: O += P Delta (rows 0-63 of the A tile are Ũ's bytes: their products
-                                  // land in the Delta rows of D3, already read); G5: Z += K̃^T Delta
+                                  // land in the Delta rows of D3, already read); G5: Z += K̃^T Delta, once the
+                                  // o warps' rows of Z are written back
+                    const bool zs = thread_wait(misc + M2_ZST, (uint32_t)(nl & 1), abort);
                     fence_after();
+                    if (zs) {
                     const uint32_t aPA = smem_u32(sm + slot + R_P - 8192), aKT = smem_u32(sm + slot + R_KT),
                                    aDL = smem_u32(sm + W2_DL);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) mma_ss(d3(nl), desc_kmajor(aPA, 128, j), desc_mnmajor(aDL, 64, j), ID_G4, 1);
-#pragma unroll
                     for (int j = 0; j < 4; ++j)
                         mma_ss(tmem + W2_TM_Z, desc_mnmajor(aKT, 64, j), desc_mnmajor(aDL, 64, j), ID_G5, 1);
+                    mma_commit(misc + M2_G5 + 8 * (nl & 1));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) mma_ss(d3(nl), desc_kmajor(aPA, 128, j), desc_mnmajor(aDL, 64, j), ID_G4, 1);
                     mma_commit(misc + M2_G45 + 8 * (nl & 1));
+                    }
                 }
             }
         }

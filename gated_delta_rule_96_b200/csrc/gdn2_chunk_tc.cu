@@ -1026,37 +1026,42 @@ __global__ void __launch_bounds__(NT, 1)
 
 // ============================================================================ segment scan
 // S_g = M_(g-1) S_(g-1) + N_(g-1) along the segments of each chain (g = 1 .. nseg-1), S_0 = S0.
-// One block per (chain, 16-column slice of S); fp32.
+// One block per (chain, 16-column slice of S); fp32.  Each step stages M_(g-1) (64 KB) in shared
+// memory with coalesced loads; thread (r0, col) keeps rows r0, r0 + 16, ..., r0 + 112 of its column.
+constexpr int SCAN_SMEM = (KD * KD + KD * 16) * 4;   // M, then the previous state's column slice
 __global__ void __launch_bounds__(256) segment_scan_kernel(const float *__restrict__ M, const float *__restrict__ N,
-                                                           const float *S0, float *__restrict__ Sg,
-                                                           int nseg) {
-    __shared__ float sprev[KD][16];
+                                                           const float *S0, float *__restrict__ Sg, int nseg) {
+    extern __shared__ float scan_sm[];
+    float *Ms = scan_sm, *sprev = scan_sm + KD * KD;   // Ms [KD][KD], sprev [KD][16]
     const int chain = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
     const size_t KV = (size_t)KD * VD;
     const int col = tid & 15, r0 = tid >> 4;   // rows r0, r0 + 16, ..., r0 + 112
     for (int r = r0; r < KD; r += 16) {
         const float v = S0 ? S0[chain * KV + (size_t)r * VD + c0 + col] : 0.f;
-        sprev[r][col] = v;
+        sprev[r * 16 + col] = v;
         Sg[((size_t)chain * nseg) * KV + (size_t)r * VD + c0 + col] = v;
     }
-    __syncthreads();
     for (int g = 1; g < nseg; ++g) {
         const float *Mg = M + ((size_t)chain * nseg + g - 1) * KV, *Ng = N + ((size_t)chain * nseg + g - 1) * KV;
+        __syncthreads();   // the previous step's reads of Ms are done
+        for (int i = tid; i < KD * KD / 4; i += 256)
+            reinterpret_cast<float4 *>(Ms)[i] = __ldg(reinterpret_cast<const float4 *>(Mg) + i);
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = Ng[(size_t)(r0 + 16 * i) * VD + c0 + col];
-        for (int kk = 0; kk < KD; ++kk) {
-            const float sv = sprev[kk][col];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(Mg[(size_t)(r0 + 16 * i) * VD + kk], sv, acc[i]);
-        }
         __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < KD; ++kk) {
+            const float sv = sprev[kk * 16 + col];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(Ms[(r0 + 16 * i) * KD + kk], sv, acc[i]);
+        }
+        __syncthreads();   // every thread has read sprev
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            sprev[r0 + 16 * i][col] = acc[i];
+            sprev[(r0 + 16 * i) * 16 + col] = acc[i];
             Sg[((size_t)chain * nseg + g) * KV + (size_t)(r0 + 16 * i) * VD + c0 + col] = acc[i];
         }
-        __syncthreads();
     }
 }
 
@@ -1097,7 +1102,10 @@ size_t tc_workspace_bytes(int B, int H, int T, int, int, int, int edges) {
 
 int launch_segment_scan(const float *M, const float *N, const float *S0, float *Sg, int chains, int nseg,
                         cudaStream_t st) {
-    tcfwd::segment_scan_kernel<<<dim3(chains, tcfwd::VD / 16), 256, 0, st>>>(M, N, S0, Sg, nseg);
+    if (cudaFuncSetAttribute(tcfwd::segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tcfwd::SCAN_SMEM) != cudaSuccess)
+        return -6;
+    tcfwd::segment_scan_kernel<<<dim3(chains, tcfwd::VD / 16), 256, tcfwd::SCAN_SMEM, st>>>(M, N, S0, Sg, nseg);
     return launch_status();
 }
 
@@ -1126,7 +1134,8 @@ int launch_chunk_tc(const void *q, const void *k, const void *v, const float *al
     float *Mm = Nm + per_pass, *Sg = Mm + per_pass;
     run(sp.nseg, sp.seg_len, tcfwd::SEG_SKIP_O, nullptr, Nm);
     run(sp.nseg, sp.seg_len, tcfwd::SEG_SKIP_O | tcfwd::SEG_ZERO_WRITES | tcfwd::SEG_IDENTITY_S0, nullptr, Mm);
-    tcfwd::segment_scan_kernel<<<dim3(B * H, tcfwd::VD / 16), 256, 0, st>>>(Mm, Nm, S0, Sg, sp.nseg);
+    const int rc = launch_segment_scan(Mm, Nm, S0, Sg, B * H, sp.nseg, st);
+    if (rc != 0) return rc;
     run(sp.nseg, sp.seg_len, tcfwd::SEG_ST_LAST, Sg, ST);
     return launch_status();
 }
