@@ -19,6 +19,7 @@ __all__ = [
     "gdn2_chunk_fwd_workspace_bytes", "gdn2_chunk_fwd_path", "gdn2_workspace_status", "gdn2_status_str",
     "gdn2_chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "chunk_fwd", "decode_step", "new_workspace", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
+    "gdn2_chunk_bwd_tc", "gdn2_chunk_bwd_tc_workspace_bytes",
     "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_recurrence", "gdn2_gemm_phase_probe",
     "PHASE_PROBE_FLOPS_PER_CHUNK", "gdn2_layer_edge_maps", "gdn2_rms_norm",
 ]
@@ -74,6 +75,10 @@ def load_library():
     lib.gdn2_chunk_bwd_workspace_bytes.restype = sz
     lib.gdn2_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
     lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_chunk_bwd_tc_workspace_bytes.argtypes = [i] * 5
+    lib.gdn2_chunk_bwd_tc_workspace_bytes.restype = sz
+    lib.gdn2_chunk_bwd_tc.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
+    lib.gdn2_chunk_bwd_tc.restype = i
     lib.gdn2_layer_edge_maps.argtypes = [vp] * 10 + [i] * 5 + [vp]
     lib.gdn2_layer_edge_maps.restype = i
     lib.gdn2_rms_norm.argtypes = [vp, vp, ctypes.c_longlong, i, vp]
@@ -254,6 +259,40 @@ def gdn2_chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, d
                                            _stream(stream))
     if rc != 0:
         raise GDN2Error(rc, "gdn2_chunk_bwd")
+
+
+def gdn2_chunk_bwd_tc_workspace_bytes(B, H, T, d_k, d_v) -> int:
+    return int(load_library().gdn2_chunk_bwd_tc_workspace_bytes(B, H, T, d_k, d_v))
+
+
+def gdn2_chunk_bwd_tc(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, workspace=None,
+                      stream=None) -> None:
+    """Tensor-core backward (include/gdn2.h, gdn2_chunk_bwd_tc): the gradients of gdn2_chunk_bwd for bf16
+    tokens with d_k = d_v = 128, from bf16 tensor-core products.  A workspace passed in must start with a
+    zeroed status header (new_workspace gives one)."""
+    import torch
+    _check_cuda(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, workspace)
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    dt = _dtype_code(q)
+    for name, t in (("alpha", alpha), ("S0", S0), ("dS_T", dS_T), ("dq", dq), ("dk", dk), ("dv", dv),
+                    ("dalpha", dalpha), ("db", db), ("dw", dw), ("dS0", dS0)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    _check_dtypes(q, (("k", k), ("v", v), ("b", b), ("w", w), ("dO", dO)))
+    tk, tv, st = (B, T, H, K), (B, T, H, V), (B, H, K, V)
+    _check_shapes((("k", k, tk), ("b", b, tk), ("alpha", alpha, tk), ("v", v, tv), ("w", w, tv),
+                   ("dO", dO, tv), ("S0", S0, st), ("dS_T", dS_T, st), ("dq", dq, tk), ("dk", dk, tk),
+                   ("dalpha", dalpha, tk), ("db", db, tk), ("dv", dv, tv), ("dw", dw, tv), ("dS0", dS0, st)))
+    if workspace is None:
+        workspace = new_workspace(max(gdn2_chunk_bwd_tc_workspace_bytes(B, H, T, K, V), 256), q.device)
+    with _on_device(q):
+        rc = load_library().gdn2_chunk_bwd_tc(*(_ptr(t) for t in (q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv,
+                                                                  dalpha, db, dw, dS0)), B, H, T, K, V, dt,
+                                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                              _stream(stream))
+    if rc != 0:
+        raise GDN2Error(rc, "gdn2_chunk_bwd_tc")
 
 
 def gdn2_chunk_fwd_noalloc(q, k, v, alpha, b, w, S0, o, S_T, C=64, stream=None) -> None:

@@ -169,6 +169,41 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const float *alp
                                   d_k, d_v, dtype == GDN2_BF16 ? 1 : 0, workspace, st);
 }
 
+size_t gdn2_chunk_bwd_tc_workspace_bytes(int B, int H, int T, int d_k, int d_v) {
+    if (B < 0 || H < 0 || T < 0 || d_k != 128 || d_v != 128) return 0;
+    return gdn2::chunk_bwd_tc_workspace_bytes(B, H, T);
+}
+
+int gdn2_chunk_bwd_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                      const float *S0, const void *dO, const float *dS_T, float *dq, float *dk, float *dv,
+                      float *dalpha, float *db, float *dw, float *dS0, int B, int H, int T, int d_k, int d_v,
+                      int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (T < 0 || B < 0 || H < 0) return GDN2_ERR_SHAPE;
+    if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (dtype != GDN2_BF16 || d_k != 128 || d_v != 128) return GDN2_ERR_UNSUPPORTED;
+    if ((S0 && !aligned16(S0)) || (dS_T && !aligned16(dS_T)) || (dS0 && !aligned16(dS0))) return GDN2_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {   // S_T = S0: dS0 = dS_T; no token gradients
+        if (!dS0 || B == 0 || H == 0) return GDN2_OK;
+        const size_t state_bytes = sizeof(float) * (size_t)B * H * d_k * d_v;
+        const cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(dS0, 0, state_bytes, st);
+        return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+    }
+    int rc = check_common(q, k, v, alpha, b, w, dO, B, H, d_k, d_v, dtype);
+    if (rc != GDN2_OK) return rc;
+    if (!dq || !dk || !dv || !dalpha || !db || !dw) return GDN2_ERR_NULL;
+    if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dalpha) || !aligned16(db) ||
+        !aligned16(dw))
+        return GDN2_ERR_ALIGN;
+    if (!workspace) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    if (workspace_bytes < gdn2_chunk_bwd_tc_workspace_bytes(B, H, T, d_k, d_v)) return GDN2_ERR_WORKSPACE;
+    if (B == 0 || H == 0) return GDN2_OK;
+    return gdn2::launch_chunk_bwd_tc(q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, B, H, T,
+                                     workspace, st);
+}
+
 int gdn2_layer_edge_maps(const void *q_raw, const void *k_raw, const float *a_logit, const void *b_logit,
                          const void *w_logit, void *q, void *k, float *alpha, void *b, void *w, int B, int T, int H,
                          int d_k, int d_v, void *stream) {

@@ -39,6 +39,7 @@
 
 #include "gdn2_common.cuh"
 #include "gdn2_internal.h"
+#include "split_layout.cuh"
 #include "tc_chunk.cuh"
 #include "tc_ptx.cuh"
 
@@ -48,19 +49,9 @@ namespace split {
 using namespace gdn2::tc;
 using namespace gdn2::tcc;
 
-constexpr int C = 64, KD = 128, VD = 128;
 constexpr float SPAN_MAX_LOG2 = 173.123f;   // 120 nats in log2 units
 constexpr uint32_t WAIT_LIMIT = 1u << 22;
 constexpr uint32_t STATUS_PREP = 2u, STATUS_WALK = 4u;
-
-// ---------------------------------------------------------------------------- record (bytes)
-constexpr uint32_t R_A3 = 0;        // [-W'; Q̂]: 128 x 128 K-major (A of G3)
-constexpr uint32_t R_KT = 32768;    // K̃ [i x c]: 64 x 128 (MN-major A of G5)
-constexpr uint32_t R_U = 49152;     // Ũ [i x v]: 64 x 128
-constexpr uint32_t R_P = 65536;     // P [r x i]: 64 x 64, lower with the diagonal
-constexpr uint32_t R_VEC = 73728;   // sS, sZ, sPost: 3 x 128 fp32
-constexpr uint32_t R_COPY = R_VEC + 3 * 128 * 4;   // bytes moved per record
-constexpr uint32_t R_BYTES = 75776;                // record stride (1024-aligned)
 
 // ---------------------------------------------------------------------------- stage 1
 // One persistent CTA per SM over the window's chunk-heads, three roles working on consecutive
@@ -97,9 +88,6 @@ constexpr uint32_t ID_G3 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G4 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G5 = idesc_bf16(128, 128, 1, 1);
 
-struct TokMaps {   // [B, T, H, 128] token tensors as 4-D maps (d, H, T, B): bf16 with a 64 x 1 x 64 x 1 box
-    CUtensorMap q, k, b, v, w, alpha;   // in the 128-byte swizzle; alpha fp32 with a 128 x 1 x 64 x 1 box
-};
 
 // Bounded wait of one thread (the producer); on expiry it sets the abort flag.
 __device__ __forceinline__ bool thread_wait1(uint32_t mb, uint32_t parity, volatile uint32_t *abort) {
@@ -190,11 +178,15 @@ __device__ __noinline__ void wide_span_ap(uint32_t tmem_d1, const __nv_bfloat16 
 // L2 norms over the 128 channels, b and w pass a sigmoid, alpha = exp(-softplus(a)) comes from the decay
 // logit -- folded into the build: the inverse norms join the decay factors before their one bf16
 // rounding, so q and k are never rounded after normalisation.
-template <bool EDGES>
+// EXACT_F: each factor of a tensor-core chunk (Ê, Q̂, K̃) is one fp32 product rounded once to bf16,
+// b ⊙ k included, instead of packed bf16 products of bf16-rounded frame factors.  The backward's
+// replay builds its records this way: d(ln alpha) sums terms of both signs, and the bf16 rounding of
+// the frame factors, a relative error that differs between Ê, Q̂ and K̃, doubles its error.
+template <bool EDGES, bool EXACT_F = false>
 __global__ void __launch_bounds__(P1_NT, 1)
     prep_kernel(const __grid_constant__ TokMaps maps, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
-                const __nv_bfloat16 *b, const float *alpha, unsigned char *records, int H, int T, int n0, int nw,
-                int nch, unsigned int *status) {
+                const __nv_bfloat16 *b, const float *alpha, unsigned char *records, unsigned char *aux, int H, int T,
+                int n0, int nw, int nch, unsigned int *status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -228,6 +220,7 @@ __global__ void __launch_bounds__(P1_NT, 1)
     };
     const int njobs = (int)blockIdx.x < nch ? (nch - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     auto rec_of = [&](int j) { return records + (size_t)(blockIdx.x + j * gridDim.x) * R_BYTES; };
+    auto aux_of = [&](int j) { return aux + (size_t)(blockIdx.x + j * gridDim.x) * X_BYTES; };
 
     if (warp == 12) {
         // ------------------------------------------------------------------ producer (one thread)
@@ -350,6 +343,12 @@ __global__ void __launch_bounds__(P1_NT, 1)
                 *reinterpret_cast<float4 *>(vec + c4) = make_float4(sS[0], sS[1], sS[2], sS[3]);
                 *reinterpret_cast<float4 *>(vec + 128 + c4) = make_float4(sZ[0], sZ[1], sZ[2], sZ[3]);
                 *reinterpret_cast<float4 *>(vec + 256 + c4) = make_float4(sP[0], sP[1], sP[2], sP[3]);
+                if (aux) {   // the frame exponents, for the backward: Ê = e 2^(g - ae), K̃ = k 2^(ak - g)
+                    float *xe = reinterpret_cast<float *>(aux_of(j) + X_AE), *xk = reinterpret_cast<float *>(aux_of(j) + X_AK);
+                    *reinterpret_cast<float4 *>(xe + c4) = make_float4(m2[0], m2[1], m2[2], m2[3]);
+                    *reinterpret_cast<float4 *>(xk + c4) = wide ? make_float4(gC[0], gC[1], gC[2], gC[3])
+                                                                : make_float4(m2[0], m2[1], m2[2], m2[3]);
+                }
             }
 
             // ---------------------------------------------------------------- build (in place)
@@ -401,6 +400,39 @@ __global__ void __launch_bounds__(P1_NT, 1)
                     float f1[4];
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) f1[jj] = fast_exp2(pre[jj] + fast_log2(al[0][jj]) - m2[jj]);
+                    if (EXACT_F) {
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            const int r = p0 + p;
+                            if (p > 0)
+#pragma unroll
+                                for (int jj = 0; jj < 4; ++jj) f1[jj] *= al[p][jj];
+                            const float2 q01 = unpack2(rq[p].x), q23 = unpack2(rq[p].y);
+                            const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
+                            const float2 b01 = unpack2(rb[p].x), b23 = unpack2(rb[p].y);
+                            const float sk = ik(p), sq = iq(p);
+                            *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(r, c4, 128)) =
+                                make_uint2(pack_bf16(b01.x * k01.x * (f1[0] * sk), b01.y * k01.y * (f1[1] * sk)),
+                                           pack_bf16(b23.x * k23.x * (f1[2] * sk), b23.y * k23.y * (f1[3] * sk)));
+                            *reinterpret_cast<uint2 *>(S + P1_EQ + sw_off(64 + r, c4, 128)) =
+                                make_uint2(pack_bf16(q01.x * (f1[0] * sq), q01.y * (f1[1] * sq)),
+                                           pack_bf16(q23.x * (f1[2] * sq), q23.y * (f1[3] * sq)));
+                        }
+                        float f2[4];
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) f2[jj] = fast_exp2(m2[jj] - (pre[jj] + lw[jj]));
+#pragma unroll
+                        for (int p = 7; p >= 0; --p) {
+                            const int r = p0 + p;
+                            const float2 k01 = unpack2(rk[p].x), k23 = unpack2(rk[p].y);
+                            const float sk = ik(p);
+                            *reinterpret_cast<uint2 *>(S + P1_KT + sw_off(r, c4, 64)) =
+                                make_uint2(pack_bf16(k01.x * (f2[0] * sk), k01.y * (f2[1] * sk)),
+                                           pack_bf16(k23.x * (f2[2] * sk), k23.y * (f2[3] * sk)));
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) f2[jj] *= al[p][jj];
+                        }
+                    } else {
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
                         const int r = p0 + p;
@@ -427,6 +459,7 @@ __global__ void __launch_bounds__(P1_NT, 1)
                                        bmul2(rk[p].y, pack_bf16(f2[2] * ik(p), f2[3] * ik(p))));
 #pragma unroll
                         for (int jj = 0; jj < 4; ++jj) f2[jj] *= al[p][jj];
+                    }
                     }
                 } else {
                     float run[4] = {pre[0], pre[1], pre[2], pre[3]};
@@ -531,6 +564,10 @@ __global__ void __launch_bounds__(P1_NT, 1)
                 bulk_s2g(rec + R_KT, smem_u32(S + P1_KT), 16384);
                 bulk_s2g(rec + R_A3 + 8192, aEQ + 8192, 8192);       // Q̂: rows 64-127 of both column
                 bulk_s2g(rec + R_A3 + 24576, aEQ + 24576, 8192);     // halves of [-W'; Q̂]
+                if (aux) {   // Ê (rows 0-63 of both halves), for the backward
+                    bulk_s2g(aux_of(j) + X_E, aEQ, 8192);
+                    bulk_s2g(aux_of(j) + X_E + 8192, aEQ + 16384, 8192);
+                }
             }
             // ---------------------------------------------------------------- T = (I + A)^-1, duplicated as [T; T]
             solve_unit_lower(AS, reinterpret_cast<float *>(sm + P1_X), S + P1_W, tb, BAR_B);
@@ -545,6 +582,7 @@ __global__ void __launch_bounds__(P1_NT, 1)
             group_sync(BAR_B, 128);
             // ---------------------------------------------------------------- G2: [W'; W'] = [T; T] Ê, [Ũ; Ũ] = [T; T] U
             if (tb == 0) {
+                if (aux) bulk_s2g(aux_of(j) + X_T, aW, 8192);   // T, for the backward
                 fence_after();
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj)
@@ -555,6 +593,13 @@ __global__ void __launch_bounds__(P1_NT, 1)
                 mma_commit(misc + M1_G2);
             }
             if (!gwait(misc + M1_G2, (uint32_t)(j & 1), BAR_B, 128, abort)) break;
+            if (aux) {   // the copy of Ê has read rows 0-63 before -W' overwrites them
+                if (tb == 0) {
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                group_sync(BAR_B, 128);
+            }
             {   // lanes 0-63 (warps 8, 9): -W' rows into the [-W'; Q̂] tile; lanes 64-127 (warps 10, 11): the
                 // same rows of Ũ into the U tile; bf16
                 const int i = 32 * (wb & 1) + lane;
@@ -687,18 +732,10 @@ __device__ __forceinline__ void store_o(const CUtensorMap *map_o, unsigned char 
     }
 }
 
-// Launch flags of the segmented walk (few long chains): block blockIdx.x walks segment
-// blockIdx.x % nseg (chunks [seg * seg_len, (seg + 1) * seg_len) of the window) of chain
-// blockIdx.x / nseg; S0 and S_T are then indexed by block.
-enum : uint32_t {
-    WALK_ZERO_WRITES = 1,   // Ũ = 0: the walk propagates the state only (the segment's homogeneous map)
-    WALK_SKIP_O = 2,        // o is not stored
-    WALK_IDENTITY_S0 = 4,   // the segment starts from S = I (d_k = d_v)
-    WALK_ST_LAST = 8,       // only the chain's last segment stores S_T, at S_T[chain]
-};
 
 __global__ void __launch_bounds__(W2_NT, 1)
-    walk_kernel(const __grid_constant__ CUtensorMap map_o, const unsigned char *records, const float *S0, float *ST,
+    walk_kernel(const __grid_constant__ CUtensorMap map_o, const unsigned char *records, unsigned char *aux,
+                const float *S0, float *ST,
                 int H, int T, int n0, int nw, int nseg, int seg_len, uint32_t flags, const float *onorm,
                 unsigned int *status) {
     extern __shared__ unsigned char smem_raw[];
@@ -732,6 +769,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
     auto slot_addr = [&](int n) { return W2_SLOT + (uint32_t)(n & 1) * R_BYTES; };
     auto d3 = [&](int n) { return tmem + W2_TM_D3 + 128u * (uint32_t)(n & 1); };
     auto rec_of = [&](int nl) { return records + ((size_t)(bb * nw + c0 + nl) * H + h) * R_BYTES; };
+    auto aux_of = [&](int nl) { return aux + ((size_t)(bb * nw + c0 + nl) * H + h) * X_BYTES; };
 
     if (warp < 8) {
         const int q4 = warp & 3, cb = 64 * (warp >> 2);   // TMEM lane quarter, value-column half
@@ -764,6 +802,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
             const uint32_t slot = slot_addr(nl);
             // ---------------------------------------------------------------- record n in, chunk n-1 done
             {
+                if (aux && tid == 0) bulk_wait_read_all();   // the copies of Z̃ and Delta have read them
                 bool w_ok = mbar_wait(misc + M2_FULL + 8 * (nl & 1), (uint32_t)((nl >> 1) & 1), WAIT_LIMIT);
                 if (nl > 0)
                     w_ok = w_ok && mbar_wait(misc + M2_G5 + 8 * ((nl - 1) & 1), (uint32_t)(((nl - 1) >> 1) & 1), WAIT_LIMIT);
@@ -808,6 +847,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
                     for (int j = 0; j < 8; ++j)
                         mma_ss(d3(nl), desc_kmajor(aA3, 128, j), desc_mnmajor(aS, 128, j), ID_G3, j > 0);
                     mma_commit(misc + M2_G3);
+                    if (aux) {   // the state operand of the chunk, for the backward
+                        bulk_s2g(aux_of(nl) + X_Z, aS, 32768);
+                        bulk_commit();
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -856,6 +899,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
                 fence_async_smem();
                 fence_before();
                 group_sync(BAR_DELTA, 128);
+                if (aux && tid == 0) {   // Delta of the chunk, for the backward
+                    bulk_s2g(aux_of(nl) + X_DL, smem_u32(sm + W2_DL), 16384);
+                    bulk_commit();
+                }
                 if (tid == 0) {   // G4: O += P Delta (rows 0-63 of the A tile are Ũ's bytes: their products
                                   // land in the Delta rows of D3, already read); G5: Z += K̃^T Delta, once the
                                   // o warps' rows of Z are written back
@@ -896,6 +943,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
             }
         }
         if (!is_delta && ot == 0) bulk_wait_all();   // the o stores complete before the block exits
+        if (aux && tid == 0) bulk_wait_all();
     } else if (lane == 0) {
         // ------------------------------------------------------------------ producer: one bulk copy per record
         for (int nl = 0; nl < nc; ++nl) {
@@ -930,10 +978,9 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A [B, T, H, 128] token tensor as the 4-D map (d, H, T, B).  bf16: a 64 x 1 x 64 x 1 box in the 128-byte
-// swizzle, one box being the 64 x 64 half-tile of the operand layout; fp32 (alpha): a 128 x 1 x 64 x 1
-// box, rows of 512 bytes.  Rows past T read as zero.
-bool token_map(CUtensorMap *m, const void *base, int B, int T, int H, bool fp32 = false) {
+}  // namespace
+
+bool token_map(CUtensorMap *m, const void *base, int B, int T, int H, bool fp32) {
     const EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t es_bytes = fp32 ? 4 : 2;
@@ -952,6 +999,8 @@ int sm_count() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     return n;
 }
+
+namespace {
 
 // Plan of a two-stage call.  The record buffer holds one window of chunks of every chain (at most
 // 16,384 chunk-heads, 1.24 GB, and at least 64 chunks).  With few chains (B*H <= 64) each chain's
@@ -972,6 +1021,11 @@ SplitPlan split_plan(int B, int H, int T) {
     return {nw, nseg};
 }
 constexpr size_t kStateBytes = sizeof(float) * 128 * 128;
+// segments per chain of the backward's forward replay (one window of the whole sequence)
+int replay_segments(int chains, int NC) {
+    if (chains > 64 || NC < 32) return 1;
+    return std::max(1, std::min(128 / std::max(chains, 1), NC / 8));
+}
 
 }  // namespace
 
@@ -1008,27 +1062,76 @@ int launch_chunk_split(const void *q, const void *k, const void *v, const float 
         const int nw = std::min(plan.nw, NC - n0), nch = chains * nw;
         const float *s_in = n0 == 0 ? S0 : ST;
         prep<<<std::min(nch, nsm), split::P1_NT, smem1, st>>>(
-            maps, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)b, alpha, records, H, T,
-            n0, nw, nch, status);
+            maps, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)b, alpha, records, nullptr,
+            H, T, n0, nw, nch, status);
         int nseg = plan.nseg > 1 && nw >= 16 ? std::min(plan.nseg, nw / 8) : 1;
         if (nseg <= 1) {
-            split::walk_kernel<<<chains, split::W2_NT, smem2, st>>>(map_o, records, s_in, ST, H, T, n0, nw, 1, nw, 0u,
-                                                                    onorm, status);
+            split::walk_kernel<<<chains, split::W2_NT, smem2, st>>>(map_o, records, nullptr, s_in, ST, H, T, n0, nw, 1,
+                                                                    nw, 0u, onorm, status);
             continue;
         }
         const int seg_len = (nw + nseg - 1) / nseg;
         nseg = (nw + seg_len - 1) / seg_len;   // every segment non-empty
         const uint32_t skip = split::WALK_SKIP_O;
-        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, nullptr, Nm, H, T, n0, nw, nseg,
-                                                                       seg_len, skip, onorm, status);
+        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, nullptr, nullptr, Nm, H, T, n0,
+                                                                       nw, nseg, seg_len, skip, onorm, status);
         split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(
-            map_o, records, nullptr, Mm, H, T, n0, nw, nseg, seg_len,
+            map_o, records, nullptr, nullptr, Mm, H, T, n0, nw, nseg, seg_len,
             skip | split::WALK_ZERO_WRITES | split::WALK_IDENTITY_S0, onorm, status);
         const int rc = launch_segment_scan(Mm, Nm, s_in, Sg, chains, nseg, st);
         if (rc != 0) return rc;
-        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, Sg, ST, H, T, n0, nw, nseg,
-                                                                       seg_len, split::WALK_ST_LAST, onorm, status);
+        split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(map_o, records, nullptr, Sg, ST, H, T, n0, nw,
+                                                                       nseg, seg_len, split::WALK_ST_LAST, onorm, status);
     }
+    return launch_status();
+}
+
+// Forward replay for the backward: the two stages over the whole sequence at once (one window), o not
+// stored, every chunk-head's side record filled (Ê, T and the frame exponents by the first stage, Z̃ and
+// Delta by the final walk), S_T written.  Few long chains walk in segments as in the prefill.
+size_t replay_segment_bytes(int B, int H, int T) {
+    const int chains = B * H, NC = (T + split::C - 1) / split::C;
+    const int nseg = replay_segments(chains, NC);
+    return nseg > 1 ? 3 * kStateBytes * (size_t)chains * nseg : 0;
+}
+
+int launch_split_replay(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                        const float *S0, float *ST, int B, int H, int T, unsigned char *records, unsigned char *aux,
+                        float *seg, const CUtensorMap &any_map, unsigned int *status, cudaStream_t st) {
+    split::TokMaps maps;
+    if (!token_map(&maps.q, q, B, T, H) || !token_map(&maps.k, k, B, T, H) || !token_map(&maps.b, b, B, T, H) ||
+        !token_map(&maps.v, v, B, T, H) || !token_map(&maps.w, w, B, T, H) ||
+        !token_map(&maps.alpha, alpha, B, T, H, true))
+        return -6;
+    const int smem1 = (int)split::P1_BYTES, smem2 = (int)split::W2_BYTES;
+    if (cudaFuncSetAttribute(split::prep_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess ||
+        cudaFuncSetAttribute(split::walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
+        return -6;
+    const int nsm = sm_count();
+    if (nsm <= 0) return -6;
+    const int chains = B * H, NC = (T + split::C - 1) / split::C, nch = chains * NC;
+    split::prep_kernel<false, true><<<std::min(nch, nsm), split::P1_NT, smem1, st>>>(
+        maps, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)b, alpha, records, aux, H, T,
+        0, NC, nch, status);
+    int nseg = replay_segments(chains, NC);
+    const uint32_t skip = split::WALK_SKIP_O;
+    if (nseg <= 1) {
+        split::walk_kernel<<<chains, split::W2_NT, smem2, st>>>(any_map, records, aux, S0, ST, H, T, 0, NC, 1, NC, skip,
+                                                                nullptr, status);
+        return launch_status();
+    }
+    const int seg_len = (NC + nseg - 1) / nseg;
+    nseg = (NC + seg_len - 1) / seg_len;
+    float *Nm = seg, *Mm = Nm + (size_t)chains * nseg * 128 * 128, *Sg = Mm + (size_t)chains * nseg * 128 * 128;
+    split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(any_map, records, nullptr, nullptr, Nm, H, T, 0, NC,
+                                                                   nseg, seg_len, skip, nullptr, status);
+    split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(
+        any_map, records, nullptr, nullptr, Mm, H, T, 0, NC, nseg, seg_len,
+        skip | split::WALK_ZERO_WRITES | split::WALK_IDENTITY_S0, nullptr, status);
+    const int rc = launch_segment_scan(Mm, Nm, S0, Sg, chains, nseg, st);
+    if (rc != 0) return rc;
+    split::walk_kernel<<<chains * nseg, split::W2_NT, smem2, st>>>(any_map, records, aux, Sg, ST, H, T, 0, NC, nseg,
+                                                                   seg_len, skip | split::WALK_ST_LAST, nullptr, status);
     return launch_status();
 }
 

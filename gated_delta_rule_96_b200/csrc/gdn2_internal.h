@@ -61,4 +61,12 @@ int launch_chunk_bwd(const void *q, const void *k, const void *v, const float *a
                      float *dalpha, float *db, float *dw, float *dS0, int B, int H, int T, int K, int V, int bf16,
                      void *ws, cudaStream_t st);
 
+// Tensor-core backward (bf16 tokens, d_k = d_v = 128): forward replay by the two-stage prefill's kernels,
+// reverse walk of the state gradient, gradient kernel over every chunk-head.
+size_t chunk_bwd_tc_workspace_bytes(int B, int H, int T);
+int launch_chunk_bwd_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b, const void *w,
+                        const float *S0, const void *dO, const float *dST, float *dq, float *dk, float *dv,
+                        float *dalpha, float *db, float *dw, float *dS0, int B, int H, int T, void *ws,
+                        cudaStream_t st);
+
 }  // namespace gdn2

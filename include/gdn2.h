@@ -181,6 +181,40 @@ GDN2_API int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const f
                             int T, int d_k, int d_v, int dtype, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/* Bytes of device workspace gdn2_chunk_bwd_tc needs (0 on bad or unsupported sizes): the 256-byte
+ * status header, then per chunk of 64 steps of every chain a 75,776-byte record of the forward's chunk
+ * factors and a 124,928-byte side record of the backward, the fp32 state at the end of every chain,
+ * and, when few chains are long (B*H <= 64 and at least 32 chunks), three fp32 states per time segment
+ * of each chain.  About 200 KB per 64 steps per chain; T = 0 needs the header only. */
+GDN2_API size_t gdn2_chunk_bwd_tc_workspace_bytes(int B, int H, int T, int d_k, int d_v);
+
+/*
+ * Backward pass on the tensor cores: the same gradients as gdn2_chunk_bwd (same arguments, layouts
+ * and output dtypes), for bf16 tokens with d_k = d_v = 128 (GDN2_ERR_UNSUPPORTED otherwise).  The
+ * chunkwise WY form with C = 64 (page "NVIDIA представила Gated DeltaNet-2 ...", the paragraph on the
+ * chunkwise kernels) is differentiated product by product: a forward replay by the two-stage prefill's
+ * kernels keeps each chunk's factors, one block per chain walks the chunks backwards with the state
+ * gradient resident in tensor memory, and one kernel over every chunk-head forms the token gradients
+ * from five tcgen05 products and the gate and decay terms.
+ *
+ * Accuracy: the products take bf16 operands (the chunk factors, the state and its gradient, dO) with
+ * fp32 accumulation, so each gradient carries the bf16 relative error of the forward's tensor-core
+ * path (about 1e-2 of the tensor's largest magnitude) rather than gdn2_chunk_bwd's fp32 one.  The state
+ * gradient is carried from chunk to chunk in fp32; d(ln alpha) sums fp32 terms over at most 64 steps.
+ *
+ *   workspace  device scratch of at least gdn2_chunk_bwd_tc_workspace_bytes(...) bytes, 16-byte
+ *              aligned, whose first 256 bytes are a status header zeroed once by the caller (the
+ *              kernels' bounded waits report there; read it with gdn2_workspace_status)
+ *
+ * T = 0 writes dS0 = dS_T (or zeros).  The output buffers must not alias the inputs or each other.
+ * Five to eight kernel launches on `stream`; results are deterministic.
+ */
+GDN2_API int gdn2_chunk_bwd_tc(const void *q, const void *k, const void *v, const float *alpha, const void *b,
+                               const void *w, const float *S0, const void *dO, const float *dS_T, float *dq,
+                               float *dk, float *dv, float *dalpha, float *db, float *dw, float *dS0, int B, int H,
+                               int T, int d_k, int d_v, int dtype, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
 /*
  * Measurement aid (not part of the recurrence): runs the tensor-core products of one chunk of the
  * chunkwise prefill -- G1 [A; P] = [Ê; Q̂] K̃^T (M128 N64 K128), G2 (2 x M128 N128 K64), G3 (M128 N128

@@ -27,7 +27,8 @@ def test_header_declares_entry_points():
     for name in ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_fwd_workspace_bytes", "gdn2_status_str",
                  "gdn2_workspace_status", "gdn2_chunk_fwd_path", "gdn2_chunk_fwd_edges",
                  "gdn2_chunk_fwd_edges_workspace_bytes", "gdn2_chunk_bwd", "gdn2_chunk_bwd_workspace_bytes",
-                 "gdn2_chunk_fwd_noalloc", "gdn2_gemm_phase_probe", "gdn2_layer_edge_maps", "gdn2_rms_norm"):
+                 "gdn2_chunk_fwd_noalloc", "gdn2_gemm_phase_probe", "gdn2_layer_edge_maps", "gdn2_rms_norm",
+                 "gdn2_chunk_bwd_tc", "gdn2_chunk_bwd_tc_workspace_bytes"):
         assert name in syms
 
 
@@ -169,6 +170,40 @@ def test_chunk_bwd_validation(lib):
     assert call_bwd(lib, B=0) == 0
     # no tokens and no dS0 wanted: nothing to do, no pointer read
     assert call_bwd(lib, T=0, ptr=None, grad=None, ws=None, ws_bytes=0) == 0
+
+
+def test_bwd_tc_workspace_bytes():
+    rec, side, state = 75776, 124928, 4 * 128 * 128
+    # status header, a record and a side record per chunk-head, the end state of every chain
+    assert g.gdn2_chunk_bwd_tc_workspace_bytes(8, 16, 4096, 128, 128) == 256 + 8 * 16 * 64 * (rec + side) + 128 * state
+    assert g.gdn2_chunk_bwd_tc_workspace_bytes(2, 3, 65, 128, 128) == 256 + 6 * 2 * (rec + side) + 6 * state
+    # few long chains: the replay walks 41 chunks in min(128 / 2, 41 // 8) = 5 segments per chain, three
+    # fp32 states per segment
+    assert g.gdn2_chunk_bwd_tc_workspace_bytes(1, 2, 64 * 40 + 37, 128, 128) == \
+        256 + 2 * 41 * (rec + side) + 2 * state + 3 * state * 2 * 5
+    assert g.gdn2_chunk_bwd_tc_workspace_bytes(1, 1, 8, 64, 128) == 0
+    assert g.gdn2_chunk_bwd_tc_workspace_bytes(1, 1, 0, 128, 128) == 256
+
+
+def call_bwd_tc(lib, B=1, H=1, T=8, K=128, V=128, dtype=1, ptr=FAKE, grad=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return lib.gdn2_chunk_bwd_tc(*(ptr,) * 6, None, ptr, None, *(grad,) * 6, None, B, H, T, K, V, dtype, ws,
+                                 ws_bytes, None)
+
+
+def test_chunk_bwd_tc_validation(lib):
+    assert call_bwd_tc(lib, T=-1) == -2
+    assert call_bwd_tc(lib, dtype=5) == -3
+    assert call_bwd_tc(lib, dtype=0) == -4     # fp32 tokens: gdn2_chunk_bwd
+    assert call_bwd_tc(lib, K=64) == -4
+    assert call_bwd_tc(lib, V=64) == -4
+    assert call_bwd_tc(lib, ptr=None) == -1
+    assert call_bwd_tc(lib, grad=None) == -1
+    assert call_bwd_tc(lib, ptr=P(0x10004)) == -7
+    assert call_bwd_tc(lib, grad=P(0x10008)) == -7
+    assert call_bwd_tc(lib, ws=None) == -5
+    assert call_bwd_tc(lib, ws_bytes=1024) == -5
+    assert call_bwd_tc(lib, B=0) == 0
+    assert call_bwd_tc(lib, T=0, ptr=None, grad=None, ws=None, ws_bytes=0) == 0
 
 
 def test_edges_workspace_bytes():
