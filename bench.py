@@ -61,6 +61,25 @@ def backward_flops(B, T, H, K, V):
     return 21 * B * T * H * K * V
 
 
+def backward_bytes(B, T, H, K, V, tok_bytes=2):
+    """Algorithmic HBM bytes of one backward call: the forward's inputs and dO read once, the six
+    fp32 token gradients written once, dS_T read and dS0 written (S0 = 0 in the workload)."""
+    per_token_head = (3 * K + 2 * V) * tok_bytes + 4 * K + V * tok_bytes + 4 * (4 * K + 2 * V)
+    return B * T * H * per_token_head + 2 * 4 * B * H * K * V
+
+
+def backward_tc_mma_flops(B, T, H, K, V, C=64):
+    """Flops of the tensor-core products the tensor-core backward issues per chunk-head (its M = 128
+    tiles included): the forward replay (G1, G2, G3, G4, G5), the reverse walk (dDelta^T = dO^T P +
+    G^T K^T, dY += [-W'; Q]^T [dDelta; dO]) and the gradient kernel (T^T dDelta, [dA; dP], [dE; dQ],
+    dK)."""
+    m = 128
+    replay = 2 * m * C * K + 2 * 2 * m * V * C + 2 * m * V * K + 2 * 2 * m * V * C
+    rwalk = 2 * m * C * C + 2 * m * C * K + 2 * m * V * 2 * C
+    grad = 2 * m * V * C + 2 * m * C * V + 2 * m * K * V + 2 * m * K * C + 2 * m * K * V + 2 * 2 * m * K * C
+    return B * H * ((T + C - 1) // C) * (replay + rwalk + grad)
+
+
 def fp32_alu_peak_tflops(n_sm, sm_mhz):
     """Dense fp32 FMA peak from unit counts and clock: 128 fp32 lanes per SM, 2 flops per FMA."""
     return n_sm * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -733,7 +752,24 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=
     bwd_ms = timed(lambda: g.gdn2_chunk_bwd(X["q"], X["k"], X["v"], X["alpha"], X["b"], X["w"], None, dO, dST,
                                             grads["dq"], grads["dk"], grads["dv"], grads["dalpha"], grads["db"],
                                             grads["dw"], dS0, workspace=wsb, stream=stream))
-    del grads, dS0, wsb, X, dO, dST
+    wst = g.new_workspace(g.gdn2_chunk_bwd_tc_workspace_bytes(B, H, T, K, V), dev)
+    bwd_tc_ms = timed(lambda: g.gdn2_chunk_bwd_tc(X["q"], X["k"], X["v"], X["alpha"], X["b"], X["w"], None, dO,
+                                                  dST, grads["dq"], grads["dk"], grads["dv"], grads["dalpha"],
+                                                  grads["db"], grads["dw"], dS0, workspace=wst, stream=stream))
+    if g.gdn2_workspace_status(wst) != 0:
+        raise RuntimeError("tensor-core backward reported an internal error")
+    del grads, dS0, wsb, wst, X, dO, dST
+    peaks = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tc_bytes = backward_bytes(B, T, H, K, V)
+    tc_gbs = tc_bytes / (bwd_tc_ms * 1e-3) / 1e9
+    backward_tc = {"ms": bwd_tc_ms, "tokens_per_s": B * T / (bwd_tc_ms * 1e-3), "launches": 4,
+                   "kernels": "prep_kernel + walk_kernel (forward replay), rwalk_kernel, grad_kernel",
+                   "roofline": {"bound": "hbm", "achieved": tc_gbs, "peak": hbm, "unit": "GB/s",
+                                "frac": tc_gbs / hbm, "algorithmic_bytes_per_launch": tc_bytes,
+                                "traffic": recorded_traffic("backward_tc"),
+                                "peak_src": peaks["src"],
+                                "tensor_tflops": backward_tc_mma_flops(B, T, H, K, V) / (bwd_tc_ms * 1e-3) / 1e12}}
     n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
     sm_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
     peak = fp32_alu_peak_tflops(n_sm, sm_mhz)
@@ -777,11 +813,12 @@ def run_next_rows(g, torch, dev, stream, wl, plain_prefill_ms, clocks, with_cpu=
              "inputs": "raw q, k ~ N(0, 9), decay logit ~ N(1, 1) (alpha = exp(-softplus(a)): the plain "
                        "workload's alpha distribution), gate logits ~ N(0, 1)"}
     out = {"workload": f"{wl.name} (B{B} H{H} T{T} d_k=d_v={K}, bf16 tokens)", "backward": backward,
-           "edges_prefill": edges}
+           "backward_tc": backward_tc, "edges_prefill": edges}
     if with_cpu:
         try:
             cpu = oracle_next_rows_sample(wl)
             backward["cpu_baseline"], edges["cpu_baseline"] = cpu["backward"], cpu["edges_prefill"]
+            backward_tc["cpu_baseline"] = cpu["backward"]
         except Exception as e:   # the CPU figures are context: never lose the GPU line over them
             backward["cpu_baseline"] = edges["cpu_baseline"] = {"unavailable": repr(e)[:200]}
     try:

@@ -395,10 +395,12 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
 }
 
 __global__ void __launch_bounds__(GK_NT, 1)
-    grad_kernel(const __grid_constant__ CUtensorMap map_do, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
-                const __nv_bfloat16 *v, const __nv_bfloat16 *b, const __nv_bfloat16 *w, const float *alpha,
-                const unsigned char *records, const unsigned char *aux, float *dq, float *dk, float *dv, float *dalpha,
-                float *db, float *dw, int H, int T, int NC, unsigned int *status) {
+    grad_kernel(const __grid_constant__ CUtensorMap map_do, const __nv_bfloat16 *__restrict__ q,
+                const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+                const __nv_bfloat16 *__restrict__ b, const __nv_bfloat16 *__restrict__ w,
+                const float *__restrict__ alpha, const unsigned char *records, const unsigned char *aux,
+                float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dalpha,
+                float *__restrict__ db, float *__restrict__ dw, int H, int T, int NC, unsigned int *status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -680,12 +682,17 @@ __global__ void __launch_bounds__(GK_NT, 1)
         if (tid < 128) {
             const float rho = vecs[256 + cc];
             float acc = 0.f;
-#pragma unroll 8
-            for (int rr = 63; rr >= 0; --rr) {
-                acc += H1[rr * GLD + cc] + HQ[rr * GLD + cc];
-                if (rr < L) {
-                    const size_t o = (((size_t)bb * T + t0 + rr) * H + h) * KD + cc;
-                    dalpha[o] = (acc + rho) / fmaxf(alpha[o], FLT_MIN);
+#pragma unroll 1
+            for (int r0 = 32; r0 >= 0; r0 -= 32) {
+                float al[32];   // 32 rows of alpha in flight at once, ahead of their stores
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    al[i] = r0 + i < L ? alpha[(((size_t)bb * T + t0 + r0 + i) * H + h) * KD + cc] : 1.f;
+#pragma unroll
+                for (int i = 31; i >= 0; --i) {
+                    const int rr = r0 + i;
+                    acc += H1[rr * GLD + cc] + HQ[rr * GLD + cc];
+                    if (rr < L) dalpha[(((size_t)bb * T + t0 + rr) * H + h) * KD + cc] = (acc + rho) / fmaxf(al[i], FLT_MIN);
                 }
             }
         }
