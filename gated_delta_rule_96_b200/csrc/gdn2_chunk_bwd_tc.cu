@@ -336,8 +336,8 @@ constexpr uint32_t G_E = 139264;     // Ê [r x c]              (MN-major B of D
 constexpr uint32_t G_Q = 155648;     // Q̂ [r x c]              (MN-major B of D4)
 constexpr uint32_t G_G = 172032;     // G̃ [c x v]              (K-major B of D4)
 constexpr uint32_t G_MISC = 204800;
-constexpr uint32_t G_VEC = G_MISC + 256;   // ae, ak, rho: 3 x 128 fp32
-constexpr uint32_t G_BYTES = G_VEC + 1536 + 1024;
+constexpr uint32_t G_VEC = G_MISC + 256;   // ae, ak, rho, then two [128] hand-over sums: 5 x 128 fp32
+constexpr uint32_t G_BYTES = G_VEC + 2560 + 1024;
 // fp32 [64][GLD] arrays of the epilogue, over operand images that are dead by then ([dA; dP] stays: a
 // wide-span chunk reads it once more)
 constexpr int GLD = 132;
@@ -451,6 +451,9 @@ __global__ void __launch_bounds__(GK_NT, 1)
     const uint32_t lq = (uint32_t)(32 * q4) << 16;
     const int r = 32 * (q4 & 1) + lane;             // chunk row of this thread's TMEM lane (mod 64)
     const size_t row = ((size_t)bb * T + t0 + r) * H + h;   // its token row (valid when r < L)
+    // loads read row min(r, L - 1), always inside the tensor: a load under a condition on the row
+    // cannot be issued ahead of the branch, and each would then wait out its own memory latency
+    const size_t lrow = ((size_t)bb * T + t0 + min(r, L - 1)) * H + h;
     bool ok = true;
     uint32_t committed = 0;   // tid 0: the last MMA barrier committed (for the exit)
 
@@ -474,12 +477,10 @@ __global__ void __launch_bounds__(GK_NT, 1)
     // ---------------------------------------------------------------- R1: -dR -> [-dR; dO]; dv, dw
     if (q4 < 2) {
         uint4 vv[8], ww[8];
-        if (r < L) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                vv[u] = *reinterpret_cast<const uint4 *>(v + row * VD + cb + 8 * u);
-                ww[u] = *reinterpret_cast<const uint4 *>(w + row * VD + cb + 8 * u);
-            }
+        for (int u = 0; u < 8; ++u) {
+            vv[u] = *reinterpret_cast<const uint4 *>(v + lrow * VD + cb + 8 * u);
+            ww[u] = *reinterpret_cast<const uint4 *>(w + lrow * VD + cb + 8 * u);
         }
         ok = mbar_wait(misc + MG_M1, 0, WAIT_LIMIT) && !*abort;
         if (!ok) *abort = 1u;
@@ -566,23 +567,29 @@ __global__ void __launch_bounds__(GK_NT, 1)
         }
     }
     // ---------------------------------------------------------------- the log2-decay prefix, while the products run
-    float gpre[64];
-    const int cc = tid & 127;   // tid < 128: channel of the prefix
-    if (ok && tid < 128) {
+    // Thread tid: channel cc, rows 32 hh .. 32 hh + 31.  Every alpha of the thread is loaded before the
+    // first is used; the upper half adds the lower half's total (handed over in shared memory).
+    const int cc = tid & 127, hh = tid >> 7;
+    auto alpha_at = [&](int rr) { return alpha[(((size_t)bb * T + t0 + min(rr, L - 1)) * H + h) * KD + cc]; };
+    float gpre[32];
+    if (ok) {
+        float al[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) al[i] = alpha_at(32 * hh + i);
         float g = 0.f;
 #pragma unroll
-        for (int rr = 0; rr < 64; ++rr) {
-            const float a = rr < L ? fmaxf(alpha[(((size_t)bb * T + t0 + rr) * H + h) * KD + cc], FLT_MIN) : 1.f;
-            g += fast_log2(a);
-            gpre[rr] = g;
+        for (int i = 0; i < 32; ++i) {
+            g += fast_log2(32 * hh + i < L ? fmaxf(al[i], FLT_MIN) : 1.f);
+            gpre[i] = g;
         }
+        if (hh == 0) vecs[384 + cc] = g;
     }
     if (ok) ok = group_wait(misc + MG_M4, 0, GBAR, 256, abort);
     if (ok) {
         float *pre = reinterpret_cast<float *>(sm + G_PRE);
-        if (tid < 128)
+        const float base = hh ? vecs[384 + cc] : 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 64; ++rr) pre[rr * GLD + cc] = gpre[rr];
+        for (int i = 0; i < 32; ++i) pre[(32 * hh + i) * GLD + cc] = base + gpre[i];
         group_sync(GBAR, 256);
         // -------------------------------------------------------------- row phase
         const float *ae = vecs, *ak = vecs + 128;
@@ -596,15 +603,12 @@ __global__ void __launch_bounds__(GK_NT, 1)
             tmem_ld32(tmem + lq + GT_D3 + c0, x);
             if (rows_ek) tmem_ld32(tmem + lq + GT_D4 + c0, y);
             uint4 t1[4], t2[4];
-            if (r < L) {
+            {
+                const __nv_bfloat16 *x1 = rows_ek ? b : q;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    if (rows_ek) {
-                        t1[u] = *reinterpret_cast<const uint4 *>(b + row * KD + c0 + 8 * u);
-                        t2[u] = *reinterpret_cast<const uint4 *>(k + row * KD + c0 + 8 * u);
-                    } else {
-                        t1[u] = *reinterpret_cast<const uint4 *>(q + row * KD + c0 + 8 * u);
-                    }
+                    t1[u] = *reinterpret_cast<const uint4 *>(x1 + lrow * KD + c0 + 8 * u);
+                    if (rows_ek) t2[u] = *reinterpret_cast<const uint4 *>(k + lrow * KD + c0 + 8 * u);
                 }
             }
             wait_ld();
@@ -679,21 +683,26 @@ __global__ void __launch_bounds__(GK_NT, 1)
         }
         group_sync(GBAR, 256);
         // -------------------------------------------------------------- decay: reverse sums over the chunk
-        if (tid < 128) {
+        {   // thread tid: channel cc, rows 32 hh .. 32 hh + 31; the lower half starts from the upper
+            // half's total (handed over in shared memory)
             const float rho = vecs[256 + cc];
-            float acc = 0.f;
-#pragma unroll 1
-            for (int r0 = 32; r0 >= 0; r0 -= 32) {
-                float al[32];   // 32 rows of alpha in flight at once, ahead of their stores
+            float al[32], hs[32], tot = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    al[i] = r0 + i < L ? alpha[(((size_t)bb * T + t0 + r0 + i) * H + h) * KD + cc] : 1.f;
+            for (int i = 0; i < 32; ++i) al[i] = alpha_at(32 * hh + i);
 #pragma unroll
-                for (int i = 31; i >= 0; --i) {
-                    const int rr = r0 + i;
-                    acc += H1[rr * GLD + cc] + HQ[rr * GLD + cc];
-                    if (rr < L) dalpha[(((size_t)bb * T + t0 + rr) * H + h) * KD + cc] = (acc + rho) / fmaxf(al[i], FLT_MIN);
-                }
+            for (int i = 0; i < 32; ++i) {
+                const int rr = 32 * hh + i;
+                hs[i] = H1[rr * GLD + cc] + HQ[rr * GLD + cc];
+                tot += hs[i];
+            }
+            if (hh == 1) vecs[512 + cc] = tot;
+            group_sync(GBAR, 256);
+            float acc = hh ? 0.f : vecs[512 + cc];
+#pragma unroll
+            for (int i = 31; i >= 0; --i) {
+                const int rr = 32 * hh + i;
+                acc += hs[i];
+                if (rr < L) dalpha[(((size_t)bb * T + t0 + rr) * H + h) * KD + cc] = (acc + rho) / fmaxf(al[i], FLT_MIN);
             }
         }
     }
