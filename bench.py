@@ -417,6 +417,21 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     parts = set(args.parts.split(","))
+    if "backward_tc" in parts:   # profiling aid: the tensor-core backward on the prefill workload
+        dO_np, dST_np = synth.make_output_grads(pw)
+        BW = {"dO": torch.from_numpy(dO_np).to(dev).to(torch.bfloat16), "dST": torch.from_numpy(dST_np).to(dev),
+              "dS0": torch.empty((B, H, K, V), dtype=torch.float32, device=dev),
+              "ws": g.new_workspace(g.gdn2_chunk_bwd_tc_workspace_bytes(B, H, T, K, V), dev)}
+        for n in ("dq", "dk", "dv", "dalpha", "db", "dw"):
+            BW[n] = torch.empty((B, T, H, K), dtype=torch.float32, device=dev)
+        del dO_np, dST_np
+
+    def backward_tc():
+        if "backward_tc" not in parts:
+            return
+        g.gdn2_chunk_bwd_tc(P["q"], P["k"], P["v"], P["alpha"], P["b"], P["w"], None, BW["dO"], BW["dST"], BW["dq"],
+                            BW["dk"], BW["dv"], BW["dalpha"], BW["db"], BW["dw"], BW["dS0"], workspace=BW["ws"],
+                            stream=stream)
 
     def prefill():
         if "prefill" not in parts:
@@ -432,7 +447,10 @@ def run_ours(args):
     for _ in range(args.warmup):
         prefill()
         decode()
+        backward_tc()
     torch.cuda.synchronize(dev)
+    if "backward_tc" in parts and g.gdn2_workspace_status(BW["ws"]) != 0:
+        raise SystemExit("backward kernels reported an internal error during warm-up")
     if g.gdn2_workspace_status(ws) != 0:
         raise SystemExit("prefill kernel reported an internal error during warm-up")
 
@@ -449,6 +467,7 @@ def run_ours(args):
             b_.record(stream)
             decode()
             c.record(stream)
+            backward_tc()
         stop.record(stream)
         torch.cuda.synchronize(dev)
     barrier(pg)
@@ -845,7 +864,8 @@ def main(argv=None):
     ap.add_argument("--prefill-shape", default="",
                     help="profiling aid: B,H,T of the prefill instead of the bench workload (not a bench line)")
     ap.add_argument("--parts", default="prefill,decode",
-                    help="profiling aid: run only some parts of the step (the default runs the whole step)")
+                    help="profiling aid: run only some parts of the step (the default runs the whole step); "
+                         "'backward_tc' adds the tensor-core backward on the prefill workload")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
