@@ -111,6 +111,11 @@ def test_backward_accounting():
     assert bench.backward_flops(8, 4096, 16, 128, 128) == 21 * 8 * 4096 * 16 * 128 * 128 == 180388626432
     # 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz
     assert abs(bench.fp32_alu_peak_tflops(148, 1965.0) - 74.44992) < 1e-9
+    # tensor-core backward: q, k, v, b, w, dO bf16 and alpha fp32 read, six fp32 gradients written (5,120 B
+    # per token-head), dS_T read and dS0 written per chain
+    assert bench.backward_bytes(1, 1, 1, 128, 128) == 5120 + 2 * 4 * 128 * 128
+    assert bench.backward_bytes(8, 4096, 16, 128, 128) == 8 * 4096 * 16 * 5120 + 2 * 4 * 128 * 128 * 128
+    assert bench.backward_tc_mma_flops(8, 4096, 16, 128, 128) == 128 * 64 * bench.backward_tc_mma_flops(1, 64, 1, 128, 128)
 
 
 def test_oracle_next_rows_sample_small():
@@ -162,6 +167,7 @@ def test_next_rows_run_on_cpu_through_the_binding(rec, monkeypatch):
     out = bench.run_next_rows(g, FakeTorch(), "cpu", None, wl, 0.5, {"sm_max_mhz": 1965.0})
     names = [c[0] for c in rec.calls]
     assert names.count("gdn2_chunk_bwd") == 7 and names.count("gdn2_chunk_fwd_edges") == 7
+    assert names.count("gdn2_chunk_bwd_tc") == 7
     # segmented row 7; unfused edge layer 7; fp32 rows: tiny 3 + 20, the other 3 + 20 (small here)
     assert names.count("gdn2_chunk_fwd") == 7 + 7 + 23 + 23
     assert names.count("gdn2_layer_edge_maps") == 7 and names.count("gdn2_rms_norm") == 7
@@ -173,6 +179,9 @@ def test_next_rows_run_on_cpu_through_the_binding(rec, monkeypatch):
     assert bw["ms"] == ms and bw["tokens_per_s"] == pytest.approx(96 / (ms * 1e-3))
     assert bw["roofline"]["bound"] == "alu" and bw["roofline"]["flops_per_launch"] == bench.backward_flops(
         1, 96, 2, 128, 128)
+    bt = out["backward_tc"]
+    assert bt["ms"] == ms and bt["roofline"]["bound"] == "hbm" and bt["launches"] == 4
+    assert bt["roofline"]["algorithmic_bytes_per_launch"] == bench.backward_bytes(1, 96, 2, 128, 128)
     assert ed["ms"] == ms and ed["plain_prefill_ms"] == 0.5 and sp["ms"] == ms
     assert sp["roofline"]["algorithmic_bytes_per_launch"] == bench.prefill_bytes(1, 200, 2, 128, 128, s0=True)
     for row in (bw, ed, sp):
