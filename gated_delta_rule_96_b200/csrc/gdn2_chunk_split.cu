@@ -1012,19 +1012,21 @@ struct SplitPlan {
     int nw;     // chunks per window
     int nseg;   // segments per chain in a full window (1: plain walk)
 };
+// CTAs the segmented walks may use: one per SM of the B200 (148), so that every segment's walk runs at once.
+constexpr int kSegCtas = 148;
 SplitPlan split_plan(int B, int H, int T) {
     const int chains = B * H, NC = (T + split::C - 1) / split::C;
     int nw = chains > 0 ? std::max(64, 16384 / chains) : 64;
     nw = std::min(nw, std::max(NC, 1));
     int nseg = 1;
-    if (chains <= 64 && nw >= 32) nseg = std::max(1, std::min(128 / std::max(chains, 1), nw / 8));
+    if (chains <= 64 && nw >= 32) nseg = std::max(1, std::min(kSegCtas / std::max(chains, 1), nw / 8));
     return {nw, nseg};
 }
 constexpr size_t kStateBytes = sizeof(float) * 128 * 128;
 // segments per chain of the backward's forward replay (one window of the whole sequence)
 int replay_segments(int chains, int NC) {
     if (chains > 64 || NC < 32) return 1;
-    return std::max(1, std::min(128 / std::max(chains, 1), NC / 8));
+    return std::max(1, std::min(kSegCtas / std::max(chains, 1), NC / 8));
 }
 
 }  // namespace
