@@ -71,11 +71,11 @@ def test_workspace_bytes_tensor_core_path():
     # few long chains: the two-stage path over a window of up to 16,384 chunk-heads, each chain cut into
     # segments walked in parallel (three fp32 states per chain and segment)
     state = 4 * 128 * 128
-    # B1 H16 T65536: 1,024 chunks in one window, 8 segments of 128 chunks
+    # B1 H16 T65536: 1,024 chunks in one window, 148 // 16 = 9 segments (one walk per SM)
     assert g.gdn2_chunk_fwd_path(1, 16, 65536, 128, 128, 64, g.GDN2_BF16) == 2
     assert g.gdn2_chunk_fwd_workspace_bytes(1, 16, 65536, 128, 128, 64, g.GDN2_BF16) == \
-        256 + 16 * 1024 * rec + 3 * 16 * 8 * state
-    # B1 H2, 41 chunks: at most 64 segments by chains, at least 8 chunks each -> 5 segments of 9 chunks
+        256 + 16 * 1024 * rec + 3 * 16 * 9 * state
+    # B1 H2, 41 chunks: at most 74 segments by chains, at least 8 chunks each -> 5 segments of 9 chunks
     assert g.gdn2_chunk_fwd_workspace_bytes(1, 2, 64 * 40 + 37, 128, 128, 64, g.GDN2_BF16) == \
         256 + 2 * 41 * rec + 3 * 2 * 5 * state
     # up to 64 chains of fewer than 32 chunks: the fused kernel, status header only
