@@ -7,7 +7,7 @@
 // absorbed into the rank-1 factors, the Gram matrices, the triangular solve and the WY factors --
 // is independent from chunk to chunk; only the state update is a chain.  So:
 //
-//   stage 1, prep_kernel: fully parallel over every (batch, chunk, head), two CTAs per SM.  The
+//   stage 1, prep_kernel: fully parallel over every (batch, chunk, head), one persistent CTA per SM.  The
 //     token tiles arrive by TMA tensor copies straight into the swizzled operand layout; per
 //     chunk (g = per-channel log-decay prefix, m = its midpoint, e = b ⊙ k, u = w ⊙ v):
 //       build  Ê = e ⊙ exp(g - m), Q̂ = q ⊙ exp(g - m), K̃ = k ⊙ exp(m - g), U = u   (in place)
@@ -59,10 +59,13 @@ constexpr uint32_t STATUS_PREP = 2u, STATUS_WALK = 4u;
 //   warps 0-7   build group: alpha prefix, decay factors and the bf16 operands of chunk-head j+1,
 //               G1, then A (fp32, for the solve) and P (bf16, to the record) out of TMEM
 //   warps 8-11  solve group: T = (I + A)^-1, G2 and the W', Ũ rows of chunk-head j
-//   warp 12     producer: a two-stage ring of token tiles by TMA (alpha through one buffer)
-// The solve group stores each record by bulk copies (K̃ and Q̂ as soon as G1 has run, -W' and Ũ at the
-// end) and releases the stage once they have read it.
-constexpr int P1_NT = 416;
+// The token tiles pass through a two-stage ring filled by TMA, alpha through one buffer.  The thread
+// that frees a buffer refills it: the build group's first thread loads the next chunk-head's alpha as
+// soon as the prefix has read it, and the solve group's first thread loads the tiles of chunk-head j+2
+// into the stage of chunk-head j once the record's stores (K̃ and Q̂ as soon as G1 has run, -W' and Ũ at
+// the end) have read it.  Twelve warps, three on each of the SM's four register sub-partitions, leave
+// 168 registers per thread (a thirteenth, producer, warp would cut that to 128).
+constexpr int P1_NT = 384;
 constexpr uint32_t P1_STAGE = 81920;                 // per stage: EQ, KT, U, W tiles
 constexpr uint32_t P1_EQ = 0;                        // b -> Ê -> -W' (rows 0-63), q -> Q̂ (rows 64-127)
 constexpr uint32_t P1_KT = 32768;                    // k -> K̃
@@ -74,10 +77,10 @@ constexpr uint32_t P1_X = P1_AS + 64 * LDA * 4;      // solve group scratch (4 K
 constexpr uint32_t P1_WT = P1_X + 4096;              // build group: [8][128] log2 totals, then g_0 [128]
 constexpr uint32_t P1_MISC = P1_WT + 4608;
 constexpr uint32_t P1_BYTES = P1_MISC + 256 + 1024;  // + alignment slack
-// mbarriers: FULL and OUT per stage; alpha full / free; G1; A ready / A scratch free; G2
+// mbarriers: FULL per stage; alpha full; G1; A ready / A scratch free; G2
 enum : uint32_t {
-    M1_FULL = 0, M1_OUT = 16, M1_AFULL = 32, M1_AFREE = 40, M1_G1 = 48, M1_AREADY = 56, M1_ASFREE = 64,
-    M1_G2 = 72, M1_TSLOT = 96, M1_ABORT = 100
+    M1_FULL = 0, M1_AFULL = 32, M1_G1 = 48, M1_AREADY = 56, M1_ASFREE = 64, M1_G2 = 72, M1_TSLOT = 96,
+    M1_ABORT = 100, M1_LAST = 104   // M1_LAST: three ints, the last job loaded into stage 0, stage 1, alpha
 };
 constexpr uint32_t P1_TM_D1 = 0, P1_TM_D2 = 128, P1_TM_D3 = 256, P1_TM_COLS = 512;
 constexpr uint32_t BAR_A = 1, BAR_B = 2;   // named barriers: build group (256), solve group (128)
@@ -88,15 +91,6 @@ constexpr uint32_t ID_G3 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G4 = idesc_bf16(128, 128, 0, 1);
 constexpr uint32_t ID_G5 = idesc_bf16(128, 128, 1, 1);
 
-
-// Bounded wait of one thread (the producer); on expiry it sets the abort flag.
-__device__ __forceinline__ bool thread_wait1(uint32_t mb, uint32_t parity, volatile uint32_t *abort) {
-    if (!mbar_wait(mb, parity, WAIT_LIMIT) || *abort) {
-        *abort = 1u;
-        return false;
-    }
-    return true;
-}
 
 // Bounded wait of a warp group (named barrier `bar`, n threads): every thread gets the same verdict.
 __device__ __forceinline__ bool gwait(uint32_t mb, uint32_t parity, uint32_t bar, uint32_t n, volatile uint32_t *abort) {
@@ -195,12 +189,9 @@ __global__ void __launch_bounds__(P1_NT, 1)
 
     if (warp == 0) tmem_alloc(misc + M1_TSLOT, P1_TM_COLS);
     if (tid == 0) {
-        for (int st = 0; st < 2; ++st) {
-            mbar_init(misc + M1_FULL + 8 * st, 1);
-            mbar_init(misc + M1_OUT + 8 * st, 1);
-        }
+        for (int st = 0; st < 2; ++st) mbar_init(misc + M1_FULL + 8 * st, 1);
         mbar_init(misc + M1_AFULL, 1);
-        mbar_init(misc + M1_AFREE, 1);
+        for (int i = 0; i < 3; ++i) reinterpret_cast<volatile int *>(sm + P1_MISC + M1_LAST)[i] = -1;
         mbar_init(misc + M1_G1, 1);
         mbar_init(misc + M1_AREADY, 1);
         mbar_init(misc + M1_ASFREE, 1);
@@ -222,42 +213,45 @@ __global__ void __launch_bounds__(P1_NT, 1)
     auto rec_of = [&](int j) { return records + (size_t)(blockIdx.x + j * gridDim.x) * R_BYTES; };
     auto aux_of = [&](int j) { return aux + (size_t)(blockIdx.x + j * gridDim.x) * X_BYTES; };
 
-    if (warp == 12) {
-        // ------------------------------------------------------------------ producer (one thread)
-        if (lane == 0) {
-            prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b);
-            prefetch_tmap(&maps.v); prefetch_tmap(&maps.w); prefetch_tmap(&maps.alpha);
-            int last_tiles[2] = {-1, -1}, last_alpha = -1;
-            for (int j = 0; j < njobs; ++j) {
-                const int stg = j & 1;
-                int h, bb, n;
-                coords(blockIdx.x + j * gridDim.x, h, bb, n);
-                const int t0 = n * C;
-                // alpha into its single buffer once the previous job's prefix has read it
-                if (j >= 1 && !thread_wait1(misc + M1_AFREE, (uint32_t)((j - 1) & 1), abort)) break;
-                mbar_arrive_expect_tx(misc + M1_AFULL, 32768u);
-                tma_load_4d(smem_u32(sm + P1_A), &maps.alpha, 0, h, t0, bb, misc + M1_AFULL);
-                last_alpha = j;
-                // the token tiles once the stage's previous job is finished and its record stores have read it
-                if (j >= 2 && !thread_wait1(misc + M1_OUT + 8 * stg, (uint32_t)(((j - 2) >> 1) & 1), abort)) break;
-                const uint32_t st = smem_u32(sm + stg * P1_STAGE), fb = misc + M1_FULL + 8 * stg;
-                mbar_arrive_expect_tx(fb, 10u * 8192u);
+    // loads of chunk-head job j: alpha into its buffer; the token tiles into stage j & 1
+    auto load_alpha = [&](int j) {
+        int h, bb, n;
+        coords(blockIdx.x + j * gridDim.x, h, bb, n);
+        mbar_arrive_expect_tx(misc + M1_AFULL, 32768u);
+        tma_load_4d(smem_u32(sm + P1_A), &maps.alpha, 0, h, n * C, bb, misc + M1_AFULL);
+    };
+    auto load_tiles = [&](int j) {
+        int h, bb, n;
+        coords(blockIdx.x + j * gridDim.x, h, bb, n);
+        const int t0 = n * C, stg = j & 1;
+        const uint32_t st = smem_u32(sm + stg * P1_STAGE), fb = misc + M1_FULL + 8 * stg;
+        mbar_arrive_expect_tx(fb, 10u * 8192u);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    tma_load_4d(st + P1_EQ + hf * 16384, &maps.b, 64 * hf, h, t0, bb, fb);
-                    tma_load_4d(st + P1_EQ + hf * 16384 + 8192, &maps.q, 64 * hf, h, t0, bb, fb);
-                    tma_load_4d(st + P1_KT + hf * 8192, &maps.k, 64 * hf, h, t0, bb, fb);
-                    tma_load_4d(st + P1_U + hf * 8192, &maps.v, 64 * hf, h, t0, bb, fb);
-                    tma_load_4d(st + P1_W + hf * 8192, &maps.w, 64 * hf, h, t0, bb, fb);
-                }
-                last_tiles[stg] = j;
-            }
-            // no tile load may be left in flight when the block exits (after an abort)
-            for (int stg = 0; stg < 2; ++stg)
-                if (last_tiles[stg] >= 0) mbar_wait(misc + M1_FULL + 8 * stg, (uint32_t)((last_tiles[stg] >> 1) & 1), WAIT_LIMIT);
-            if (last_alpha >= 0) mbar_wait(misc + M1_AFULL, (uint32_t)(last_alpha & 1), WAIT_LIMIT);
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(st + P1_EQ + hf * 16384, &maps.b, 64 * hf, h, t0, bb, fb);
+            tma_load_4d(st + P1_EQ + hf * 16384 + 8192, &maps.q, 64 * hf, h, t0, bb, fb);
+            tma_load_4d(st + P1_KT + hf * 8192, &maps.k, 64 * hf, h, t0, bb, fb);
+            tma_load_4d(st + P1_U + hf * 8192, &maps.v, 64 * hf, h, t0, bb, fb);
+            tma_load_4d(st + P1_W + hf * 8192, &maps.w, 64 * hf, h, t0, bb, fb);
         }
-    } else if (warp < 8) {
+    };
+    // the last job each buffer was loaded for, whichever thread loaded it (for the exit: no copy may be
+    // left in flight): stage 0, stage 1, alpha
+    volatile int *last_ld = reinterpret_cast<volatile int *>(sm + P1_MISC + M1_LAST);
+    if (tid == 0) {
+        prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b);
+        prefetch_tmap(&maps.v); prefetch_tmap(&maps.w); prefetch_tmap(&maps.alpha);
+        for (int j = 0; j < 2 && j < njobs; ++j) {
+            load_tiles(j);
+            last_ld[j] = j;
+        }
+        if (njobs > 0) {
+            load_alpha(0);
+            last_ld[2] = 0;
+        }
+    }
+
+    if (warp < 8) {
         // ------------------------------------------------------------------ build group
         float *WT = reinterpret_cast<float *>(sm + P1_WT);
         float *v_g0 = WT + 8 * 128;
@@ -306,7 +300,10 @@ __global__ void __launch_bounds__(P1_NT, 1)
                 *reinterpret_cast<float4 *>(v_g0 + c4) =
                     make_float4(fast_log2(al[0][0]), fast_log2(al[0][1]), fast_log2(al[0][2]), fast_log2(al[0][3]));
             group_sync(BAR_A, 256);
-            if (tid == 0) mbar_arrive(misc + M1_AFREE);   // the alpha buffer has been read
+            if (tid == 0 && j + 1 < njobs) {   // the alpha buffer has been read: the next chunk-head's in
+                load_alpha(j + 1);
+                last_ld[2] = j + 1;
+            }
             float pre[4] = {0.f, 0.f, 0.f, 0.f}, gC[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int w2 = 0; w2 < 8; ++w2) {
@@ -635,7 +632,10 @@ __global__ void __launch_bounds__(P1_NT, 1)
                 bulk_s2g(rec + R_U, aU, 16384);
                 bulk_commit();
                 bulk_wait_read_all();
-                mbar_arrive(misc + M1_OUT + 8 * stg);
+                if (j + 2 < njobs) {   // the stage is free: chunk-head j+2's tiles in
+                    load_tiles(j + 2);
+                    last_ld[stg] = j + 2;
+                }
             }
         }
         if (tb == 0) {   // the record stores complete before the block exits
@@ -646,7 +646,13 @@ __global__ void __launch_bounds__(P1_NT, 1)
     fence_before();
     __syncthreads();
     fence_after();
-    if (tid == 0 && *abort) atomicOr(status, STATUS_PREP);
+    if (tid == 0) {   // no tile or alpha load may be left in flight when the block exits (after an abort)
+        for (int stg = 0; stg < 2; ++stg)
+            if (last_ld[stg] >= 0) mbar_wait(misc + M1_FULL + 8 * stg, (uint32_t)((last_ld[stg] >> 1) & 1), WAIT_LIMIT);
+        if (last_ld[2] >= 0) mbar_wait(misc + M1_AFULL, (uint32_t)(last_ld[2] & 1), WAIT_LIMIT);
+        if (*abort) atomicOr(status, STATUS_PREP);
+    }
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, P1_TM_COLS);
 }
 
