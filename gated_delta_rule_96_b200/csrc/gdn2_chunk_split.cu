@@ -951,11 +951,25 @@ __global__ void __launch_bounds__(W2_NT, 1)
         if (!is_delta && ot == 0) bulk_wait_all();   // the o stores complete before the block exits
         if (aux && tid == 0) bulk_wait_all();
     } else if (lane == 0) {
-        // ------------------------------------------------------------------ producer: one bulk copy per record
+        // ------------------------------------------------------------------ producer: bulk copies per record
+        // A walk that stores no o reads only -W' (rows 0-63 of both column halves of the G3 tile), K̃, Ũ
+        // (not when the writes are off) and the factors: Q̂ and P feed only the o rows of D3, which it never
+        // reads, so their products run on whatever the slot held before.
+        const uint32_t part_ku = zero_writes ? 16384u : 32768u;
+        const uint32_t bytes = store_out ? R_COPY : 2 * 8192u + part_ku + 3 * 128 * 4;
         for (int nl = 0; nl < nc; ++nl) {
             if (nl >= 2 && !thread_wait(misc + M2_G45 + 8 * (nl & 1), (uint32_t)(((nl - 2) >> 1) & 1), abort)) break;
-            mbar_arrive_expect_tx(misc + M2_FULL + 8 * (nl & 1), R_COPY);
-            bulk_g2s(smem_u32(sm + slot_addr(nl)), rec_of(nl), R_COPY, misc + M2_FULL + 8 * (nl & 1));
+            const uint32_t full = misc + M2_FULL + 8 * (nl & 1), dst = smem_u32(sm + slot_addr(nl));
+            const unsigned char *src = rec_of(nl);
+            mbar_arrive_expect_tx(full, bytes);
+            if (store_out) {
+                bulk_g2s(dst, src, R_COPY, full);
+            } else {
+                bulk_g2s(dst + R_A3, src + R_A3, 8192, full);
+                bulk_g2s(dst + R_A3 + 16384, src + R_A3 + 16384, 8192, full);
+                bulk_g2s(dst + R_KT, src + R_KT, part_ku, full);   // K̃, and Ũ right after it
+                bulk_g2s(dst + R_VEC, src + R_VEC, 3 * 128 * 4, full);
+            }
         }
     }
     fence_before();

@@ -1027,12 +1027,15 @@ __global__ void __launch_bounds__(NT, 1)
 // ============================================================================ segment scan
 // S_g = M_(g-1) S_(g-1) + N_(g-1) along the segments of each chain (g = 1 .. nseg-1), S_0 = S0.
 // One block per (chain, 16-column slice of S); fp32.  Each step stages M_(g-1) (64 KB) in shared
-// memory with coalesced loads; thread (r0, col) keeps rows r0, r0 + 16, ..., r0 + 112 of its column.
-constexpr int SCAN_SMEM = (KD * KD + KD * 16) * 4;   // M, then the previous state's column slice
+// memory, rows padded to SCAN_LD floats so that the two rows a warp reads fall in different banks;
+// the next step's M is loaded into registers while this step computes.  Thread (r0, col) keeps rows
+// r0, r0 + 16, ..., r0 + 112 of its column and reads M four k at a time.
+constexpr int SCAN_LD = KD + 4;
+constexpr int SCAN_SMEM = (KD * SCAN_LD + KD * 16) * 4;   // M, then the previous state's column slice
 __global__ void __launch_bounds__(256) segment_scan_kernel(const float *__restrict__ M, const float *__restrict__ N,
                                                            const float *S0, float *__restrict__ Sg, int nseg) {
     extern __shared__ float scan_sm[];
-    float *Ms = scan_sm, *sprev = scan_sm + KD * KD;   // Ms [KD][KD], sprev [KD][16]
+    float *Ms = scan_sm, *sprev = scan_sm + KD * SCAN_LD;   // Ms [KD][SCAN_LD], sprev [KD][16]
     const int chain = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
     const size_t KV = (size_t)KD * VD;
     const int col = tid & 15, r0 = tid >> 4;   // rows r0, r0 + 16, ..., r0 + 112
@@ -1041,20 +1044,39 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(const float *__restri
         sprev[r * 16 + col] = v;
         Sg[((size_t)chain * nseg) * KV + (size_t)r * VD + c0 + col] = v;
     }
+    constexpr int NV = KD * KD / 4 / 256;   // float4 of M per thread
+    float4 mreg[NV];
+    auto load_m = [&](int g) {
+        const float4 *Mg = reinterpret_cast<const float4 *>(M + ((size_t)chain * nseg + g - 1) * KV);
+#pragma unroll
+        for (int u = 0; u < NV; ++u) mreg[u] = __ldg(Mg + tid + 256 * u);
+    };
+    if (nseg > 1) load_m(1);
     for (int g = 1; g < nseg; ++g) {
-        const float *Mg = M + ((size_t)chain * nseg + g - 1) * KV, *Ng = N + ((size_t)chain * nseg + g - 1) * KV;
+        const float *Ng = N + ((size_t)chain * nseg + g - 1) * KV;
         __syncthreads();   // the previous step's reads of Ms are done
-        for (int i = tid; i < KD * KD / 4; i += 256)
-            reinterpret_cast<float4 *>(Ms)[i] = __ldg(reinterpret_cast<const float4 *>(Mg) + i);
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int i = tid + 256 * u;   // float4 i of M: row i / 32, columns 4 (i % 32) ..
+            *reinterpret_cast<float4 *>(Ms + (i >> 5) * SCAN_LD + 4 * (i & 31)) = mreg[u];
+        }
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = Ng[(size_t)(r0 + 16 * i) * VD + c0 + col];
         __syncthreads();
-#pragma unroll 4
-        for (int kk = 0; kk < KD; ++kk) {
-            const float sv = sprev[kk * 16 + col];
+        if (g + 1 < nseg) load_m(g + 1);
+#pragma unroll 2
+        for (int kk = 0; kk < KD; kk += 4) {
+            const float s0 = sprev[kk * 16 + col], s1 = sprev[(kk + 1) * 16 + col], s2 = sprev[(kk + 2) * 16 + col],
+                        s3 = sprev[(kk + 3) * 16 + col];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(Ms[(r0 + 16 * i) * KD + kk], sv, acc[i]);
+            for (int i = 0; i < 8; ++i) {
+                const float4 m = *reinterpret_cast<const float4 *>(Ms + (r0 + 16 * i) * SCAN_LD + kk);
+                acc[i] = fmaf(m.x, s0, acc[i]);
+                acc[i] = fmaf(m.y, s1, acc[i]);
+                acc[i] = fmaf(m.z, s2, acc[i]);
+                acc[i] = fmaf(m.w, s3, acc[i]);
+            }
         }
         __syncthreads();   // every thread has read sprev
 #pragma unroll

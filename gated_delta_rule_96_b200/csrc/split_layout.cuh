@@ -25,6 +25,8 @@ constexpr uint32_t R_P = 65536;     // P [r x i]: 64 x 64, lower with the diagon
 constexpr uint32_t R_VEC = 73728;   // sS, sZ, sPost: 3 x 128 fp32
 constexpr uint32_t R_COPY = R_VEC + 3 * 128 * 4;   // bytes moved per record
 constexpr uint32_t R_BYTES = 75776;                // record stride (1024-aligned)
+// a walk that stores no o copies K̃ and Ũ as one range
+static_assert(R_U == R_KT + 16384 && R_COPY <= R_BYTES, "record layout");
 
 // ---------------------------------------------------------------------------- backward side record
 // Written by the forward replay (first stage: Ê, T and the frame exponents; second stage: Z̃, Delta)
